@@ -1,0 +1,179 @@
+/*
+ * yoco.h -- C ABI of libyoco.so, the B200 (sm_100a) attention core of the
+ * YOCO / YOCO++ decoder-decoder architecture.
+ *
+ * The method (sources by page title and section):
+ *  - "You Only Cache Once: Decoder-Decoder Architectures for Language Models"
+ *    (paperlayer summary of arXiv 2405.05254v2), section 2 "You Only Cache
+ *    Once": a self-decoder produces one global KV cache that every
+ *    cross-decoder layer reuses through cross-attention; section 3 "Design
+ *    Choices of Self-Decoder", "Sliding-Window Attention": the self-decoder
+ *    attends within a fixed window, so its cache is bounded.
+ *  - "YOCO: Caching Once for Decoder-Decoder Long-Context Language Models"
+ *    (podcast transcript), cue 12: the self-decoder output is normalised once
+ *    and projected by one pair of matrices into the shared K and V; each
+ *    cross-decoder layer has its own query projection and attends causally,
+ *    with grouped-query heads; cue 26: every cross layer streams the whole
+ *    shared KV at each decode step.
+ *  - "YOCO++: Enhancing YOCO with KV Residual Connections for Efficient LLM
+ *    Inference", Abstract: each bottom-half layer's KV gets a weighted
+ *    residual connection to the bottom layer's KV.
+ *
+ * Conventions shared by every call
+ *  - Layouts are token-major and dense: Q and O are [B, T, Hq, D], K and V
+ *    are [B, T, Hkv, D] (or packed [rows, Hkv, D] for the shared decode
+ *    cache).  Query head h reads KV head h / (Hq / Hkv).
+ *  - Element type is cfg->dtype (bf16 or fp32) for every Q/K/V/O/x/W buffer;
+ *    softmax and accumulation are fp32.  lse outputs are fp32, natural log.
+ *  - Every pointer is a DEVICE pointer unless stated; the caller owns every
+ *    buffer.  The library allocates no device memory; scratch comes from the
+ *    caller's workspace argument.
+ *  - Every data pointer must be 16-byte aligned.
+ *  - Calls are asynchronous on the caller's stream and never synchronise the
+ *    host.  Arguments are validated before anything is launched; on
+ *    YOCO_ERR_INVALID / YOCO_ERR_UNSUPPORTED / YOCO_ERR_WORKSPACE nothing was
+ *    launched and no buffer was touched.  YOCO_ERR_CUDA reports a launch
+ *    error.  Device-side bounded waits that give up set a device status word
+ *    that yoco_get_device_status() reports.
+ *  - Masks: a query at absolute position p sees key position j when j <= p
+ *    (causal, section 1 "Architecture": both halves use causal masking) and,
+ *    for sliding-window calls, also j > p - window (the window counts the
+ *    query's own position).
+ */
+#ifndef YOCO_H_
+#define YOCO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    YOCO_OK = 0,
+    YOCO_ERR_INVALID = 1,      /* bad argument (null, misaligned, bad shape) */
+    YOCO_ERR_UNSUPPORTED = 2,  /* valid but not built (head_dim, group size) */
+    YOCO_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
+    YOCO_ERR_WORKSPACE = 4,    /* workspace missing or too small */
+    YOCO_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
+} yoco_status;
+
+typedef enum { YOCO_BF16 = 0, YOCO_FP32 = 1 } yoco_dtype;
+
+/* Attention shape: Hq query heads, Hkv KV heads (Hq % Hkv == 0, group
+ * Hq/Hkv in {1, 2, 4, 8}, Hkv <= 32), head dim D in {64, 128}.
+ * scale 0 means 1/sqrt(D). */
+typedef struct {
+    int32_t Hq;
+    int32_t Hkv;
+    int32_t D;
+    float scale;
+    int32_t dtype; /* yoco_dtype */
+} yoco_attn_cfg;
+
+/* K/V producer with the YOCO++ weighted residual fused into its epilogue.
+ * Podcast cue 12 (normalise once, project by one pair of matrices) and the
+ * YOCO++ Abstract (KV of a bottom-half layer plus a weight times the bottom
+ * layer's KV).
+ *   [K | V] = N(x) . W_kv^T;  K += w_k * k_base;  V += w_v * v_base
+ * x       [n_tok, d_model]
+ * w_kv    [2*Hkv*D, d_model] row-major (one output feature per row; rows
+ *         0 .. Hkv*D-1 produce K, the rest produce V)
+ * apply_ln  nonzero: N = LayerNorm without affine (biased variance, ln_eps);
+ *           zero: N = identity
+ * k_base, v_base  [n_tok, Hkv, D] or NULL (no blend for that tensor)
+ * dst_rows  NULL: token t is written to output row t.  Otherwise a device
+ *           int64 [n_tok]: token t is written to row dst_rows[t] of k_out /
+ *           v_out (appending to the shared cache); rows must be distinct and
+ *           inside the caller's buffers.
+ * k_out, v_out  [rows, Hkv, D]
+ * With w = 0 (or NULL bases) this is the plain global-KV projection. */
+yoco_status yoco_kv_project_blend(const void *x, int64_t n_tok, int32_t d_model,
+                                  const void *w_kv, int32_t apply_ln, float ln_eps,
+                                  const void *k_base, const void *v_base, float w_k, float w_v,
+                                  const int64_t *dst_rows, void *k_out, void *v_out,
+                                  const yoco_attn_cfg *cfg, cudaStream_t stream);
+
+/* Self-decoder sliding-window attention over a prompt, then the ring fill.
+ * Section 3 "Sliding-Window Attention".
+ * q [B, T, Hq, D]; k, v [B, T, Hkv, D]; o [B, T, Hq, D]; lse [B, Hq, T] or NULL.
+ * Query row i sees keys j with i - window < j <= i.
+ * ring_k, ring_v [B, window, Hkv, D] and slot_pos int32 [B, window]: all three
+ * NULL (no ring) or all set.  After the call slot s holds the newest position
+ * p < T with p mod window == s, and slot_pos = p, or -1 (and zero K/V) when no
+ * such position exists. */
+yoco_status yoco_swa_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t T,
+                             int32_t window, void *o, float *lse, void *ring_k, void *ring_v,
+                             int32_t *slot_pos, const yoco_attn_cfg *cfg, cudaStream_t stream);
+
+/* Self-decoder sliding-window decode step over the ring.
+ * q [B, Hq, D]; k_new, v_new [B, Hkv, D] (already blended); pos device int64
+ * [B]: absolute position of the new token of each sequence.  The new K/V is
+ * written to slot pos mod window (slot_pos updated), then the query attends
+ * to every slot whose stored position lies in (pos - window, pos].
+ * o [B, Hq, D].  workspace: yoco_swa_decode_workspace_size() bytes. */
+yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
+                            const int64_t *pos, int32_t B, int32_t window, void *ring_k,
+                            void *ring_v, int32_t *slot_pos, void *o, void *workspace,
+                            size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream);
+
+/* Cross-decoder causal prefill over the one shared KV.  Section 2 and
+ * podcast cue 12: every cross layer has its own Q and attends causally to the
+ * same K_g, V_g.
+ * q [B, Tq, Hq, D]; k, v [B, Tkv, Hkv, D]; o [B, Tq, Hq, D]; lse [B, Hq, Tq] or
+ * NULL.  Query row i sits at absolute position q_pos0 + i (chunked prefill);
+ * requires 0 <= q_pos0 and q_pos0 + Tq <= Tkv. */
+yoco_status yoco_cross_prefill(const void *q, const void *k, const void *v, int32_t B,
+                               int64_t Tq, int64_t Tkv, int64_t q_pos0, void *o, float *lse,
+                               const yoco_attn_cfg *cfg, cudaStream_t stream);
+
+/* Cross-decoder decode step: one new query token per sequence reads the whole
+ * shared cache (podcast cue 26), split across the GPU and merged.
+ * q [B, Hq, D]; k_cache, v_cache packed [rows, Hkv, D]; sequence b owns rows
+ * [seq_start[b], seq_start[b] + seq_len[b]) (device int64 / int32 arrays,
+ * seq_len >= 1 and including the new token's row).  max_len >= every
+ * seq_len (host value; sizes the split plan without a device read).
+ * o [B, Hq, D]; lse [B, Hq] or NULL.
+ * workspace: device scratch of yoco_cross_decode_workspace_size() bytes. */
+yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_cache,
+                              const int64_t *seq_start, const int32_t *seq_len, int32_t B,
+                              int64_t max_len, void *o, float *lse, void *workspace,
+                              size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream);
+
+/* Workspace bytes for yoco_cross_decode / yoco_swa_decode (0 on bad args). */
+size_t yoco_cross_decode_workspace_size(int32_t B, int64_t max_len, const yoco_attn_cfg *cfg);
+size_t yoco_swa_decode_workspace_size(int32_t B, int32_t window, const yoco_attn_cfg *cfg);
+
+/* Auxiliary dense projection used around the attention core (query and
+ * output projections of the small end-to-end stack):
+ *   out = N(x) . W^T + base_w * base
+ * x [n, d_in]; w [d_out, d_in]; base [n, d_out] or NULL; out [n, d_out];
+ * dtype is a yoco_dtype. */
+yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, int32_t d_out,
+                        int32_t apply_ln, float ln_eps, const void *base, float base_w,
+                        void *out, int32_t dtype, cudaStream_t stream);
+
+/* KV-cache bytes of one sequence of N tokens (section 2: O(N + C L) for YOCO
+ * versus N x L for a Transformer): one global K/V of N rows plus, per
+ * self-decoder layer, a ring of min(window, N) rows.  Host only. */
+double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_attn_cfg *cfg);
+
+/* Synchronises the stream, then returns and clears the device status word:
+ * YOCO_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call,
+ * YOCO_ERR_CUDA if the stream reports an error, else YOCO_OK. */
+yoco_status yoco_get_device_status(cudaStream_t stream);
+
+/* Static description of a status code. */
+const char *yoco_status_string(yoco_status s);
+
+/* Library version string. */
+const char *yoco_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* YOCO_H_ */

@@ -1,0 +1,237 @@
+"""Python binding of libyoco.so, the B200 (sm_100a) attention core of the
+YOCO / YOCO++ decoder-decoder architecture.
+
+Argument marshalling only: every function passes torch CUDA tensors as raw
+device pointers, plus the current CUDA stream, to the C ABI declared in
+include/yoco.h, and raises YocoError on a non-OK status.  Every computation
+runs in the library's CUDA kernels; there is no CPU or PyTorch fallback, and
+importing a function fails loudly when libyoco.so is missing.
+
+Entry points (same names as the C ABI, without the ``yoco_`` prefix):
+kv_project_blend, swa_prefill, swa_decode, cross_prefill, cross_decode,
+plus linear, workspace sizes, cache_bytes and device_status.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_prefill",
+           "swa_decode", "cross_prefill", "cross_decode", "cross_decode_workspace_size",
+           "swa_decode_workspace_size", "cache_bytes", "device_status", "AttnCfg"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT = range(6)
+BF16, FP32 = 0, 1
+_DT = {torch.bfloat16: BF16, torch.float32: FP32}
+
+
+class YocoError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = _LIB.yoco_status_string(status).decode() if _LIB is not None else str(status)
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+class AttnCfg(ctypes.Structure):
+    _fields_ = [("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+def lib_path():
+    return os.path.join(_HERE, "libyoco.so")
+
+
+def load():
+    """Load libyoco.so (built in-tree by shared_kv_decoder_b200.build)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"libyoco.so not found at {path}; build it with "
+                           "`python -m shared_kv_decoder_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+    cfgp = ctypes.POINTER(AttnCfg)
+    st = ctypes.c_int
+    sigs = {
+        "yoco_kv_project_blend": (st, [vp, i64, i32, vp, i32, f32, vp, vp, f32, f32, vp, vp, vp,
+                                       cfgp, vp]),
+        "yoco_linear": (st, [vp, i64, i32, vp, i32, i32, f32, vp, f32, vp, i32, vp]),
+        "yoco_swa_prefill": (st, [vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, cfgp, vp]),
+        "yoco_swa_decode": (st, [vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_cross_prefill": (st, [vp, vp, vp, i32, i64, i64, i64, vp, vp, cfgp, vp]),
+        "yoco_cross_decode": (st, [vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_cross_decode_workspace_size": (sz, [i32, i64, cfgp]),
+        "yoco_swa_decode_workspace_size": (sz, [i32, i32, cfgp]),
+        "yoco_cache_bytes": (ctypes.c_double, [i32, i32, i64, cfgp]),
+        "yoco_get_device_status": (st, [vp]),
+        "yoco_status_string": (ctypes.c_char_p, [st]),
+        "yoco_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = L
+    return L
+
+
+def _check(status, where):
+    if status != OK:
+        raise YocoError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("libyoco takes CUDA tensors only")
+            if not t.is_contiguous():
+                raise ValueError("libyoco takes contiguous tensors only")
+
+
+def _cfg(Hq, Hkv, D, dtype, scale=0.0):
+    return AttnCfg(int(Hq), int(Hkv), int(D), float(scale), _DT[dtype])
+
+
+def kv_project_blend(x, w_kv, Hkv, D, k_base=None, v_base=None, w_k=0.0, w_v=0.0,
+                     dst_rows=None, k_out=None, v_out=None, apply_ln=True, eps=1e-5):
+    """[K | V] = LN(x) W_kv^T (+ w_k K_base, + w_v V_base), fused epilogue.
+    x [n, d]; w_kv [2*Hkv*D, d]; bases [n, Hkv, D]; returns (k_out, v_out)."""
+    L = load()
+    n, d = x.shape
+    if k_out is None:
+        k_out = torch.empty((n, Hkv, D), dtype=x.dtype, device=x.device)
+    if v_out is None:
+        v_out = torch.empty((n, Hkv, D), dtype=x.dtype, device=x.device)
+    _dev(x, w_kv, k_base, v_base, dst_rows, k_out, v_out)
+    cfg = _cfg(Hkv, Hkv, D, x.dtype)
+    _check(L.yoco_kv_project_blend(_ptr(x), n, d, _ptr(w_kv), int(bool(apply_ln)), eps,
+                                   _ptr(k_base), _ptr(v_base), float(w_k), float(w_v),
+                                   _ptr(dst_rows), _ptr(k_out), _ptr(v_out), ctypes.byref(cfg),
+                                   _stream()), "yoco_kv_project_blend")
+    return k_out, v_out
+
+
+def linear(x, w, base=None, base_w=1.0, apply_ln=False, eps=1e-5, out=None):
+    """out = N(x) W^T + base_w * base.  x [n, d_in]; w [d_out, d_in]."""
+    L = load()
+    n, d_in = x.shape
+    d_out = w.shape[0]
+    if out is None:
+        out = torch.empty((n, d_out), dtype=x.dtype, device=x.device)
+    _dev(x, w, base, out)
+    _check(L.yoco_linear(_ptr(x), n, d_in, _ptr(w), d_out, int(bool(apply_ln)), eps, _ptr(base),
+                         float(base_w), _ptr(out), _DT[x.dtype], _stream()), "yoco_linear")
+    return out
+
+
+def swa_prefill(q, k, v, window, ring=None, want_lse=False, scale=0.0, o=None):
+    """Sliding-window prefill.  q [B, T, Hq, D]; k, v [B, T, Hkv, D].
+    ring: None, or a tuple (ring_k, ring_v, slot_pos) to fill.
+    Returns o (and lse [B, Hq, T] when want_lse)."""
+    L = load()
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device) if want_lse else None
+    rk, rv, sp = ring if ring is not None else (None, None, None)
+    _dev(q, k, v, o, lse, rk, rv, sp)
+    cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
+    _check(L.yoco_swa_prefill(_ptr(q), _ptr(k), _ptr(v), B, T, int(window), _ptr(o), _ptr(lse),
+                              _ptr(rk), _ptr(rv), _ptr(sp), ctypes.byref(cfg), _stream()),
+           "yoco_swa_prefill")
+    return (o, lse) if want_lse else o
+
+
+def swa_decode_workspace_size(B, window, Hq, Hkv, D, dtype):
+    cfg = _cfg(Hq, Hkv, D, dtype)
+    return int(load().yoco_swa_decode_workspace_size(B, window, ctypes.byref(cfg)))
+
+
+def swa_decode(q, k_new, v_new, pos, ring_k, ring_v, slot_pos, window, workspace=None,
+               scale=0.0, o=None):
+    """One sliding-window decode step.  q [B, Hq, D]; k_new, v_new [B, Hkv, D];
+    pos int64 [B]; ring_k, ring_v [B, window, Hkv, D]; slot_pos int32 [B, window]."""
+    L = load()
+    B, Hq, D = q.shape
+    Hkv = k_new.shape[1]
+    if workspace is None:
+        workspace = torch.empty(swa_decode_workspace_size(B, window, Hq, Hkv, D, q.dtype),
+                                dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    _dev(q, k_new, v_new, pos, ring_k, ring_v, slot_pos, o, workspace)
+    cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
+    _check(L.yoco_swa_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(pos), B, int(window),
+                             _ptr(ring_k), _ptr(ring_v), _ptr(slot_pos), _ptr(o), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), ctypes.byref(cfg),
+                             _stream()), "yoco_swa_decode")
+    return o
+
+
+def cross_prefill(q, k, v, q_pos0=0, want_lse=False, scale=0.0, o=None):
+    """Causal cross-attention over the shared KV.  q [B, Tq, Hq, D];
+    k, v [B, Tkv, Hkv, D]; query row i at absolute position q_pos0 + i."""
+    L = load()
+    B, Tq, Hq, D = q.shape
+    Tkv, Hkv = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if want_lse else None
+    _dev(q, k, v, o, lse)
+    cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
+    _check(L.yoco_cross_prefill(_ptr(q), _ptr(k), _ptr(v), B, Tq, Tkv, int(q_pos0), _ptr(o),
+                                _ptr(lse), ctypes.byref(cfg), _stream()), "yoco_cross_prefill")
+    return (o, lse) if want_lse else o
+
+
+def cross_decode_workspace_size(B, max_len, Hq, Hkv, D, dtype):
+    cfg = _cfg(Hq, Hkv, D, dtype)
+    return int(load().yoco_cross_decode_workspace_size(B, max_len, ctypes.byref(cfg)))
+
+
+def cross_decode(q, k_cache, v_cache, seq_start, seq_len, max_len, workspace=None,
+                 want_lse=False, scale=0.0, o=None):
+    """One cross-decoder decode step over the packed shared cache.
+    q [B, Hq, D]; caches [rows, Hkv, D]; seq_start int64 [B]; seq_len int32 [B]."""
+    L = load()
+    B, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    if workspace is None:
+        workspace = torch.empty(cross_decode_workspace_size(B, max_len, Hq, Hkv, D, q.dtype),
+                                dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if want_lse else None
+    _dev(q, k_cache, v_cache, seq_start, seq_len, o, lse, workspace)
+    cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
+    _check(L.yoco_cross_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_start),
+                               _ptr(seq_len), B, int(max_len), _ptr(o), _ptr(lse),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               ctypes.byref(cfg), _stream()), "yoco_cross_decode")
+    return (o, lse) if want_lse else o
+
+
+def cache_bytes(L_self, window, N, Hkv, D, dtype=torch.bfloat16):
+    cfg = _cfg(Hkv, Hkv, D, dtype)
+    return float(load().yoco_cache_bytes(L_self, window, N, ctypes.byref(cfg)))
+
+
+def device_status():
+    """Synchronise the current stream and return the device status code."""
+    return int(load().yoco_get_device_status(_stream()))

@@ -1,0 +1,226 @@
+// C ABI of libyoco.so (declared in include/yoco.h): argument validation and
+// dispatch to the sm_100a kernels.  Nothing is launched unless every check
+// passes; the library never allocates device memory and never synchronises
+// the host on a hot call.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/yoco.h"
+#include "launch.h"
+
+using namespace yoco;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void *p) { return p == nullptr || aligned16(p); }
+
+yoco_status check_cfg(const yoco_attn_cfg *cfg) {
+    if (!cfg) return YOCO_ERR_INVALID;
+    if (cfg->Hq < 1 || cfg->Hkv < 1 || cfg->Hq % cfg->Hkv != 0) return YOCO_ERR_INVALID;
+    if (cfg->dtype != YOCO_BF16 && cfg->dtype != YOCO_FP32) return YOCO_ERR_INVALID;
+    if (!(cfg->scale >= 0.f) || isinf(cfg->scale)) return YOCO_ERR_INVALID;
+    if (cfg->D != 64 && cfg->D != 128) return YOCO_ERR_UNSUPPORTED;
+    const int G = cfg->Hq / cfg->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return YOCO_ERR_UNSUPPORTED;
+    return YOCO_OK;
+}
+
+float eff_scale(const yoco_attn_cfg *cfg) {
+    return cfg->scale > 0.f ? cfg->scale : 1.0f / sqrtf((float)cfg->D);
+}
+
+yoco_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return YOCO_OK;
+    if (e == cudaErrorNotSupported) return YOCO_ERR_UNSUPPORTED;
+    return YOCO_ERR_CUDA;
+}
+
+// Attention prefill dispatch: bf16 goes to the tcgen05 kernel; fp32 (and any
+// bf16 shape that kernel was not built for) to the CUDA-core kernel.
+yoco_status run_prefill(const PrefillArgs &a, cudaStream_t s) {
+    if (a.dtype == kBF16) {
+        const cudaError_t e = launch_prefill_tc(a, s);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();
+    }
+    return from_cuda(launch_prefill_simt(a, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *yoco_version(void) { return "yoco-b200 0.1 (sm_100a)"; }
+
+const char *yoco_status_string(yoco_status s) {
+    switch (s) {
+        case YOCO_OK: return "ok";
+        case YOCO_ERR_INVALID: return "invalid argument";
+        case YOCO_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case YOCO_ERR_CUDA: return "CUDA error";
+        case YOCO_ERR_WORKSPACE: return "workspace missing or too small";
+        case YOCO_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+yoco_status yoco_kv_project_blend(const void *x, int64_t n_tok, int32_t d_model, const void *w_kv,
+                                  int32_t apply_ln, float ln_eps, const void *k_base,
+                                  const void *v_base, float w_k, float w_v,
+                                  const int64_t *dst_rows, void *k_out, void *v_out,
+                                  const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (n_tok < 0 || d_model < 1 || !(ln_eps > 0.f) || !isfinite(w_k) || !isfinite(w_v))
+        return YOCO_ERR_INVALID;
+    if (n_tok == 0) return YOCO_OK;
+    if (!ok_ptr(x) || !ok_ptr(w_kv) || !ok_ptr(k_out) || !ok_ptr(v_out) || !ok_opt(k_base) ||
+        !ok_opt(v_base) || !ok_opt(dst_rows))
+        return YOCO_ERR_INVALID;
+    if ((int64_t)d_model * dtype_bytes(cfg->dtype) % 16 != 0) return YOCO_ERR_INVALID;
+    LinearArgs a;
+    a.x = x; a.w = w_kv; a.n = n_tok; a.d_in = d_model;
+    a.d_out = 2 * cfg->Hkv * cfg->D; a.split_col = cfg->Hkv * cfg->D;
+    a.apply_ln = apply_ln ? 1 : 0; a.eps = ln_eps;
+    a.out0 = k_out; a.out1 = v_out; a.base0 = k_base; a.base1 = v_base;
+    a.w0 = w_k; a.w1 = w_v; a.dst_rows = dst_rows; a.dtype = cfg->dtype;
+    return from_cuda(launch_linear_simt(a, stream));
+}
+
+yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, int32_t d_out,
+                        int32_t apply_ln, float ln_eps, const void *base, float base_w, void *out,
+                        int32_t dtype, cudaStream_t stream) {
+    if (dtype != YOCO_BF16 && dtype != YOCO_FP32) return YOCO_ERR_INVALID;
+    if (n < 0 || d_in < 1 || d_out < 1 || !(ln_eps > 0.f) || !isfinite(base_w))
+        return YOCO_ERR_INVALID;
+    if (n == 0) return YOCO_OK;
+    if (!ok_ptr(x) || !ok_ptr(w) || !ok_ptr(out) || !ok_opt(base)) return YOCO_ERR_INVALID;
+    LinearArgs a;
+    a.x = x; a.w = w; a.n = n; a.d_in = d_in; a.d_out = d_out; a.split_col = d_out;
+    a.apply_ln = apply_ln ? 1 : 0; a.eps = ln_eps;
+    a.out0 = out; a.out1 = nullptr; a.base0 = base; a.base1 = nullptr;
+    a.w0 = base_w; a.w1 = 0.f; a.dst_rows = nullptr; a.dtype = dtype;
+    return from_cuda(launch_linear_simt(a, stream));
+}
+
+yoco_status yoco_swa_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t T,
+                             int32_t window, void *o, float *lse, void *ring_k, void *ring_v,
+                             int32_t *slot_pos, const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (B < 0 || T < 0 || window < 1) return YOCO_ERR_INVALID;
+    const int rings = (ring_k != nullptr) + (ring_v != nullptr) + (slot_pos != nullptr);
+    if (rings != 0 && rings != 3) return YOCO_ERR_INVALID;
+    if (B == 0) return YOCO_OK;
+    if (T > 0 && (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_opt(lse)))
+        return YOCO_ERR_INVALID;
+    if (rings == 3 && (!ok_ptr(ring_k) || !ok_ptr(ring_v) || !ok_ptr(slot_pos)))
+        return YOCO_ERR_INVALID;
+    if (T > 0) {
+        PrefillArgs a;
+        a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+        a.B = B; a.Tq = T; a.Tkv = T; a.q_pos0 = 0; a.window = window;
+        a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
+        a.scale = eff_scale(cfg);
+        st = run_prefill(a, stream);
+        if (st != YOCO_OK) return st;
+    }
+    if (rings == 3)
+        return from_cuda(launch_ring_fill(k, v, B, T, window, cfg->Hkv, cfg->D, cfg->dtype, ring_k,
+                                          ring_v, slot_pos, stream));
+    return YOCO_OK;
+}
+
+yoco_status yoco_cross_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t Tq,
+                               int64_t Tkv, int64_t q_pos0, void *o, float *lse,
+                               const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (B < 0 || Tq < 0 || Tkv < 0 || q_pos0 < 0 || q_pos0 + Tq > Tkv) return YOCO_ERR_INVALID;
+    if (B == 0 || Tq == 0) return YOCO_OK;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_opt(lse)) return YOCO_ERR_INVALID;
+    PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.Tq = Tq; a.Tkv = Tkv; a.q_pos0 = q_pos0; a.window = 0;
+    a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
+    a.scale = eff_scale(cfg);
+    return run_prefill(a, stream);
+}
+
+size_t yoco_cross_decode_workspace_size(int32_t B, int64_t max_len, const yoco_attn_cfg *cfg) {
+    if (check_cfg(cfg) != YOCO_OK) return 0;
+    DecodePlan pl;
+    if (!make_decode_plan(B, max_len, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl)) return 0;
+    return pl.ws_bytes;
+}
+
+size_t yoco_swa_decode_workspace_size(int32_t B, int32_t window, const yoco_attn_cfg *cfg) {
+    return yoco_cross_decode_workspace_size(B, window, cfg);
+}
+
+yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_cache,
+                              const int64_t *seq_start, const int32_t *seq_len, int32_t B,
+                              int64_t max_len, void *o, float *lse, void *workspace,
+                              size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (B < 0 || max_len < 1) return YOCO_ERR_INVALID;
+    if (B == 0) return YOCO_OK;
+    if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_start) ||
+        !seq_len || !ok_ptr(o) || !ok_opt(lse))
+        return YOCO_ERR_INVALID;
+    DecodePlan pl;
+    if (!make_decode_plan(B, max_len, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl))
+        return YOCO_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace) || ws_bytes < pl.ws_bytes) return YOCO_ERR_WORKSPACE;
+    DecodeArgs a;
+    a.q = q; a.k = k_cache; a.v = v_cache; a.seq_start = seq_start; a.seq_len = seq_len;
+    a.slot_pos = nullptr; a.pos = nullptr; a.window = 0;
+    a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
+    a.scale = eff_scale(cfg); a.o = o; a.lse = lse; a.ws = workspace;
+    return from_cuda(launch_decode(a, pl, stream));
+}
+
+yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
+                            const int64_t *pos, int32_t B, int32_t window, void *ring_k,
+                            void *ring_v, int32_t *slot_pos, void *o, void *workspace,
+                            size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (B < 0 || window < 1) return YOCO_ERR_INVALID;
+    if (B == 0) return YOCO_OK;
+    if (!ok_ptr(q) || !ok_ptr(k_new) || !ok_ptr(v_new) || !ok_ptr(pos) || !ok_ptr(ring_k) ||
+        !ok_ptr(ring_v) || !ok_ptr(slot_pos) || !ok_ptr(o))
+        return YOCO_ERR_INVALID;
+    DecodePlan pl;
+    if (!make_decode_plan(B, window, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl))
+        return YOCO_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace) || ws_bytes < pl.ws_bytes) return YOCO_ERR_WORKSPACE;
+    st = from_cuda(launch_ring_write(k_new, v_new, pos, B, window, cfg->Hkv, cfg->D, cfg->dtype,
+                                     ring_k, ring_v, slot_pos, stream));
+    if (st != YOCO_OK) return st;
+    DecodeArgs a;
+    a.q = q; a.k = ring_k; a.v = ring_v; a.seq_start = nullptr; a.seq_len = nullptr;
+    a.slot_pos = slot_pos; a.pos = pos; a.window = window;
+    a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
+    a.scale = eff_scale(cfg); a.o = o; a.lse = nullptr; a.ws = workspace;
+    return from_cuda(launch_decode(a, pl, stream));
+}
+
+double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_attn_cfg *cfg) {
+    if (!cfg || L_self < 0 || window < 0 || N < 0 || cfg->Hkv < 1 || cfg->D < 1) return -1.0;
+    const double row = 2.0 * cfg->Hkv * cfg->D * (cfg->dtype == YOCO_BF16 ? 2.0 : 4.0);
+    const int64_t c = window < N ? window : N;
+    return row * ((double)N + (double)L_self * (double)c);
+}
+
+yoco_status yoco_get_device_status(cudaStream_t stream) {
+    const cudaError_t e = cudaStreamSynchronize(stream);
+    const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc();
+    if (s) return YOCO_ERR_TIMEOUT;
+    return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,102 @@
+// Host-side launchers of the libyoco kernels (internal; the public ABI is
+// include/yoco.h).  Every launcher assumes its arguments were validated by
+// the API layer and returns the cudaError_t of its launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace yoco {
+
+enum Dtype { kBF16 = 0, kFP32 = 1 };
+
+inline size_t dtype_bytes(int dt) { return dt == kBF16 ? 2 : 4; }
+
+// ------------------------------------------------------------ decode plan
+// One decode "unit" is a contiguous token range of one sequence, streamed
+// through shared memory by one CTA for every KV head.  Its partial softmax
+// state (m, l, o) per query head and per consumer-warp subset goes to the
+// workspace; a merge kernel combines them.
+struct DecodePlan {
+    int64_t stage_tokens;  // tokens per pipeline stage (128 / Hkv)
+    int64_t split;         // tokens per unit (multiple of stage_tokens)
+    int64_t n_split;       // units per sequence at max_len
+    int sub;               // partial entries per unit per head (8 / Hkv)
+    int stages;            // pipeline depth
+    size_t smem_bytes;     // dynamic shared memory per CTA
+    size_t ws_bytes;       // workspace bytes
+};
+bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dtype,
+                      DecodePlan *plan);
+
+struct DecodeArgs {
+    const void *q;        // [B, Hq, D]
+    const void *k;        // cache [rows, Hkv, D]
+    const void *v;
+    const int64_t *seq_start;  // [B] (cross) or NULL (ring: b * window)
+    const int32_t *seq_len;    // [B] (cross) or NULL (ring: window slots)
+    const int32_t *slot_pos;   // ring only: [B, window]
+    const int64_t *pos;        // ring only: [B]
+    int32_t window;            // ring only
+    int32_t B, Hq, Hkv, D, dtype;
+    float scale;
+    void *o;       // [B, Hq, D]
+    float *lse;    // [B, Hq] or NULL
+    void *ws;      // workspace
+};
+cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s);
+
+// SWA ring write of one new token per sequence.
+cudaError_t launch_ring_write(const void *k_new, const void *v_new, const int64_t *pos,
+                              int32_t B, int32_t window, int Hkv, int D, int dtype,
+                              void *ring_k, void *ring_v, int32_t *slot_pos, cudaStream_t s);
+
+// Ring fill after a prefill of T tokens.
+cudaError_t launch_ring_fill(const void *k, const void *v, int32_t B, int64_t T, int32_t window,
+                             int Hkv, int D, int dtype, void *ring_k, void *ring_v,
+                             int32_t *slot_pos, cudaStream_t s);
+
+// ------------------------------------------------------------- prefill
+struct PrefillArgs {
+    const void *q;   // [B, Tq, Hq, D]
+    const void *k;   // [B, Tkv, Hkv, D]
+    const void *v;
+    void *o;         // [B, Tq, Hq, D]
+    float *lse;      // [B, Hq, Tq] or NULL
+    int32_t B;
+    int64_t Tq, Tkv, q_pos0;
+    int32_t window;  // 0: causal only
+    int32_t Hq, Hkv, D, dtype;
+    float scale;
+};
+// CUDA-core path (any dtype; the fp32 path).
+cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t s);
+// Tensor-core path (bf16): tcgen05 + TMEM + TMA.  Returns cudaErrorNotSupported
+// when the shape is outside what it was built for.
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s);
+
+// ------------------------------------------------------------ projection
+struct LinearArgs {
+    const void *x;      // [n, d_in]
+    const void *w;      // [d_out, d_in]
+    int64_t n;
+    int32_t d_in, d_out;
+    int32_t apply_ln;
+    float eps;
+    int32_t split_col;  // columns < split_col -> out0/base0, the rest -> out1/base1
+    void *out0, *out1;
+    const void *base0, *base1;
+    float w0, w1;
+    const int64_t *dst_rows;  // optional row remap of the outputs
+    int32_t dtype;
+};
+cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
+
+// Device status words of the translation units that hold bounded waits.
+unsigned int read_and_clear_status_decode();
+unsigned int read_and_clear_status_prefill_tc();
+
+int device_sm_count();
+
+}  // namespace yoco

@@ -1,0 +1,101 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, validates arguments before launching anything, and its host
+helpers (workspace sizing, cache accounting) are right."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import oracle
+import shared_kv_decoder_b200 as yoco
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(yoco_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = yoco.load()
+    names = _declared()
+    assert len(names) >= 12
+    for n in sorted(names):
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert L.yoco_version().startswith(b"yoco-b200")
+
+
+def test_status_strings():
+    L = yoco.load()
+    for s in range(6):
+        assert L.yoco_status_string(s)
+    assert L.yoco_status_string(99) == b"unknown status"
+
+
+def _cfg(Hq=32, Hkv=8, D=128, dtype=0, scale=0.0):
+    return yoco.AttnCfg(Hq, Hkv, D, scale, dtype)
+
+
+FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+@pytest.mark.parametrize("cfg,expect", [
+    (_cfg(Hq=30, Hkv=8), yoco.ERR_INVALID),          # Hq % Hkv
+    (_cfg(D=96), yoco.ERR_UNSUPPORTED),               # head dim not built
+    (_cfg(Hq=48, Hkv=3), yoco.ERR_UNSUPPORTED),       # group 16
+    (_cfg(dtype=7), yoco.ERR_INVALID),
+    (_cfg(scale=-1.0), yoco.ERR_INVALID),
+])
+def test_bad_cfg_rejected_before_launch(cfg, expect):
+    L = yoco.load()
+    st = L.yoco_cross_prefill(FAKE, FAKE, FAKE, 1, 128, 128, 0, FAKE, None, ctypes.byref(cfg), None)
+    assert st == expect
+
+
+def test_bad_arguments_rejected_before_launch():
+    L = yoco.load()
+    c = _cfg()
+    b = ctypes.byref(c)
+    # q_pos0 + Tq > Tkv
+    assert L.yoco_cross_prefill(FAKE, FAKE, FAKE, 1, 128, 100, 0, FAKE, None, b, None) == yoco.ERR_INVALID
+    # null and misaligned pointers
+    assert L.yoco_cross_prefill(None, FAKE, FAKE, 1, 128, 128, 0, FAKE, None, b, None) == yoco.ERR_INVALID
+    assert L.yoco_cross_prefill(MISALIGNED, FAKE, FAKE, 1, 128, 128, 0, FAKE, None, b, None) == yoco.ERR_INVALID
+    # window < 1, partial ring arguments
+    assert L.yoco_swa_prefill(FAKE, FAKE, FAKE, 1, 64, 0, FAKE, None, None, None, None, b, None) == yoco.ERR_INVALID
+    assert L.yoco_swa_prefill(FAKE, FAKE, FAKE, 1, 64, 8, FAKE, None, FAKE, None, None, b, None) == yoco.ERR_INVALID
+    # decode: max_len < 1, workspace missing / too small
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, FAKE, None, FAKE, 1 << 30, b, None) == yoco.ERR_INVALID
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 1000, FAKE, None, None, 0, b, None) == yoco.ERR_WORKSPACE
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 1000, FAKE, None, FAKE, 16, b, None) == yoco.ERR_WORKSPACE
+    # projection: bad eps
+    assert L.yoco_kv_project_blend(FAKE, 4, 64, FAKE, 1, 0.0, None, None, 0.0, 0.0, None, FAKE, FAKE, b, None) == yoco.ERR_INVALID
+    # empty inputs are a successful no-op (nothing launched)
+    assert L.yoco_cross_prefill(FAKE, FAKE, FAKE, 0, 128, 128, 0, FAKE, None, b, None) == yoco.OK
+    assert L.yoco_cross_prefill(FAKE, FAKE, FAKE, 1, 0, 128, 0, FAKE, None, b, None) == yoco.OK
+    assert L.yoco_kv_project_blend(FAKE, 0, 64, FAKE, 1, 1e-5, None, None, 0.0, 0.0, None, FAKE, FAKE, b, None) == yoco.OK
+
+
+def test_workspace_size_monotone_and_positive():
+    sizes = [yoco.cross_decode_workspace_size(B, L, 32, 8, 128, torch.bfloat16)
+             for B, L in [(1, 1), (1, 4096), (16, 131072), (16, 262144)]]
+    assert all(s > 0 for s in sizes)
+    assert sizes == sorted(sizes)
+    assert yoco.cross_decode_workspace_size(1, 0, 32, 8, 128, torch.bfloat16) == 0
+    # group size 16 has no decode build
+    assert yoco.cross_decode_workspace_size(1, 100, 32, 2, 128, torch.bfloat16) == 0
+
+
+@pytest.mark.parametrize("L_self,window,N", [(13, 1024, 1 << 20), (2, 32, 16), (0, 8, 100), (3, 64, 0)])
+def test_cache_bytes_matches_oracle(L_self, window, N):
+    got = yoco.cache_bytes(L_self, window, N, 8, 128, torch.bfloat16)
+    assert got == oracle.cache_bytes_yoco(L_self, window, N, 8, 128, 2)
