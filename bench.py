@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the YOCO / YOCO++ attention core on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic,
+seeded inputs (bf16, ~N(0,1); weights ~N(0,1/d)):
+
+  swa      self-decoder layer slice: K/V projection of B=4 x T=65536 tokens
+           (d=4096) with the YOCO++ blend fused, sliding-window prefill
+           (window 1024, 32q/8kv heads, head_dim 128) with ring fill, then one
+           decode step (projection of 4 new tokens + ring write + window read)
+  gkv      global KV produced once: LN(x) W_kv^g for T=32768 tokens
+  prefill  cross-decoder causal prefill, T=32768, 32q/8kv, head_dim 128,
+           14 cross layers (each its own Q) over the one shared K/V   <- value
+  decode   one decode step: global-KV append of 16 new tokens, then 16 cross
+           layers each read the whole shared cache, batch 16, ragged
+           lengths uniform in [65536, 131072]                          <- decode
+
+`value` is the cross-decoder prefill throughput in TFLOP/s of algorithmic
+work (causal pairs only: 4 * Hq * D * sum_i (i + 1) per layer); `decode`
+carries tokens/s and HBM GB/s.  Inputs are resident in HBM when the timed
+region starts; a 256 MB buffer is rewritten between steps to flush L2 (every
+part's inputs are also larger than L2).  Times are CUDA events on the
+launching stream; with several GPUs each rank runs an independent replica and
+the max over ranks is taken.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl yoco|reference]
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "cross-decoder prefill TFLOP/s + decode tokens/s & HBM GB/s, 1 B200"
+WORKLOAD = ("cross-decoder causal prefill B=1 T=32768 32q/8kv D=128 x14 layers over one shared KV "
+            "+ decode step B=16 ragged 64K-128K x16 layers + SWA/blend layer slice B=4 T=65536 W=1024")
+
+P = dict(T=32768, Hq=32, Hkv=8, D=128, layers=14, d=4096)          # cross prefill
+DEC = dict(B=16, lo=65536, hi=131072, Hq=32, Hkv=8, D=128, layers=16, d=4096)
+SWA = dict(B=4, T=65536, W=1024, Hq=32, Hkv=8, D=128, d=4096)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["yoco", "reference"], default="yoco")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def prefill_flops_per_layer(T, Hq, D, q_pos0=0, window=0):
+    """4 * Hq * D * sum over query rows of the visible key count."""
+    import numpy as np
+    i = np.arange(T, dtype=np.float64) + q_pos0
+    vis = i + 1 if window <= 0 else np.minimum(i + 1, window)
+    return 4.0 * Hq * D * float(vis.sum())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        loaded = [s for s in sm if mx and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- workloads
+def make_workload(dev):
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    import workloads as wl
+    bf = torch.bfloat16
+    W = {}
+    # cross prefill: x_mid -> global K/V, then 14 layers each with its own Q
+    T, Hq, Hkv, D, d = P["T"], P["Hq"], P["Hkv"], P["D"], P["d"]
+    W["x_mid"] = wl.normal((T, d), 1100, bf, dev)
+    W["w_g"] = wl.normal((2 * Hkv * D, d), 1101, bf, dev, std=d ** -0.5)
+    W["kg"] = torch.empty((1, T, Hkv, D), dtype=bf, device=dev)
+    W["vg"] = torch.empty((1, T, Hkv, D), dtype=bf, device=dev)
+    W["qs"] = [wl.normal((1, T, Hq, D), 1200 + l, bf, dev) for l in range(P["layers"])]
+    W["o"] = torch.empty((1, T, Hq, D), dtype=bf, device=dev)
+    # decode: packed shared cache of 16 ragged sequences
+    lens = wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], 2000)
+    starts = torch.cumsum(torch.cat([torch.zeros(1, dtype=torch.int64), lens[:-1]]), 0)
+    rows = int(lens.sum())
+    W["lens"], W["starts"], W["rows"] = lens, starts, rows
+    W["kc"] = wl.normal((rows, Hkv, D), 2001, bf, dev)
+    W["vc"] = wl.normal((rows, Hkv, D), 2002, bf, dev)
+    W["x_new"] = wl.normal((DEC["B"], d), 2003, bf, dev)
+    W["w_gd"] = wl.normal((2 * Hkv * D, d), 2004, bf, dev, std=d ** -0.5)
+    W["qd"] = [wl.normal((DEC["B"], Hq, D), 2100 + l, bf, dev) for l in range(DEC["layers"])]
+    W["od"] = torch.empty((DEC["B"], Hq, D), dtype=bf, device=dev)
+    W["seq_start"] = starts.to(dev)
+    W["seq_len"] = lens.to(torch.int32).to(dev)
+    W["dst_rows"] = (starts + lens - 1).to(dev)
+    W["max_len"] = int(lens.max())
+    W["ws"] = torch.empty(yoco.cross_decode_workspace_size(DEC["B"], W["max_len"], Hq, Hkv, D, bf),
+                          dtype=torch.uint8, device=dev)
+    # self-decoder slice
+    B4, T4, W4 = SWA["B"], SWA["T"], SWA["W"]
+    n4 = B4 * T4
+    W["x4"] = wl.normal((n4, d), 3001, bf, dev)
+    W["w4"] = wl.normal((2 * Hkv * D, d), 3002, bf, dev, std=d ** -0.5)
+    W["k1"] = wl.normal((n4, Hkv, D), 3003, bf, dev)
+    W["v1"] = wl.normal((n4, Hkv, D), 3004, bf, dev)
+    W["w_l"] = float(wl.uniform((1,), 3005)[0])
+    W["k4"] = torch.empty((B4, T4, Hkv, D), dtype=bf, device=dev)
+    W["v4"] = torch.empty((B4, T4, Hkv, D), dtype=bf, device=dev)
+    W["q4"] = wl.normal((B4, T4, Hq, D), 3006, bf, dev)
+    W["o4"] = torch.empty((B4, T4, Hq, D), dtype=bf, device=dev)
+    W["ring"] = (torch.empty((B4, W4, Hkv, D), dtype=bf, device=dev),
+                 torch.empty((B4, W4, Hkv, D), dtype=bf, device=dev),
+                 torch.empty((B4, W4), dtype=torch.int32, device=dev))
+    W["x4t"] = wl.normal((B4, d), 3007, bf, dev)
+    W["k1t"] = wl.normal((B4, Hkv, D), 3008, bf, dev)
+    W["v1t"] = wl.normal((B4, Hkv, D), 3009, bf, dev)
+    W["q4t"] = wl.normal((B4, Hq, D), 3010, bf, dev)
+    W["k4t"] = torch.empty((B4, Hkv, D), dtype=bf, device=dev)
+    W["v4t"] = torch.empty((B4, Hkv, D), dtype=bf, device=dev)
+    W["o4t"] = torch.empty((B4, Hq, D), dtype=bf, device=dev)
+    W["pos4"] = torch.full((B4,), T4, dtype=torch.int64, device=dev)
+    W["ws4"] = torch.empty(yoco.swa_decode_workspace_size(B4, W4, Hq, Hkv, D, bf),
+                           dtype=torch.uint8, device=dev)
+    W["flush"] = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    return W
+
+
+def run_step(W, ev=None):
+    """One pass of the hot path.  ev: dict of per-part event lists to record."""
+    import shared_kv_decoder_b200 as yoco
+    Hkv, D = P["Hkv"], P["D"]
+
+    def rec(name, i):
+        if ev is not None:
+            ev[name][i].record()
+
+    # self-decoder slice (projection + blend, SWA prefill + ring, one decode step)
+    rec("swa", 0)
+    yoco.kv_project_blend(W["x4"], W["w4"], Hkv, D, W["k1"], W["v1"], W["w_l"], W["w_l"],
+                          k_out=W["k4"].view(-1, Hkv, D), v_out=W["v4"].view(-1, Hkv, D))
+    yoco.swa_prefill(W["q4"], W["k4"], W["v4"], SWA["W"], ring=W["ring"], o=W["o4"])
+    yoco.kv_project_blend(W["x4t"], W["w4"], Hkv, D, W["k1t"], W["v1t"], W["w_l"], W["w_l"],
+                          k_out=W["k4t"], v_out=W["v4t"])
+    rk, rv, sp = W["ring"]
+    yoco.swa_decode(W["q4t"], W["k4t"], W["v4t"], W["pos4"], rk, rv, sp, SWA["W"],
+                    workspace=W["ws4"], o=W["o4t"])
+    rec("swa", 1)
+    # global KV, produced once
+    rec("gkv", 0)
+    yoco.kv_project_blend(W["x_mid"], W["w_g"], Hkv, D, k_out=W["kg"].view(-1, Hkv, D),
+                          v_out=W["vg"].view(-1, Hkv, D))
+    rec("gkv", 1)
+    # cross-decoder prefill, 14 layers
+    for l in range(P["layers"]):
+        if ev is not None:
+            ev["prefill_l"][2 * l].record()
+        yoco.cross_prefill(W["qs"][l], W["kg"], W["vg"], o=W["o"])
+        if ev is not None:
+            ev["prefill_l"][2 * l + 1].record()
+    # decode step: append 16 new global-KV rows, then 16 cross layers
+    rec("decode", 0)
+    yoco.kv_project_blend(W["x_new"], W["w_gd"], Hkv, D, dst_rows=W["dst_rows"],
+                          k_out=W["kc"], v_out=W["vc"])
+    for l in range(DEC["layers"]):
+        if ev is not None:
+            ev["decode_l"][2 * l].record()
+        yoco.cross_decode(W["qd"][l], W["kc"], W["vc"], W["seq_start"], W["seq_len"],
+                          W["max_len"], workspace=W["ws"], o=W["od"])
+        if ev is not None:
+            ev["decode_l"][2 * l + 1].record()
+    rec("decode", 1)
+
+
+def new_events():
+    import torch
+    mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    return {"swa": mk(2), "gkv": mk(2), "decode": mk(2), "prefill_l": mk(2 * P["layers"]),
+            "decode_l": mk(2 * DEC["layers"]), "step": mk(2)}
+
+
+def e2e_prefill(W, steps, warmup):
+    """Prefill through the public API with HOST buffers: every step copies the
+    step's Q (14 layers) and the shared K/V from pinned host memory and reads
+    every layer's output back, inside the timed region."""
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    hq = [q.cpu().pin_memory() for q in W["qs"]]
+    hk = W["kg"].cpu().pin_memory()
+    hv = W["vg"].cpu().pin_memory()
+    ho = torch.empty(W["o"].shape, dtype=W["o"].dtype).pin_memory()
+    dq = torch.empty_like(W["qs"][0])
+    dk, dv = torch.empty_like(W["kg"]), torch.empty_like(W["vg"])
+    s = torch.cuda.current_stream()
+    times = []
+    for it in range(warmup + steps):
+        W["flush"].zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        for l in range(P["layers"]):
+            dq.copy_(hq[l], non_blocking=True)
+            yoco.cross_prefill(dq, dk, dv, o=W["o"])
+            ho.copy_(W["o"], non_blocking=True)
+        e1.record()
+        s.synchronize()
+        if it >= warmup:
+            times.append(e0.elapsed_time(e1))
+    h2d = sum(q.numel() * q.element_size() for q in hq) + 2 * hk.numel() * hk.element_size()
+    d2h = P["layers"] * ho.numel() * ho.element_size()
+    return times, h2d, d2h
+
+
+# ------------------------------------------------------------ CPU baseline
+def cpu_baseline(W, seconds, label="oracle"):
+    """The oracle, as it stands, on sampled query rows of the prefill
+    workload (layer 0), timed on this host's cores."""
+    import numpy as np
+    import oracle
+    T, Hq, D = P["T"], P["Hq"], P["D"]
+    k = W["kg"].double().cpu().numpy() if hasattr(W["kg"], "double") else W["kg"]
+    v = W["vg"].double().cpu().numpy() if hasattr(W["vg"], "double") else W["vg"]
+    q = W["qs"][0] if not hasattr(W["qs"][0], "double") else W["qs"][0].double().cpu().numpy()
+    rng = np.random.default_rng(7)
+
+    def run(n):
+        rows = np.sort(rng.integers(0, T, size=n))
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, 0, 0, rows=[(0, int(i)) for i in rows])
+        dt = time.perf_counter() - t0
+        return dt, 4.0 * Hq * D * float((rows + 1).sum()), n
+
+    dt, fl, n = run(4)
+    n2 = max(4, int(4 * seconds / max(dt, 1e-3)))
+    dt, fl, n = run(n2)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} random query rows (all 32 heads) of cross prefill layer 0, T=32768, "
+                      f"fp64, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm, on the same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import workloads as wl
+    T, Hq, Hkv, D = P["T"], P["Hq"], P["Hkv"], P["D"]
+    # the shared K/V and layer-0 Q on the host (bf16-rounded, widened to fp64)
+    W = {"kg": wl.normal((1, T, Hkv, D), 1300, torch.bfloat16).double().numpy(),
+         "vg": wl.normal((1, T, Hkv, D), 1301, torch.bfloat16).double().numpy(),
+         "qs": [wl.normal((1, T, Hq, D), 1200, torch.bfloat16).double().numpy()]}
+    per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for it in range(args.warmup + args.steps):
+        cb = cpu_baseline(W, per_step)
+        if it >= args.warmup:
+            vals.append(cb)
+    value = statistics.median(c["value"] for c in vals)
+    flops_per_step = prefill_flops_per_layer(T, Hq, D) * P["layers"]
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": flops_per_step / (value * 1e12) * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference",
+           "config": {"workload": WORKLOAD, "model": "YOCO attention core (synthetic)",
+                      "global_batch": 1, "seq_len": T, "parallelism": "replicas",
+                      "note": "each step times the oracle on a bounded sample of query rows; "
+                              "ms_per_step is extrapolated to the 14-layer prefill"},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": vals[0]["cores"],
+                            "kind": "oracle", "sample": vals[0]["sample"]},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import shared_kv_decoder_b200 as yoco
+    yoco.load()
+    peaks = load_peaks()
+    W = make_workload(dev)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        W["flush"].zero_()
+        run_step(W)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = yoco.launch_count()
+    evs = []
+    for _ in range(args.steps):
+        W["flush"].zero_()
+        ev = new_events()
+        ev["step"][0].record()
+        run_step(W, ev)
+        ev["step"][1].record()
+        evs.append(ev)
+    torch.cuda.synchronize()
+    launches = yoco.launch_count() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+
+    def pair(ev, name, i=0):
+        return ev[name][i].elapsed_time(ev[name][i + 1])
+
+    step_ms = [pair(e, "step") for e in evs]
+    pre_l = [pair(e, "prefill_l", 2 * l) for e in evs for l in range(P["layers"])]
+    dec_l = [pair(e, "decode_l", 2 * l) for e in evs for l in range(DEC["layers"])]
+    pre_ms = [sum(pair(e, "prefill_l", 2 * l) for l in range(P["layers"])) for e in evs]
+    dec_ms = [pair(e, "decode") for e in evs]
+    swa_ms = [pair(e, "swa") for e in evs]
+    gkv_ms = [pair(e, "gkv") for e in evs]
+
+    tot = {"step": sum(step_ms), "pre": sum(pre_ms), "dec": sum(dec_ms)}
+    if world > 1:
+        t = torch.tensor([tot["step"], tot["pre"], tot["dec"]], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot = {"step": float(t[0]), "pre": float(t[1]), "dec": float(t[2])}
+
+    f_layer = prefill_flops_per_layer(P["T"], P["Hq"], P["D"])
+    value = world * args.steps * P["layers"] * f_layer / (tot["pre"] * 1e-3) / 1e12
+    dec_bytes_layer = float(W["lens"].sum()) * DEC["Hkv"] * DEC["D"] * 2 * 2
+    dec_tok_s = world * args.steps * DEC["B"] / (tot["dec"] * 1e-3)
+    dec_gbs_layer = dec_bytes_layer / (statistics.mean(dec_l) * 1e-3) / 1e9
+    pre_tflops_launch = f_layer / (statistics.mean(pre_l) * 1e-3) / 1e12
+    n4 = SWA["B"] * SWA["T"]
+    swa_proj_fl = 2.0 * n4 * P["d"] * 2 * SWA["Hkv"] * SWA["D"]
+    swa_att_fl = SWA["B"] * prefill_flops_per_layer(SWA["T"], SWA["Hq"], SWA["D"], 0, SWA["W"])
+    gkv_fl = 2.0 * P["T"] * P["d"] * 2 * P["Hkv"] * P["D"]
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot["step"] / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "model": "YOCO attention core (synthetic, random init)",
+                   "global_batch": world, "seq_len": P["T"], "parallelism": "replicas",
+                   "l2": "every part's inputs exceed L2; 256 MB rewritten between steps"},
+        "decode": {"tokens_per_s": dec_tok_s, "hbm_gbs": dec_gbs_layer,
+                   "frac_hbm": dec_gbs_layer / peaks["hbm"], "ms_per_decode_step": tot["dec"] / args.steps,
+                   "bytes_per_layer": dec_bytes_layer},
+        "swa_slice": {"ms": statistics.mean(swa_ms),
+                      "flops": swa_proj_fl + swa_att_fl},
+        "gkv": {"ms": statistics.mean(gkv_ms), "tflops": gkv_fl / (statistics.mean(gkv_ms) * 1e-3) / 1e12},
+        "roofline": {"kernel": "cross prefill (yoco_cross_prefill)", "bound": "tensor",
+                     "achieved": pre_tflops_launch, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                     "frac": pre_tflops_launch / peaks["bf16_sus"], "traffic": None,
+                     "peak_src": f"{peaks['src']} bf16 sustained"},
+        "roofline_decode": {"kernel": "cross decode (yoco_cross_decode)", "bound": "hbm",
+                            "achieved": dec_gbs_layer, "peak": peaks["hbm"], "unit": "GB/s",
+                            "frac": dec_gbs_layer / peaks["hbm"], "traffic": None,
+                            "peak_src": f"{peaks['src']} hbm"},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if not args.no_e2e:
+        times, h2d, d2h = e2e_prefill(W, args.steps, 1)
+        e2e_ms = sum(times)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        out["e2e"] = {"value": world * len(times) * P["layers"] * f_layer / (e2e_ms * 1e-3) / 1e12,
+                      "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(W, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

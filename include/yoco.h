@@ -169,6 +169,10 @@ yoco_status yoco_get_device_status(cudaStream_t stream);
 /* Static description of a status code. */
 const char *yoco_status_string(yoco_status s);
 
+/* Number of kernels this library has launched in this process (host-side
+ * counter, incremented at every launch on every stream). */
+uint64_t yoco_launch_count(void);
+
 /* Library version string. */
 const char *yoco_version(void);
 

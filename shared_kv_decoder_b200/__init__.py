@@ -18,7 +18,7 @@ import torch
 
 __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_prefill",
            "swa_decode", "cross_prefill", "cross_decode", "cross_decode_workspace_size",
-           "swa_decode_workspace_size", "cache_bytes", "device_status", "AttnCfg"]
+           "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -72,6 +72,7 @@ def load():
         "yoco_get_device_status": (st, [vp]),
         "yoco_status_string": (ctypes.c_char_p, [st]),
         "yoco_version": (ctypes.c_char_p, []),
+        "yoco_launch_count": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -230,6 +231,11 @@ def cross_decode(q, k_cache, v_cache, seq_start, seq_len, max_len, workspace=Non
 def cache_bytes(L_self, window, N, Hkv, D, dtype=torch.bfloat16):
     cfg = _cfg(Hkv, Hkv, D, dtype)
     return float(load().yoco_cache_bytes(L_self, window, N, ctypes.byref(cfg)))
+
+
+def launch_count():
+    """Kernels launched by the library so far in this process."""
+    return int(load().yoco_launch_count())
 
 
 def device_status():

@@ -5,10 +5,17 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/yoco.h"
 #include "launch.h"
 
 using namespace yoco;
+
+namespace yoco {
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace yoco
 
 namespace {
 
@@ -53,6 +60,8 @@ yoco_status run_prefill(const PrefillArgs &a, cudaStream_t s) {
 extern "C" {
 
 const char *yoco_version(void) { return "yoco-b200 0.1 (sm_100a)"; }
+
+uint64_t yoco_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char *yoco_status_string(yoco_status s) {
     switch (s) {

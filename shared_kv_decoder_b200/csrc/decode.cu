@@ -365,6 +365,7 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
     const int64_t units = (int64_t)a.B * pl.n_split;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, device_sm_count()));
     kern<<<grid, kDecodeThreads, pl.smem_bytes, st>>>(p);
+    note_launches(2);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int mgrid = (int)(((int64_t)a.B * a.Hq + 3) / 4);
@@ -418,6 +419,7 @@ cudaError_t launch_ring_write(const void *k_new, const void *v_new, const int64_
                               void *ring_v, int32_t *slot_pos, cudaStream_t st) {
     if (B == 0) return cudaSuccess;
     const int64_t re = (int64_t)Hkv * D;
+    note_launches(1);
     if (dtype == kBF16)
         ring_write_kernel<__nv_bfloat16><<<B, 256, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new), pos,
@@ -464,6 +466,7 @@ cudaError_t launch_ring_fill(const void *k, const void *v, int32_t B, int64_t T,
     if (B == 0) return cudaSuccess;
     const int64_t re = (int64_t)Hkv * D;
     dim3 grid(window, B);
+    note_launches(1);
     if (dtype == kBF16)
         ring_fill_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), T, window,

@@ -99,4 +99,7 @@ unsigned int read_and_clear_status_prefill_tc();
 
 int device_sm_count();
 
+// Host-side count of kernel launches (reported by yoco_launch_count()).
+void note_launches(int n);
+
 }  // namespace yoco

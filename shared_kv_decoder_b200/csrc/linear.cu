@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const LinearArgs a) {
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t st) {
     if (a.n == 0 || a.d_out == 0) return cudaSuccess;
     dim3 grid((unsigned)((a.d_out + kLinBN - 1) / kLinBN), (unsigned)((a.n + kLinBM - 1) / kLinBM));
+    note_launches(1);
     if (a.dtype == kBF16)
         linear_simt_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else

@@ -118,6 +118,7 @@ template <typename T>
 static cudaError_t launch_simt_t(const PrefillArgs &a, cudaStream_t st) {
     dim3 grid((unsigned)((a.Tq + kSimtBQ - 1) / kSimtBQ), a.Hq, a.B);
     const float sl2 = a.scale * kLog2e;
+    note_launches(1);
     if (a.D == 128)
         attn_prefill_simt_kernel<T, 128><<<grid, 128, 0, st>>>(a, sl2);
     else if (a.D == 64)
