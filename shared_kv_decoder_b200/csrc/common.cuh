@@ -77,10 +77,10 @@ YOCO_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// A wait gives up after this many SM clock cycles (about one second at the
-// B200's clocks): far above any legitimate wait, short enough that a lost
-// arrive becomes an error status rather than a hung GPU.
-constexpr long long kWaitLimitCycles = 2000000000LL;
+// A wait gives up after this many SM clock cycles (about 0.1 s at the B200's
+// clocks): far above any legitimate wait (microseconds), short enough that a
+// lost arrive becomes an error status rather than a hung GPU.
+constexpr long long kWaitLimitCycles = 200000000LL;
 
 // Bounded wait on an mbarrier phase.  Returns false (and sets *status) when
 // the limit passes without the phase completing.

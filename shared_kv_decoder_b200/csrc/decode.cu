@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
     constexpr int DPL = CPL * EPC;            // dims per lane
     static_assert(CPL >= 1 && CPR % kLanesPerTok == 0, "head dim too small for the lane layout");
 
+    if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
     extern __shared__ __align__(128) unsigned char smem[];
     const int64_t row_elems = (int64_t)p.Hkv * D;
     const size_t half_bytes = (size_t)kRowsPerStage * D * sizeof(T);
