@@ -143,6 +143,24 @@ yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_
                               int64_t max_len, void *o, float *lse, void *workspace,
                               size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream);
 
+/* yoco_cross_decode for callers that cannot allocate device memory: a C host
+ * or plugin that is handed only its input and output buffers, or a process
+ * whose framework already holds nearly all device memory in its own pool.
+ * The method's pages have no counterpart to this call; it exists for them.
+ * Same arguments and result as yoco_cross_decode, without the workspace: the
+ * split-KV scratch is a 32 MiB array inside the library, reserved on every
+ * GPU that loads it until the process exits.  A decode whose plan needs more
+ * (see yoco_cross_decode_workspace_size) returns YOCO_ERR_WORKSPACE and
+ * launches nothing.  The first call on a device looks up the array's address
+ * on that device (which must be current); make it before any stream capture.
+ * All calls on a device share the array and leave their partials in it;
+ * nothing needs clearing between calls, but calls whose kernels overlap on
+ * the GPU race on it, so serialise them. */
+yoco_status yoco_cross_decode_static(const void *q, const void *k_cache, const void *v_cache,
+                                     const int64_t *seq_start, const int32_t *seq_len, int32_t B,
+                                     int64_t max_len, void *o, float *lse,
+                                     const yoco_attn_cfg *cfg, cudaStream_t stream);
+
 /* Workspace bytes for yoco_cross_decode / yoco_swa_decode (0 on bad args). */
 size_t yoco_cross_decode_workspace_size(int32_t B, int64_t max_len, const yoco_attn_cfg *cfg);
 size_t yoco_swa_decode_workspace_size(int32_t B, int32_t window, const yoco_attn_cfg *cfg);
