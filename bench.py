@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj"], default=None,
+                    help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
 
 
@@ -339,8 +341,69 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_case(args):
+    """One kernel on a small case whose inputs still exceed L2 (126 MB):
+      prefill  cross prefill T=16384, 32q/8kv, D=128 (Q 128 MB, K+V 64 MB)
+      decode   cross decode, batch 16, lengths in [16384, 32768] (cache ~1.6 GB)
+      swa      sliding-window prefill B=1, T=65536, window 1024 (Q 512 MB)
+      proj     K/V projection + blend, 32768 tokens, d=4096 (x 256 MB)
+    Prints one JSON line with the mean launch time and the work rate."""
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    import workloads as wl
+    bf, dev = torch.bfloat16, "cuda"
+    yoco.load()
+    Hq, Hkv, D = 32, 8, 128
+    if args.case == "prefill":
+        T = 16384
+        q = wl.normal((1, T, Hq, D), 1, bf, dev); k = wl.normal((1, T, Hkv, D), 2, bf, dev)
+        v = wl.normal((1, T, Hkv, D), 3, bf, dev); o = torch.empty_like(q)
+        fn = lambda: yoco.cross_prefill(q, k, v, o=o)
+        work, unit = prefill_flops_per_layer(T, Hq, D), "TFLOP/s"
+    elif args.case == "decode":
+        lens = wl.ragged_lengths(16, 16384, 32768, 9)
+        starts = torch.cumsum(torch.cat([torch.zeros(1, dtype=torch.int64), lens[:-1]]), 0)
+        rows = int(lens.sum())
+        kc = wl.normal((rows, Hkv, D), 4, bf, dev); vc = wl.normal((rows, Hkv, D), 5, bf, dev)
+        q = wl.normal((16, Hq, D), 6, bf, dev); o = torch.empty_like(q)
+        ss, sl = starts.to(dev), lens.to(torch.int32).to(dev)
+        ws = torch.empty(yoco.cross_decode_workspace_size(16, int(lens.max()), Hq, Hkv, D, bf),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: yoco.cross_decode(q, kc, vc, ss, sl, int(lens.max()), workspace=ws, o=o)
+        work, unit = rows * Hkv * D * 4.0, "GB/s"
+    elif args.case == "swa":
+        T, Wn = 65536, 1024
+        q = wl.normal((1, T, Hq, D), 7, bf, dev); k = wl.normal((1, T, Hkv, D), 8, bf, dev)
+        v = wl.normal((1, T, Hkv, D), 9, bf, dev); o = torch.empty_like(q)
+        fn = lambda: yoco.swa_prefill(q, k, v, Wn, o=o)
+        work, unit = prefill_flops_per_layer(T, Hq, D, 0, Wn), "TFLOP/s"
+    else:
+        n, d = 32768, 4096
+        x = wl.normal((n, d), 10, bf, dev); w = wl.normal((2 * Hkv * D, d), 11, bf, dev, std=d ** -0.5)
+        kb = wl.normal((n, Hkv, D), 12, bf, dev); vb = wl.normal((n, Hkv, D), 13, bf, dev)
+        ko = torch.empty_like(kb); vo = torch.empty_like(vb)
+        fn = lambda: yoco.kv_project_blend(x, w, Hkv, D, kb, vb, 0.5, 0.5, k_out=ko, v_out=vo)
+        work, unit = 2.0 * n * d * 2 * Hkv * D, "TFLOP/s"
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    times = []
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(); fn(); e1.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.mean(times)
+    rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print(json.dumps({"case": args.case, "ms": ms, "rate": rate, "unit": unit,
+                      "status": yoco.device_status()}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.impl == "reference":
         run_reference(args)
         return

@@ -31,6 +31,7 @@
 #include "launch.h"
 
 #include <algorithm>
+#include <type_traits>
 
 namespace yoco {
 
@@ -277,6 +278,255 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
     if (warp == kConsumerWarps && lane == 0) producer_drain(full, it, p.stages);
 }
 
+// ---------------------------------------------------------------------------
+// bf16 decode on the tensor cores (mma.sync m16n8k16, fp32 accumulate).
+//
+// The CUDA-core kernel above spends ~150 instructions per KB of K/V (unpack,
+// per-head FMAs, eight-lane butterflies) and is issue-bound well below HBM
+// bandwidth.  Here the GQA group's query heads form the M rows of a
+// 16 x 16 A fragment (G <= 8 real rows), so S = q K^T and O += P V are a few
+// warp-wide MMAs per 16 tokens and the kernel is left waiting on HBM only.
+// Stage layout in shared memory: one row per token holding all KV heads,
+// with a 16-byte pad so that the eight consecutive token rows an ldmatrix
+// gathers fall in distinct bank groups; each token row is one bulk copy.
+// P goes from the S accumulators straight into the A fragment of P.V
+// (tokens 0-7 and 8-15 of the warp's 16 are the two S column tiles).
+YOCO_DEV void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+YOCO_DEV void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// c += A * B for one m16n8k16 tile; the A rows 8-15 are always zero here.
+YOCO_DEV void mma_16816(float *c, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+YOCO_DEV uint32_t pack2_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+YOCO_DEV float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const DecodeKParams p) {
+    if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
+    static_assert(G >= 1 && G <= 8, "query heads per KV head");
+    extern __shared__ __align__(128) unsigned char smem[];
+    const uint32_t head_bytes = D * 2;
+    const uint32_t row_bytes = (uint32_t)p.Hkv * head_bytes;  // one token, every KV head
+    const uint32_t RS = row_bytes + 16;                        // padded shared row stride
+    const uint32_t half = (uint32_t)p.stage_tokens * RS;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)p.stages * 2 * half);
+    uint64_t *empty = full + p.stages;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(p.v);
+    const int64_t row_elems = (int64_t)p.Hkv * D;
+    const int64_t total_units = (int64_t)p.B * p.n_split;
+    const uint32_t smem0 = smem_u32(smem);
+    uint32_t it = 0;
+
+    for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x) {
+        const int b = (int)(u / p.n_split);
+        const int64_t s = u % p.n_split;
+        const int64_t len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
+        const int64_t t0 = s * p.split;
+        if (t0 >= len) continue;
+        const int64_t n_tok = min(p.split, len - t0);
+        const int64_t row0 = (p.seq_start ? p.seq_start[b] : (int64_t)b * p.window) + t0;
+        const int n_st = (int)((n_tok + p.stage_tokens - 1) / p.stage_tokens);
+
+        if (warp == kConsumerWarps) {
+            // ---------------------------------------------------- producer
+            // One bulk copy per token row and tensor; the copies of a stage are
+            // spread over the warp's lanes, since one thread issuing many small
+            // copies cannot keep HBM busy.
+            for (int i = 0; i < n_st; ++i) {
+                const uint32_t itg = it + i;
+                const int st = (int)(itg % p.stages);
+                const uint32_t ph = (itg / p.stages) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u, &g_status_decode))) {
+                    if (lane == 0) producer_drain(full, it + i, p.stages);
+                    return;
+                }
+                const int cnt = (int)min(p.stage_tokens, n_tok - (int64_t)i * p.stage_tokens);
+                unsigned char *sk = smem + (size_t)st * 2 * half;
+                const int64_t r = row0 + (int64_t)i * p.stage_tokens;
+                if (lane == 0) mbar_arrive_expect_tx(&full[st], 2u * (uint32_t)cnt * row_bytes);
+                __syncwarp();
+                for (int c = lane; c < 2 * cnt; c += 32) {
+                    const int tk = c >> 1;
+                    if (c & 1)
+                        bulk_g2s(sk + half + (size_t)tk * RS, vg + (r + tk) * row_elems, row_bytes,
+                                 &full[st]);
+                    else
+                        bulk_g2s(sk + (size_t)tk * RS, kg + (r + tk) * row_elems, row_bytes, &full[st]);
+                }
+            }
+        } else {
+            // --------------------------------------------------- consumers
+            const int g = warp % p.Hkv;      // KV head
+            const int j = warp / p.Hkv;      // 16-token subset of every stage
+            const int gq = lane >> 2;        // fragment row: query head of the group
+            const int t = lane & 3;
+            const int64_t pos_b = p.pos ? p.pos[b] : 0;
+            const int32_t *sp = p.slot_pos ? p.slot_pos + (int64_t)b * p.window + t0 : nullptr;
+
+            uint32_t qa[D / 16][2];
+            if (gq < G) {
+                const __nv_bfloat16 *qr = static_cast<const __nv_bfloat16 *>(p.q) +
+                                          ((int64_t)b * p.Hq + (int64_t)g * G + gq) * D;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    qa[kk][0] = *reinterpret_cast<const uint32_t *>(qr + 16 * kk + 2 * t);
+                    qa[kk][1] = *reinterpret_cast<const uint32_t *>(qr + 16 * kk + 8 + 2 * t);
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) qa[kk][0] = qa[kk][1] = 0u;
+            }
+            float o[D / 8][4];
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            float m = -INFINITY, l = 0.f;
+            const int tok0 = j * kTokPerWarp;
+
+            for (int i = 0; i < n_st; ++i) {
+                const uint32_t itg = it + i;
+                const int st = (int)(itg % p.stages);
+                const uint32_t ph = (itg / p.stages) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph, &g_status_decode))) return;
+                const uint32_t kb = smem0 + (uint32_t)st * 2 * half + (uint32_t)g * head_bytes;
+                const uint32_t vb = kb + half;
+                const int64_t base_tok = (int64_t)i * p.stage_tokens + tok0;
+                const int cnt = (int)min(p.stage_tokens, n_tok - (int64_t)i * p.stage_tokens);
+                if (cnt < p.stage_tokens) {
+                    // rows past the unit's end hold stale bytes: zero this head's V
+                    // part of them so that 0-weight rows add exact zeros
+                    for (int idx = lane; idx < kTokPerWarp * (D / 8); idx += 32) {
+                        const int lt = tok0 + idx / (D / 8);
+                        if (lt >= cnt) {
+                            unsigned char *dst = smem + (size_t)st * 2 * half + half +
+                                                 (size_t)lt * RS + (size_t)g * head_bytes +
+                                                 (size_t)(idx % (D / 8)) * 16;
+                            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                    __syncwarp();
+                }
+
+                float sc[2][4];
+#pragma unroll
+                for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+                {
+                    const int mat = lane >> 3, rr = lane & 7;
+                    const uint32_t rowa = kb + (uint32_t)(tok0 + 8 * (mat >> 1) + rr) * RS;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(rowa + (uint32_t)(2 * kk + (mat & 1)) * 16, b0, b1, b2, b3);
+                        mma_16816(sc[0], qa[kk][0], qa[kk][1], b0, b1);
+                        mma_16816(sc[1], qa[kk][0], qa[kk][1], b2, b3);
+                    }
+                }
+                float pv[2][2];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int n = 0; n < 2; ++n) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int lt = 8 * n + 2 * t + e;
+                        const int64_t tok = base_tok + lt;
+                        bool vld = tok < n_tok;
+                        if (vld && sp) {
+                            const int32_t sp_t = sp[tok];
+                            vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window;
+                        }
+                        const float v = vld ? sc[n][e] * p.scale_log2 : -INFINITY;
+                        pv[n][e] = v;
+                        mx = fmaxf(mx, v);
+                    }
+                }
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                if (mx > m + 8.f) {
+                    // move the reference max only when it grows by more than 2^8
+                    const float alpha = (m == -INFINITY) ? 0.f : ex2f(m - mx);
+                    m = mx;
+                    l *= alpha;
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n) {
+                        o[n][0] *= alpha;
+                        o[n][1] *= alpha;
+                    }
+                }
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                const float p00 = ex2f(pv[0][0] + neg_m), p01 = ex2f(pv[0][1] + neg_m);
+                const float p10 = ex2f(pv[1][0] + neg_m), p11 = ex2f(pv[1][1] + neg_m);
+                l += (p00 + p01) + (p10 + p11);
+                const uint32_t a0 = pack2_bf16(p00, p01);
+                const uint32_t a2 = pack2_bf16(p10, p11);
+                {
+                    const int mat = lane >> 3, rr = lane & 7;
+                    const uint32_t rowa = vb + (uint32_t)(tok0 + 8 * (mat & 1) + rr) * RS +
+                                          (uint32_t)(mat >> 1) * 16;
+#pragma unroll
+                    for (int n = 0; n < D / 8; n += 2) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(rowa + (uint32_t)n * 16, b0, b1, b2, b3);
+                        mma_16816(o[n], a0, a2, b0, b1);
+                        mma_16816(o[n + 1], a0, a2, b2, b3);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
+
+            // l over the quad of lanes that share a row; o columns are disjoint
+            l += __shfl_xor_sync(0xffffffffu, l, 1);
+            l += __shfl_xor_sync(0xffffffffu, l, 2);
+            const int64_t entry = ((int64_t)b * p.n_split + s) * p.sub + j;
+            if (gq < G) {
+                const int64_t hq = (int64_t)g * G + gq;
+                float *dst = p.ws_o + (entry * p.Hq + hq) * D;
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n)
+                    *reinterpret_cast<float2 *>(dst + 8 * n + 2 * t) = make_float2(o[n][0], o[n][1]);
+                if (t == 0) {
+                    p.ws_ml[(entry * p.Hq + hq) * 2 + 0] = m;
+                    p.ws_ml[(entry * p.Hq + hq) * 2 + 1] = l;
+                }
+            }
+        }
+        it += (uint32_t)n_st;
+    }
+    if (warp == kConsumerWarps && lane == 0) producer_drain(full, it, p.stages);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const float *ws_o, const float *ws_ml,
                                                            const int32_t *seq_len, int32_t window,
@@ -329,7 +579,11 @@ bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dt
     per = ((per + pl.stage_tokens - 1) / pl.stage_tokens) * pl.stage_tokens;
     pl.split = std::max(per, min_split);
     pl.n_split = (max_len + pl.split - 1) / pl.split;
-    const size_t stage_bytes = 2 * (size_t)kRowsPerStage * D * dtype_bytes(dtype);
+    // fp32: 128 packed rows of [D] per tensor; bf16 (tensor-core kernel): one
+    // padded row of [Hkv, D] + 16 bytes per token per tensor
+    const size_t stage_bytes =
+        dtype == kBF16 ? 2 * (size_t)pl.stage_tokens * ((size_t)Hkv * D * 2 + 16)
+                       : 2 * (size_t)kRowsPerStage * D * dtype_bytes(dtype);
     pl.stages = (int)std::max<size_t>(1, std::min<size_t>(4, (200 * 1024) / stage_bytes));
     pl.smem_bytes = pl.stages * stage_bytes + 2 * pl.stages * sizeof(uint64_t);
     const size_t entries = (size_t)B * pl.n_split * pl.sub * Hq;
@@ -348,7 +602,8 @@ int device_sm_count() {
 
 template <typename T, int D, int G>
 static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t st) {
-    auto kern = decode_split_kernel<T, D, G>;
+    auto kern = std::is_same<T, __nv_bfloat16>::value ? decode_mma_kernel<D, G>
+                                                      : decode_split_kernel<T, D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)pl.smem_bytes);
     if (e != cudaSuccess) return e;
