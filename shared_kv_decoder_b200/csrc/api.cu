@@ -44,6 +44,14 @@ yoco_status from_cuda(cudaError_t e) {
     return YOCO_ERR_CUDA;
 }
 
+// Projection dispatch: the tensor-core kernel where it applies, else CUDA cores.
+yoco_status run_linear(const LinearArgs &a, cudaStream_t s) {
+    const cudaError_t e = launch_linear_tc(a, s);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+    cudaGetLastError();
+    return from_cuda(launch_linear_simt(a, s));
+}
+
 // Attention prefill dispatch: bf16 goes to the tcgen05 kernel; fp32 (and any
 // bf16 shape that kernel was not built for) to the CUDA-core kernel.
 yoco_status run_prefill(const PrefillArgs &a, cudaStream_t s) {
@@ -95,7 +103,7 @@ yoco_status yoco_kv_project_blend(const void *x, int64_t n_tok, int32_t d_model,
     a.apply_ln = apply_ln ? 1 : 0; a.eps = ln_eps;
     a.out0 = k_out; a.out1 = v_out; a.base0 = k_base; a.base1 = v_base;
     a.w0 = w_k; a.w1 = w_v; a.dst_rows = dst_rows; a.dtype = cfg->dtype;
-    return from_cuda(launch_linear_simt(a, stream));
+    return run_linear(a, stream);
 }
 
 yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, int32_t d_out,
@@ -111,7 +119,7 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
     a.apply_ln = apply_ln ? 1 : 0; a.eps = ln_eps;
     a.out0 = out; a.out1 = nullptr; a.base0 = base; a.base1 = nullptr;
     a.w0 = base_w; a.w1 = 0.f; a.dst_rows = nullptr; a.dtype = dtype;
-    return from_cuda(launch_linear_simt(a, stream));
+    return run_linear(a, stream);
 }
 
 yoco_status yoco_swa_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t T,
@@ -227,7 +235,8 @@ double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_at
 
 yoco_status yoco_get_device_status(cudaStream_t stream) {
     const cudaError_t e = cudaStreamSynchronize(stream);
-    const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc();
+    const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc() |
+                           read_and_clear_status_project_tc();
     if (s) return YOCO_ERR_TIMEOUT;
     return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;
 }

@@ -92,10 +92,14 @@ struct LinearArgs {
     int32_t dtype;
 };
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
+// Tensor-core path (bf16, >= 512 tokens, output width a multiple of 256):
+// LayerNorm folded into the epilogue.  cudaErrorNotSupported otherwise.
+cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
 
 // Device status words of the translation units that hold bounded waits.
 unsigned int read_and_clear_status_decode();
 unsigned int read_and_clear_status_prefill_tc();
+unsigned int read_and_clear_status_project_tc();
 
 int device_sm_count();
 

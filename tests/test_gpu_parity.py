@@ -219,3 +219,38 @@ def test_linear_matches_oracle(cuda_lib, dtype):
     out = cuda_lib.linear(x.cuda(), w.cuda(), base.cuda(), 1.0, apply_ln=True)
     ref = oracle.project(x, w, True) + to_np(base)
     assert_close(out, ref, dtype, "out")
+
+
+# ------------------------------------------- tensor-core projection (n >= 512)
+@pytest.mark.parametrize("n,d,Hkv,D,mean,apply_ln", [
+    (1000, 512, 8, 128, 0.0, True),     # 8 row tiles of 127 with a ragged tail
+    (640, 1024, 2, 64, 0.0, True),      # one 256-wide output chunk holding K and V
+    (2048, 4096, 8, 128, 3.0, True),    # large row mean: exercises the LayerNorm fold
+    (777, 256, 4, 128, 0.0, False),
+])
+def test_kv_project_blend_tensor_core(cuda_lib, n, d, Hkv, D, mean, apply_ln):
+    x = (wl.normal((n, d), 730 + n, torch.float32) + mean).to(BF)
+    w = wl.normal((2 * Hkv * D, d), 731, BF, std=d ** -0.5)
+    kb = wl.normal((n, Hkv, D), 732, BF)
+    vb = wl.normal((n, Hkv, D), 733, BF)
+    k, v = cuda_lib.kv_project_blend(x.cuda(), w.cuda(), Hkv, D, kb.cuda(), vb.cuda(), 0.3, 0.7,
+                                     apply_ln=apply_ln)
+    rk, rv = oracle.kv_project_blend(x, w, Hkv, D, kb, vb, 0.3, 0.7, apply_ln=apply_ln)
+    assert_close(k, rk, BF, "k")
+    assert_close(v, rv, BF, "v")
+
+
+def test_kv_project_tensor_core_scatter(cuda_lib):
+    n, d, Hkv, D = 600, 512, 8, 128
+    rows = 1500
+    x = wl.normal((n, d), 740, BF)
+    w = wl.normal((2 * Hkv * D, d), 741, BF, std=d ** -0.5)
+    dst = torch.randperm(rows, generator=wl.gen(742))[:n].to(torch.int64)
+    kc = torch.full((rows, Hkv, D), 9.0, dtype=BF, device="cuda")
+    vc = torch.full((rows, Hkv, D), -9.0, dtype=BF, device="cuda")
+    cuda_lib.kv_project_blend(x.cuda(), w.cuda(), Hkv, D, dst_rows=dst.cuda(), k_out=kc, v_out=vc)
+    rk, rv = oracle.kv_project_blend(x, w, Hkv, D)
+    untouched = sorted(set(range(rows)) - set(dst.tolist()))
+    assert torch.all(kc[untouched] == 9.0) and torch.all(vc[untouched] == -9.0)
+    assert_close(kc[dst.cuda()], rk, BF, "k")
+    assert_close(vc[dst.cuda()], rv, BF, "v")
