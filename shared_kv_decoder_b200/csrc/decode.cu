@@ -44,7 +44,7 @@ constexpr int kTokPerWarp = 16;     // stage tokens handled by one consumer warp
 constexpr int kLanesPerTok = 8;
 constexpr int kTokPerPass = 32 / kLanesPerTok;
 constexpr int kPasses = kTokPerWarp / kTokPerPass;
-constexpr int64_t kTargetUnits = 148 * 8;
+constexpr int64_t kTargetUnits = 148 * 12;
 
 struct DecodeKParams {
     const void *q, *k, *v;
@@ -59,6 +59,41 @@ struct DecodeKParams {
     float scale_log2;
     float *ws_o, *ws_ml;
 };
+
+// The u-th non-empty unit, counting sequence by sequence (a sequence of len
+// tokens has ceil(len / split) units).  Computed by each warp with a
+// 32-sequence-wide prefix scan, so every CTA strides over the same compact
+// list and the ragged lengths spread evenly over the grid.  False when u is
+// past the last unit.
+static __device__ bool find_unit(const DecodeKParams &p, int64_t u, int *b_out, int64_t *s_out) {
+    const int lane = threadIdx.x & 31;
+    int64_t base = 0;
+    for (int b0 = 0; b0 < p.B; b0 += 32) {
+        const int b = b0 + lane;
+        int64_t len = 0;
+        if (b < p.B) len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
+        // never more units than the workspace plan holds (lengths above max_len
+        // are a caller error; their tail is not read)
+        const int64_t cnt = len > 0 ? min((len + p.split - 1) / p.split, p.n_split) : 0;
+        int64_t incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int64_t total = __shfl_sync(0xffffffffu, incl, 31);
+        if (u < base + total) {
+            const unsigned hit = __ballot_sync(0xffffffffu, base + incl > u);
+            const int src = __ffs(hit) - 1;
+            const int64_t excl = __shfl_sync(0xffffffffu, incl - cnt, src);
+            *b_out = b0 + src;
+            *s_out = u - base - excl;
+            return true;
+        }
+        base += total;
+    }
+    return false;
+}
 
 // Before the producer leaves, wait (bounded) until the copies of the last
 // `stages` iterations have landed, so no bulk copy is still writing into this
@@ -98,15 +133,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
 
     const T *kg = static_cast<const T *>(p.k);
     const T *vg = static_cast<const T *>(p.v);
-    const int64_t total_units = (int64_t)p.B * p.n_split;
     uint32_t it = 0;  // pipeline iteration counter shared by producer and consumers
 
-    for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x) {
-        const int b = (int)(u / p.n_split);
-        const int64_t s = u % p.n_split;
+    for (int64_t u = blockIdx.x;; u += gridDim.x) {
+        int b;
+        int64_t s;
+        if (!find_unit(p, u, &b, &s)) break;
         const int64_t len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
         const int64_t t0 = s * p.split;
-        if (t0 >= len) continue;
         const int64_t n_tok = min(p.split, len - t0);
         const int64_t row0 = (p.seq_start ? p.seq_start[b] : (int64_t)b * p.window) + t0;
         const int n_st = (int)((n_tok + p.stage_tokens - 1) / p.stage_tokens);
@@ -345,16 +379,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const Dec
     const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k);
     const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(p.v);
     const int64_t row_elems = (int64_t)p.Hkv * D;
-    const int64_t total_units = (int64_t)p.B * p.n_split;
     const uint32_t smem0 = smem_u32(smem);
     uint32_t it = 0;
 
-    for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x) {
-        const int b = (int)(u / p.n_split);
-        const int64_t s = u % p.n_split;
+    for (int64_t u = blockIdx.x;; u += gridDim.x) {
+        int b;
+        int64_t s;
+        if (!find_unit(p, u, &b, &s)) break;
         const int64_t len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
         const int64_t t0 = s * p.split;
-        if (t0 >= len) continue;
         const int64_t n_tok = min(p.split, len - t0);
         const int64_t row0 = (p.seq_start ? p.seq_start[b] : (int64_t)b * p.window) + t0;
         const int n_st = (int)((n_tok + p.stage_tokens - 1) / p.stage_tokens);
