@@ -13,18 +13,23 @@
 // keys of the matching KV head.  Warp roles:
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  For each KV
 //              tile it reads S from TMEM, masks (diagonal / window / tail tiles
-//              only), takes the row max, computes P = 2^(S*scale*log2e - m) in
-//              fp32, writes P as bf16 into shared memory in the UMMA K-major
-//              128-byte-swizzled layout and signals the MMA warp.  The running
-//              max is only moved (and O in TMEM rescaled) when it grows by more
-//              than 2^8, which keeps O exact after the final 1/l.
+//              only), takes the row max (3-input max tree), computes
+//              P = 2^(S*scale*log2e - m) in fp32 on packed pairs -- half the
+//              exponentials on MUFU, half on an FMA-pipe polynomial -- and
+//              writes P as bf16 pairs back into TMEM (two P buffers).  The
+//              running max is only moved (and O in TMEM rescaled) when it grows
+//              by more than 2^8, which keeps O exact after the final 1/l.
 //   warp 4     TMA producer: lane 0 loads Q then K tiles, lane 1 V tiles,
-//              into a two-deep ring each (mbarrier complete_tx).
+//              into a three-deep ring each (mbarrier complete_tx).
 //   warp 5     MMA issuer (one thread): S_t = Q K_t^T into one of two TMEM S
 //              buffers, issued one tile ahead so the tensor core computes
 //              S_{t+1} while the softmax works on S_t; then O += P_t V_t with
-//              V read MN-major straight from its TMA tile.
-// TMEM: S0 [128 x 128] fp32, S1, O [128 x D] fp32 (512 columns allocated).
+//              P read from TMEM (A operand in tensor memory) and V read
+//              MN-major straight from its TMA tile.  Keeping P out of shared
+//              memory matters: at N = 128 the operand reads of one MMA already
+//              use the whole shared-memory bandwidth.
+// TMEM: S0, S1 [128 x 128] fp32, O [128 x D] fp32, P0, P1 [128 x 128] bf16
+// (512 columns allocated).
 // Every mbarrier wait is bounded; a wait that gives up sets the status word,
 // and all roles then fall through to the common exit, which waits for issued
 // copies and MMAs before freeing TMEM.
@@ -50,11 +55,11 @@ template <int D>
 struct Smem {
     static constexpr int KB = D / 64;                  // 64-element column blocks
     static constexpr uint32_t TILE = (uint32_t)KB * kBlk;
+    static constexpr int STAGES = 3;
     static constexpr uint32_t Q = 0;
-    static constexpr uint32_t K = Q + TILE;            // 2 stages
-    static constexpr uint32_t V = K + 2 * TILE;        // 2 stages
-    static constexpr uint32_t P = V + 2 * TILE;        // 2 blocks (128 keys)
-    static constexpr uint32_t BAR = P + 2 * kBlk;
+    static constexpr uint32_t K = Q + TILE;            // STAGES stages
+    static constexpr uint32_t V = K + STAGES * TILE;   // STAGES stages
+    static constexpr uint32_t BAR = V + STAGES * TILE;
     static constexpr uint32_t BYTES = BAR + 256;
     static constexpr uint32_t ALLOC = BYTES + 1024;    // alignment slack
 };
@@ -71,15 +76,15 @@ struct TcParams {
 
 enum Bar {
     kQFull = 0,
-    kKFull = 1,   // 2
-    kKEmpty = 3,  // 2
-    kVFull = 5,   // 2
-    kVEmpty = 7,  // 2
-    kSFull = 9,   // 2
-    kPFull = 11,
-    kODone = 12,
-    kDrain = 13,
-    kNumBars = 14
+    kKFull = 1,   // 3
+    kKEmpty = 4,  // 3
+    kVFull = 7,   // 3
+    kVEmpty = 10, // 3
+    kSFull = 13,  // 2
+    kPFull = 15,  // 2: P buffer t&1 written (tile t)
+    kODone = 17,  // 2: P.V of tile u (P buffer u&1) finished
+    kDrain = 19,
+    kNumBars = 20
 };
 
 YOCO_DEV bool wait1(uint64_t *bar, uint32_t parity) {
@@ -122,15 +127,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kQFull], 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < L::STAGES; ++s) {
             mbar_init(&bars[kKFull + s], 1);
             mbar_init(&bars[kKEmpty + s], 1);
             mbar_init(&bars[kVFull + s], 1);
             mbar_init(&bars[kVEmpty + s], 1);
-            mbar_init(&bars[kSFull + s], 1);
         }
-        mbar_init(&bars[kPFull], 128);
-        mbar_init(&bars[kODone], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kSFull + s], 1);
+            mbar_init(&bars[kPFull + s], 128);
+            mbar_init(&bars[kODone + s], 1);
+        }
         mbar_init(&bars[kDrain], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -143,8 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448) P1 [448,512)
     const uint32_t tS0 = tmem, tS1 = tmem + 128;
     const uint32_t tO = tmem + 256;
+    const uint32_t tP0 = tmem + 384, tP1 = tmem + 448;
 
     if (warp == 4) {
         // ------------------------------------------------------ TMA producer
@@ -154,8 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < KB; ++kb)
                 tc::tma_load_4d(base + L::Q + kb * kBlk, &tm_q, kb * 64, h, (int)i0, b, &bars[kQFull]);
             for (int t = 0; t < n_kv; ++t) {
-                const int st = t & 1;
-                if (!wait1(&bars[kKEmpty + st], ((t >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+                const int st = t % L::STAGES;
+                if (!wait1(&bars[kKEmpty + st], ((t / L::STAGES) & 1) ^ 1)) { *abort_flag = 1; break; }
                 if (*abort_flag) break;
                 mbar_arrive_expect_tx(&bars[kKFull + st], BN * D * 2);
                 const int j0 = (jt_lo + t) * BN;
@@ -165,14 +174,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++issued;
             }
             // drain: the last copies issued must land before this CTA may exit
-            for (int t = max(0, issued - 2); t < issued; ++t)
-                if (!wait1(&bars[kKFull + (t & 1)], (t >> 1) & 1)) break;
+            for (int t = max(0, issued - L::STAGES); t < issued; ++t)
+                if (!wait1(&bars[kKFull + t % L::STAGES], (t / L::STAGES) & 1)) break;
             wait1(&bars[kQFull], 0);
         } else if (lane == 1) {
             int issued = 0;
             for (int t = 0; t < n_kv; ++t) {
-                const int st = t & 1;
-                if (!wait1(&bars[kVEmpty + st], ((t >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+                const int st = t % L::STAGES;
+                if (!wait1(&bars[kVEmpty + st], ((t / L::STAGES) & 1) ^ 1)) { *abort_flag = 1; break; }
                 if (*abort_flag) break;
                 mbar_arrive_expect_tx(&bars[kVFull + st], BN * D * 2);
                 const int j0 = (jt_lo + t) * BN;
@@ -181,8 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     &bars[kVFull + st]);
                 ++issued;
             }
-            for (int t = max(0, issued - 2); t < issued; ++t)
-                if (!wait1(&bars[kVFull + (t & 1)], (t >> 1) & 1)) break;
+            for (int t = max(0, issued - L::STAGES); t < issued; ++t)
+                if (!wait1(&bars[kVFull + t % L::STAGES], (t / L::STAGES) & 1)) break;
         }
     } else if (warp == 5) {
         // ---------------------------------------------------------- MMA issue
@@ -191,23 +200,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idPV = tc::idesc_bf16(BM, D, false, true);
             bool ok = wait1(&bars[kQFull], 0);
             auto issue_pv = [&](int u) -> bool {
-                if (!wait1(&bars[kPFull], u & 1)) return false;
-                if (!wait1(&bars[kVFull + (u & 1)], (u >> 1) & 1)) return false;
+                const int vs = u % L::STAGES;
+                if (!wait1(&bars[kPFull + (u & 1)], (u >> 1) & 1)) return false;
+                if (!wait1(&bars[kVFull + vs], (u / L::STAGES) & 1)) return false;
                 tc::fence_after_sync();
-                const uint32_t vb = base + L::V + (u & 1) * L::TILE;
+                const uint32_t vb = base + L::V + vs * L::TILE;
+                const uint32_t tp = (u & 1) ? tP1 : tP0;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t ad = tc::smem_desc_sw128(base + L::P + (kk >> 2) * kBlk + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = tc::smem_desc_sw128(vb + kk * 2048, kBlk, 1024);
-                    tc::mma_bf16_ss(tO, ad, bd, idPV, (u > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_bf16_ts(tO, tp + kk * 8, bd, idPV, (u > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc::mma_commit(&bars[kVEmpty + (u & 1)]);
-                tc::mma_commit(&bars[kODone]);
+                tc::mma_commit(&bars[kVEmpty + vs]);
+                tc::mma_commit(&bars[kODone + (u & 1)]);
                 return true;
             };
             for (int t = 0; ok && t < n_kv; ++t) {
-                const int st = t & 1;
-                if (!wait1(&bars[kKFull + st], (t >> 1) & 1) || *abort_flag) { ok = false; break; }
+                const int st = t % L::STAGES;
+                if (!wait1(&bars[kKFull + st], (t / L::STAGES) & 1) || *abort_flag) { ok = false; break; }
                 tc::fence_after_sync();
                 const uint32_t kbase = base + L::K + st * L::TILE;
 #pragma unroll
@@ -254,9 +264,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     s[c] = vis ? s[c] : -INFINITY;
                 }
             }
-            float mx = s[0];
+            // row max: 3-input max tree, eight independent chains
+            float a8[8];
 #pragma unroll
-            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            for (int k = 0; k < 8; ++k) a8[k] = tc::max3(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+            for (int c = 24; c < 120; c += 16)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a8[k] = tc::max3(a8[k], s[c + k], s[c + 8 + k]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a8[k] = fmaxf(a8[k], s[120 + k]);
+            const float mx = tc::max3(tc::max3(a8[0], a8[1], a8[2]), tc::max3(a8[3], a8[4], a8[5]),
+                                      fmaxf(a8[6], a8[7]));
             const float m_cand = mx * p.scale_log2;
             float alpha = 1.f;
             const bool grow = m_cand > m + 8.f;
@@ -265,46 +284,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m = m_cand;
             }
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            float rs = 0.f;
+            // P = 2^(S * scale * log2e - m): scale on packed pairs; exponentials
+            // split between MUFU (columns with bit 4 clear) and the FMA-pipe
+            // polynomial (bit 4 set)
+            const uint64_t sl2 = tc::f2_pack(p.scale_log2, p.scale_log2);
+            const uint64_t nm2 = tc::f2_pack(neg_m, neg_m);
+            uint64_t rs2a = 0, rs2b = 0;
 #pragma unroll
             for (int c = 0; c < BN; c += 2) {
-                const float e0 = tc::ex2(fmaf(s[c], p.scale_log2, neg_m));
-                const float e1 = tc::ex2(fmaf(s[c + 1], p.scale_log2, neg_m));
-                rs += e0 + e1;
+                float x0, x1, e0, e1;
+                tc::f2_unpack(tc::f2_fma(tc::f2_pack(s[c], s[c + 1]), sl2, nm2), x0, x1);
+                if ((c & 16) == 0) {
+                    e0 = tc::ex2(x0);
+                    e1 = tc::ex2(x1);
+                } else {
+                    tc::exp2_pair_poly(x0, x1, e0, e1);
+                }
+                if (c & 2)
+                    rs2b = tc::f2_add(rs2b, tc::f2_pack(e0, e1));
+                else
+                    rs2a = tc::f2_add(rs2a, tc::f2_pack(e0, e1));
                 pk[c / 2] = tc::pack_bf16x2(e0, e1);
             }
-            l = l * alpha + rs;
-            if (t >= 1) {
-                // P buffer and O are free once the previous P.V has finished
-                if (!waitw(&bars[kODone], (t - 1) & 1)) { ok = false; break; }
+            float ra0, ra1, rb0, rb1;
+            tc::f2_unpack(rs2a, ra0, ra1);
+            tc::f2_unpack(rs2b, rb0, rb1);
+            l = l * alpha + ((ra0 + ra1) + (rb0 + rb1));
+            // O must hold P_{t-1} V before it is rescaled
+            if (t >= 1 && __any_sync(0xffffffffu, grow)) {
+                if (!waitw(&bars[kODone + ((t - 1) & 1)], ((t - 1) >> 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
-                if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-                    for (int c = 0; c < D; c += 32) {
-                        float o[32];
-                        tc::tmem_ld32(tO + lane_off + c, o);
-                        tc::wait_ld();
+                for (int c = 0; c < D; c += 32) {
+                    float o[32];
+                    tc::tmem_ld32(tO + lane_off + c, o);
+                    tc::wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                        tc::tmem_st32(tO + lane_off + c, o);
-                    }
-                    tc::wait_st();
+                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                    tc::tmem_st32(tO + lane_off + c, o);
                 }
+                tc::wait_st();
             }
-            // P row r -> two 128-byte-swizzled K-major blocks (keys 0-63, 64-127)
-#pragma unroll
-            for (int c = 0; c < BN / 8; ++c) {
-                const uint32_t blk = base + L::P + (c >> 3) * kBlk;
-                const uint32_t addr = blk + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c]),
-                             "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                             : "memory");
+            // P buffer t&1 in TMEM is free once P_{t-2} V has finished
+            if (t >= 2) {
+                if (!waitw(&bars[kODone + (t & 1)], ((t - 2) >> 1) & 1)) { ok = false; break; }
             }
-            fence_proxy_async_smem();
+            // P row r (bf16 pairs) -> TMEM lane r, 64 columns of buffer t&1
+            const uint32_t tp = ((t & 1) ? tP1 : tP0) + lane_off;
+            tc::tmem_st32u(tp, pk);
+            tc::tmem_st32u(tp + 32, pk + 32);
+            tc::wait_st();
             tc::fence_before_sync();
-            mbar_arrive(&bars[kPFull]);
+            mbar_arrive(&bars[kPFull + (t & 1)]);
         }
-        if (ok && waitw(&bars[kODone], (n_kv - 1) & 1)) {
+        if (ok && waitw(&bars[kODone + ((n_kv - 1) & 1)], ((n_kv - 1) >> 1) & 1)) {
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +

@@ -111,6 +111,32 @@ YOCO_DEV void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uin
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x 16, bf16 pairs packed in 32-bit
+// columns, lane = row) read straight from tensor memory.
+YOCO_DEV void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit columns of this warp's 32 TMEM lanes from registers.
+YOCO_DEV void tmem_st32u(uint32_t taddr, const uint32_t *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
 // Arrive on an mbarrier when every tcgen05.mma issued so far by this thread completes.
 YOCO_DEV void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -132,6 +158,67 @@ YOCO_DEV float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+YOCO_DEV float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// ---------------------------------------------------- packed fp32 pairs
+YOCO_DEV uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+YOCO_DEV void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+YOCO_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+YOCO_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+YOCO_DEV uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__host__ __device__ constexpr uint64_t f2_const(uint32_t bits) {
+    return ((uint64_t)bits << 32) | bits;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe instead of MUFU, so that the
+// softmax can split its exponentials between the two units.  Method: Cody-Waite
+// range reduction -- n = round(x) by adding 1.5 * 2^23 (the rounded integer
+// lands in the low mantissa bits), f = x - n in [-1/2, 1/2] -- then 2^f from a
+// degree-3 polynomial whose coefficients are a relative-error minimax (Remez)
+// fit on [-1/2, 1/2] (max relative error 7.5e-5, far below the bf16 rounding
+// of P), and 2^n applied by adding n to the exponent field.  x is clamped to
+// -125 so the exponent never leaves the normal range (2^-125 stands in for 0).
+YOCO_DEV void exp2_pair_poly(float x0, float x1, float &e0, float &e1) {
+    constexpr uint64_t kRound = f2_const(0x4B400000u);  // 1.5 * 2^23
+    constexpr uint64_t kC0 = f2_const(1065352009u);     // 0.99992806
+    constexpr uint64_t kC1 = f2_const(1060206989u);     // 0.69326097
+    constexpr uint64_t kC2 = f2_const(1048080141u);     // 0.24261113
+    constexpr uint64_t kC3 = f2_const(1029831600u);     // 0.05517167
+    const uint64_t X = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t T = f2_add(X, kRound);
+    const uint64_t F = f2_sub(X, f2_sub(T, kRound));
+    uint64_t P = f2_fma(F, kC3, kC2);
+    P = f2_fma(P, F, kC1);
+    P = f2_fma(P, F, kC0);
+    float p0, p1, t0, t1;
+    f2_unpack(P, p0, p1);
+    f2_unpack(T, t0, t1);
+    e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 YOCO_DEV uint32_t pack_bf16x2(float lo, float hi) {
