@@ -14,9 +14,10 @@
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  For each KV
 //              tile it reads S from TMEM, masks (diagonal / window / tail tiles
 //              only), takes the row max (3-input max tree), computes
-//              P = 2^(S*scale*log2e - m) in fp32 on packed pairs -- half the
-//              exponentials on MUFU, half on an FMA-pipe polynomial -- and
-//              writes P as bf16 pairs back into TMEM (two P buffers).  The
+//              P = 2^(S*scale*log2e - m) in fp32 on packed pairs -- three
+//              quarters of the exponentials on MUFU, a quarter on an FMA-pipe
+//              polynomial -- and writes P as bf16 pairs back into TMEM (two P
+//              buffers).  The
 //              running max is only moved (and O in TMEM rescaled) when it grows
 //              by more than 2^8, which keeps O exact after the final 1/l.
 //   warp 4     TMA producer: lane 0 loads Q then K tiles, lane 1 V tiles,
@@ -285,8 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
             // P = 2^(S * scale * log2e - m): scale on packed pairs; exponentials
-            // split between MUFU (columns with bit 4 clear) and the FMA-pipe
-            // polynomial (bit 4 set)
+            // split between MUFU and the FMA-pipe polynomial (columns 48-63 and
+            // 112-127, a quarter: the split measured fastest, since MUFU and the
+            // issue slots then run out at about the same time)
             const uint64_t sl2 = tc::f2_pack(p.scale_log2, p.scale_log2);
             const uint64_t nm2 = tc::f2_pack(neg_m, neg_m);
             uint64_t rs2a = 0, rs2b = 0;
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < BN; c += 2) {
                 float x0, x1, e0, e1;
                 tc::f2_unpack(tc::f2_fma(tc::f2_pack(s[c], s[c + 1]), sl2, nm2), x0, x1);
-                if ((c & 16) == 0) {
+                if ((c & 48) != 48) {
                     e0 = tc::ex2(x0);
                     e1 = tc::ex2(x1);
                 } else {
