@@ -71,6 +71,19 @@ def load_peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
+def reduce_max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over every rank of the default
+    process group (identity without one): each rank runs an independent
+    replica, and the job is as slow as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def prefill_flops_per_layer(T, Hq, D, q_pos0=0, window=0):
     """4 * Hq * D * sum over query rows of the visible key count."""
     import numpy as np
@@ -459,11 +472,8 @@ def main():
     swa_ms = [pair(e, "swa") for e in evs]
     gkv_ms = [pair(e, "gkv") for e in evs]
 
-    tot = {"step": sum(step_ms), "pre": sum(pre_ms), "dec": sum(dec_ms)}
-    if world > 1:
-        t = torch.tensor([tot["step"], tot["pre"], tot["dec"]], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot = {"step": float(t[0]), "pre": float(t[1]), "dec": float(t[2])}
+    mx = reduce_max_over_ranks([sum(step_ms), sum(pre_ms), sum(dec_ms)], dev)
+    tot = {"step": mx[0], "pre": mx[1], "dec": mx[2]}
 
     f_layer = prefill_flops_per_layer(P["T"], P["Hq"], P["D"])
     value = world * args.steps * P["layers"] * f_layer / (tot["pre"] * 1e-3) / 1e12
@@ -503,11 +513,7 @@ def main():
     }
     if not args.no_e2e:
         times, h2d, d2h = e2e_prefill(W, args.steps, 1)
-        e2e_ms = sum(times)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        e2e_ms = reduce_max_over_ranks([sum(times)], dev)[0]
         out["e2e"] = {"value": world * len(times) * P["layers"] * f_layer / (e2e_ms * 1e-3) / 1e12,
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
