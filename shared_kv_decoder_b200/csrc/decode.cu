@@ -578,20 +578,31 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *ws_o, co
     float M = -INFINITY;
     for (int64_t e = lane; e < n_e; e += 32) M = fmaxf(M, ws_ml[((e0 + e) * Hq + h) * 2]);
     M = warp_max(M);
-    float L = 0.f;
+    // lanes compute the weights of 32 entries at a time; the weighted sum then
+    // walks those entries with several partial rows in flight per lane
+    float Lp = 0.f;
     constexpr int DPL = D / 32;
     float acc[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-    for (int64_t e = 0; e < n_e; ++e) {
-        const float me = ws_ml[((e0 + e) * Hq + h) * 2];
-        const float le = ws_ml[((e0 + e) * Hq + h) * 2 + 1];
-        const float w = (me == -INFINITY) ? 0.f : exp2f(me - M);
-        L += le * w;
-        const float *src = ws_o + ((e0 + e) * Hq + h) * D;
+    for (int64_t c = 0; c < n_e; c += 32) {
+        const int64_t e = c + lane;
+        float w = 0.f;
+        if (e < n_e) {
+            const float me = ws_ml[((e0 + e) * Hq + h) * 2];
+            w = (me == -INFINITY) ? 0.f : exp2f(me - M);
+            Lp = fmaf(ws_ml[((e0 + e) * Hq + h) * 2 + 1], w, Lp);
+        }
+        const int cnt = (int)min((int64_t)32, n_e - c);
+        const float *src = ws_o + ((e0 + c) * Hq + h) * D + lane;
+#pragma unroll 8
+        for (int k = 0; k < cnt; ++k) {
+            const float wk = __shfl_sync(0xffffffffu, w, k);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, src[lane + 32 * i], acc[i]);
+            for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wk, src[(int64_t)k * Hq * D + 32 * i], acc[i]);
+        }
     }
+    const float L = warp_sum(Lp);
     const float inv = L > 0.f ? 1.f / L : 0.f;
     T *dst = o + ((int64_t)b * Hq + h) * D;
 #pragma unroll
