@@ -254,3 +254,20 @@ def test_kv_project_tensor_core_scatter(cuda_lib):
     assert torch.all(kc[untouched] == 9.0) and torch.all(vc[untouched] == -9.0)
     assert_close(kc[dst.cuda()], rk, BF, "k")
     assert_close(vc[dst.cuda()], rv, BF, "v")
+
+
+@pytest.mark.parametrize("window", [0, 300])
+def test_prefill_huge_score_growth(cuda_lib, window):
+    # For some query rows, a key in a LATER KV tile scores far above everything
+    # seen before (hundreds of log2 units): the kernel must move its running
+    # reference max (redoing that tile) without overflow or loss.
+    B, T, Hq, Hkv, D = 1, 700, 8, 2, 128
+    G = Hq // Hkv
+    q, k, v = _qkv(B, T, T, Hq, Hkv, D, BF, 760)
+    for i, j in [(650, 600), (699, 520), (300, 290), (259, 257)]:
+        k[0, j] = (q[0, i].view(Hkv, G, D)[:, 0] * 20.0).to(BF)
+    o, lse = cuda_lib.cross_prefill(q.cuda(), k.cuda(), v.cuda(), want_lse=True) if window == 0 else \
+        cuda_lib.swa_prefill(q.cuda(), k.cuda(), v.cuda(), window, want_lse=True)
+    ro, rlse = oracle.attention(q, k, v, 0, window)
+    assert_close(o, ro, BF, "o")
+    assert_close(lse, rlse.transpose(0, 2, 1), BF, "lse", max_abs=2e-3, rel_l2=1e-4)
