@@ -43,7 +43,7 @@ WORKLOAD = ("cross-decoder causal prefill B=1 T=32768 32q/8kv D=128 x14 layers o
             "+ decode step B=16 ragged 64K-128K x16 layers + SWA/blend layer slice B=4 T=65536 W=1024")
 
 P = dict(T=32768, Hq=32, Hkv=8, D=128, layers=14, d=4096)          # cross prefill
-DEC = dict(B=16, lo=65536, hi=131072, Hq=32, Hkv=8, D=128, layers=16, d=4096)
+DEC = dict(B=16, lo=65536, hi=131072, Hq=32, Hkv=8, D=128, layers=16, d=4096, seed=2000)
 SWA = dict(B=4, T=65536, W=1024, Hq=32, Hkv=8, D=128, d=4096)
 
 
@@ -56,7 +56,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj"], default=None,
+    ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer"],
+                    default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
 
@@ -69,6 +70,29 @@ def load_peaks():
                     bf16_sus=float(d["bf16_tflops_sustained"]), src="measured")
     except Exception:
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# DRAM bytes (read + write) per launch of the roofline kernels, from one ncu
+# capture of the benchmark's own launch shape (--case prefill_layer /
+# decode_layer).  Each figure is keyed by the SHA-256 of the kernel source it
+# was taken on: once that source changes the figure no longer describes the
+# kernel, and the report carries null instead.
+TRAFFIC = {
+    "prefill": {"bytes": None, "source": "shared_kv_decoder_b200/csrc/prefill_tc.cu", "sha256": None},
+    "decode": {"bytes": None, "source": "shared_kv_decoder_b200/csrc/decode.cu", "sha256": None},
+}
+
+
+def traffic(kind):
+    import hashlib
+    t = TRAFFIC[kind]
+    if t["bytes"] is None:
+        return None
+    try:
+        h = hashlib.sha256(open(os.path.join(ROOT, t["source"]), "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return float(t["bytes"]) if h == t["sha256"] else None
 
 
 def reduce_max_over_ranks(values, device=None):
@@ -158,7 +182,7 @@ def make_workload(dev):
     W["qs"] = [wl.normal((1, T, Hq, D), 1200 + l, bf, dev) for l in range(P["layers"])]
     W["o"] = torch.empty((1, T, Hq, D), dtype=bf, device=dev)
     # decode: packed shared cache of 16 ragged sequences
-    lens = wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], 2000)
+    lens = wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], DEC["seed"])
     starts = torch.cumsum(torch.cat([torch.zeros(1, dtype=torch.int64), lens[:-1]]), 0)
     rows = int(lens.sum())
     W["lens"], W["starts"], W["rows"] = lens, starts, rows
@@ -360,6 +384,8 @@ def run_case(args):
       decode   cross decode, batch 16, lengths in [16384, 32768] (cache ~1.6 GB)
       swa      sliding-window prefill B=1, T=65536, window 1024 (Q 512 MB)
       proj     K/V projection + blend, 32768 tokens, d=4096 (x 256 MB)
+      prefill_layer / decode_layer  one launch of the full benchmark's own
+               prefill layer (T=32768) / decode layer (batch 16, 64K-128K)
     Prints one JSON line with the mean launch time and the work rate."""
     import torch
     import shared_kv_decoder_b200 as yoco
@@ -367,14 +393,15 @@ def run_case(args):
     bf, dev = torch.bfloat16, "cuda"
     yoco.load()
     Hq, Hkv, D = 32, 8, 128
-    if args.case == "prefill":
-        T = 16384
+    if args.case in ("prefill", "prefill_layer"):
+        T = 16384 if args.case == "prefill" else P["T"]
         q = wl.normal((1, T, Hq, D), 1, bf, dev); k = wl.normal((1, T, Hkv, D), 2, bf, dev)
         v = wl.normal((1, T, Hkv, D), 3, bf, dev); o = torch.empty_like(q)
         fn = lambda: yoco.cross_prefill(q, k, v, o=o)
         work, unit = prefill_flops_per_layer(T, Hq, D), "TFLOP/s"
-    elif args.case == "decode":
-        lens = wl.ragged_lengths(16, 16384, 32768, 9)
+    elif args.case in ("decode", "decode_layer"):
+        lens = (wl.ragged_lengths(16, 16384, 32768, 9) if args.case == "decode" else
+                wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], DEC["seed"]))
         starts = torch.cumsum(torch.cat([torch.zeros(1, dtype=torch.int64), lens[:-1]]), 0)
         rows = int(lens.sum())
         kc = wl.normal((rows, Hkv, D), 4, bf, dev); vc = wl.normal((rows, Hkv, D), 5, bf, dev)
@@ -502,11 +529,11 @@ def main():
         "gkv": {"ms": statistics.mean(gkv_ms), "tflops": gkv_fl / (statistics.mean(gkv_ms) * 1e-3) / 1e12},
         "roofline": {"kernel": "cross prefill (yoco_cross_prefill)", "bound": "tensor",
                      "achieved": pre_tflops_launch, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                     "frac": pre_tflops_launch / peaks["bf16_sus"], "traffic": None,
+                     "frac": pre_tflops_launch / peaks["bf16_sus"], "traffic": traffic("prefill"),
                      "peak_src": f"{peaks['src']} bf16 sustained"},
         "roofline_decode": {"kernel": "cross decode (yoco_cross_decode)", "bound": "hbm",
                             "achieved": dec_gbs_layer, "peak": peaks["hbm"], "unit": "GB/s",
-                            "frac": dec_gbs_layer / peaks["hbm"], "traffic": None,
+                            "frac": dec_gbs_layer / peaks["hbm"], "traffic": traffic("decode"),
                             "peak_src": f"{peaks['src']} hbm"},
         "gpu_launches": launches,
         "clocks": clk,

@@ -9,26 +9,26 @@
 // here, laid out for B200:
 //
 //  * A CTA owns one unit = a contiguous token range of one sequence for ALL
-//    KV heads, so each pipeline stage is ONE contiguous block of HBM
-//    (128 rows of [Hkv, D] K plus the same of V) moved by a single
-//    cp.async.bulk per tensor into a 2-4 deep shared-memory ring (mbarrier
-//    complete_tx).  A dedicated producer warp issues the copies; eight
-//    consumer warps compute.  Persistent grid: one CTA per SM strides over
-//    the units.
-//  * Consumer warp w serves KV head w % Hkv and a 16-token subset of each
-//    stage; its eight-lane groups each own one token and split the head dim
-//    in 16-byte chunks (conflict-free shared loads), with every query head
-//    of the GQA group held in registers, so K/V bytes are read once for all
-//    Hq/Hkv query heads.
-//  * Softmax is online in the exp2 domain, rescaled once per stage; every
-//    token group keeps its own running max, merged with the other groups at
-//    the end of the unit; the partial (m, l, o) goes to the workspace and a
-//    second kernel merges the splits (log-sum-exp weighting, one warp per
-//    (sequence, query head)).
+//    KV heads, so K/V bytes are read once for every query head of the GQA
+//    group.  Persistent grid: one CTA per SM strides over a compact list of
+//    the non-empty units.  One producer warp fills a shared-memory ring of
+//    stages (128 token-head rows of K and of V each); eight consumer warps
+//    compute, warp w serving KV head w % Hkv and a 16-token subset of every
+//    stage.
+//  * bf16 (decode_tma_kernel): each stage arrives as a few 16 KB TMA tensor
+//    boxes with the 128-byte swizzle; S = q K^T and O += P V are warp-wide
+//    mma.sync tiles with the group's query heads as the A rows.  fp32
+//    (decode_split_kernel) runs on the CUDA cores from one bulk copy per stage
+//    and tensor.
+//  * Softmax is online in the exp2 domain; the reference max only moves when
+//    it grows by more than 2^8.  The partial (m, l, o) of each unit goes to
+//    the workspace and a second kernel merges the splits (log-sum-exp
+//    weighting, one warp per (sequence, query head)).
 //  * Ring mode (self-decoder): the cache is the ring [B, window, Hkv, D] and
 //    a slot is visible when its stored position lies in (pos - window, pos].
 #include "common.cuh"
 #include "launch.h"
+#include "tc.cuh"
 
 #include <algorithm>
 #include <type_traits>
@@ -319,12 +319,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
 // per-head FMAs, eight-lane butterflies) and is issue-bound well below HBM
 // bandwidth.  Here the GQA group's query heads form the M rows of a
 // 16 x 16 A fragment (G <= 8 real rows), so S = q K^T and O += P V are a few
-// warp-wide MMAs per 16 tokens and the kernel is left waiting on HBM only.
-// Stage layout in shared memory: one row per token holding all KV heads,
-// with a 16-byte pad so that the eight consecutive token rows an ldmatrix
-// gathers fall in distinct bank groups; each token row is one bulk copy.
-// P goes from the S accumulators straight into the A fragment of P.V
-// (tokens 0-7 and 8-15 of the warp's 16 are the two S column tiles).
+// warp-wide MMAs per 16 tokens.  P goes from the S accumulators straight into
+// the A fragment of P.V (tokens 0-7 and 8-15 of the warp's 16 are the two S
+// column tiles).
 YOCO_DEV void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -354,18 +351,37 @@ YOCO_DEV float ex2f(float x) {
     return y;
 }
 
+// decode_tma_kernel: stages reach shared memory as TMA tensor copies.  The
+// cache is viewed as the tensor {D, token, KV head} (token stride Hkv*D, head
+// stride D), and one box {64, stage_tokens, Hkv} -- 16 KB, every head of the
+// stage's tokens for one 64-column block -- lands as 128-byte rows ordered
+// [head][token] under the 128-byte swizzle.  A stage is 2*D/64 such copies;
+// an earlier feed with one 2 KB bulk copy per token row and tensor (rows
+// padded by 16 bytes against bank conflicts) kept fewer bytes in flight and
+// streamed 9% slower.  For a head, the eight token rows one ldmatrix gathers
+// are consecutive swizzled rows, so they fall in eight different bank groups.
+// A stage that ends a sequence short of stage_tokens is not copied: no box
+// may read past the sequence (the cache's end is not known to the kernel), so
+// each consumer warp loads its own head's valid rows with plain loads and
+// zeroes the rest.
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const DecodeKParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    decode_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const DecodeKParams p) {
     if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
     static_assert(G >= 1 && G <= 8, "query heads per KV head");
-    extern __shared__ __align__(128) unsigned char smem[];
-    const uint32_t head_bytes = D * 2;
-    const uint32_t row_bytes = (uint32_t)p.Hkv * head_bytes;  // one token, every KV head
-    const uint32_t RS = row_bytes + 16;                        // padded shared row stride
-    const uint32_t half = (uint32_t)p.stage_tokens * RS;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)p.stages * 2 * half);
+    constexpr int KB = D / 64;                       // 64-column blocks per head row
+    constexpr uint32_t kBox = kRowsPerStage * 128;   // one box: 128 rows of 128 bytes
+    constexpr uint32_t kStage = 2 * KB * kBox;       // K boxes then V boxes
+    constexpr int kChunks = D / 8;                   // 16-byte chunks per head row
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;   // the swizzle repeats every 1024 bytes
+    unsigned char *smem = smem_raw + (sbase - raw);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)p.stages * kStage);
     uint64_t *empty = full + p.stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ST = (int)p.stage_tokens;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -378,8 +394,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const Dec
 
     const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k);
     const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(p.v);
-    const int64_t row_elems = (int64_t)p.Hkv * D;
-    const uint32_t smem0 = smem_u32(smem);
     uint32_t it = 0;
 
     for (int64_t u = blockIdx.x;; u += gridDim.x) {
@@ -390,13 +404,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const Dec
         const int64_t t0 = s * p.split;
         const int64_t n_tok = min(p.split, len - t0);
         const int64_t row0 = (p.seq_start ? p.seq_start[b] : (int64_t)b * p.window) + t0;
-        const int n_st = (int)((n_tok + p.stage_tokens - 1) / p.stage_tokens);
+        const int n_st = (int)((n_tok + ST - 1) / ST);
 
         if (warp == kConsumerWarps) {
             // ---------------------------------------------------- producer
-            // One bulk copy per token row and tensor; the copies of a stage are
-            // spread over the warp's lanes, since one thread issuing many small
-            // copies cannot keep HBM busy.
             for (int i = 0; i < n_st; ++i) {
                 const uint32_t itg = it + i;
                 const int st = (int)(itg % p.stages);
@@ -405,19 +416,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const Dec
                     if (lane == 0) producer_drain(full, it + i, p.stages);
                     return;
                 }
-                const int cnt = (int)min(p.stage_tokens, n_tok - (int64_t)i * p.stage_tokens);
-                unsigned char *sk = smem + (size_t)st * 2 * half;
-                const int64_t r = row0 + (int64_t)i * p.stage_tokens;
-                if (lane == 0) mbar_arrive_expect_tx(&full[st], 2u * (uint32_t)cnt * row_bytes);
-                __syncwarp();
-                for (int c = lane; c < 2 * cnt; c += 32) {
-                    const int tk = c >> 1;
-                    if (c & 1)
-                        bulk_g2s(sk + half + (size_t)tk * RS, vg + (r + tk) * row_elems, row_bytes,
-                                 &full[st]);
-                    else
-                        bulk_g2s(sk + (size_t)tk * RS, kg + (r + tk) * row_elems, row_bytes, &full[st]);
+                const int64_t r = row0 + (int64_t)i * ST;
+                if (lane == 0) {
+                    if (n_tok - (int64_t)i * ST >= ST) {
+                        const uint32_t dst = sbase + (uint32_t)st * kStage;
+                        mbar_arrive_expect_tx(&full[st], kStage);
+#pragma unroll
+                        for (int kb = 0; kb < KB; ++kb) {
+                            tc::tma_load_4d(dst + kb * kBox, &tm_k, kb * 64, (int)r, 0, 0, &full[st]);
+                            tc::tma_load_4d(dst + (KB + kb) * kBox, &tm_v, kb * 64, (int)r, 0, 0, &full[st]);
+                        }
+                    } else {
+                        mbar_arrive(&full[st]);  // short stage: the consumers load it
+                    }
                 }
+                __syncwarp();
             }
         } else {
             // --------------------------------------------------- consumers
@@ -446,44 +459,58 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const Dec
             for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
             float m = -INFINITY, l = 0.f;
             const int tok0 = j * kTokPerWarp;
+            // ldmatrix row addresses (byte offsets inside a box) and the swizzle
+            // term of each lane: S reads K rows tok0 + 8*(mat>>1) + rr, P.V reads
+            // V rows tok0 + 8*(mat&1) + rr; row R keeps chunk c at c ^ (R & 7)
+            const int mat = lane >> 3, rr = lane & 7;
+            const uint32_t rowS = (uint32_t)(g * ST + tok0 + 8 * (mat >> 1) + rr) * 128u;
+            const uint32_t xs = (uint32_t)((mat & 1) ^ rr);
+            const uint32_t rowP = (uint32_t)(g * ST + tok0 + 8 * (mat & 1) + rr) * 128u;
+            const uint32_t xp = (uint32_t)((mat >> 1) ^ rr);
 
             for (int i = 0; i < n_st; ++i) {
                 const uint32_t itg = it + i;
                 const int st = (int)(itg % p.stages);
                 const uint32_t ph = (itg / p.stages) & 1u;
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph, &g_status_decode))) return;
-                const uint32_t kb = smem0 + (uint32_t)st * 2 * half + (uint32_t)g * head_bytes;
-                const uint32_t vb = kb + half;
-                const int64_t base_tok = (int64_t)i * p.stage_tokens + tok0;
-                const int cnt = (int)min(p.stage_tokens, n_tok - (int64_t)i * p.stage_tokens);
-                if (cnt < p.stage_tokens) {
-                    // rows past the unit's end hold stale bytes: zero this head's V
-                    // part of them so that 0-weight rows add exact zeros
-                    for (int idx = lane; idx < kTokPerWarp * (D / 8); idx += 32) {
-                        const int lt = tok0 + idx / (D / 8);
-                        if (lt >= cnt) {
-                            unsigned char *dst = smem + (size_t)st * 2 * half + half +
-                                                 (size_t)lt * RS + (size_t)g * head_bytes +
-                                                 (size_t)(idx % (D / 8)) * 16;
-                            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t kst = sbase + (uint32_t)st * kStage;
+                const uint32_t vst = kst + KB * kBox;
+                const int64_t base_tok = (int64_t)i * ST + tok0;
+                const int cnt = (int)min((int64_t)ST, n_tok - (int64_t)i * ST);
+                if (cnt < ST) {
+                    // short stage: this warp's 16 rows of head g, valid ones from
+                    // global memory, the rest zero (0-weight rows then add exact zeros)
+                    const int64_t r = row0 + (int64_t)i * ST;
+                    for (int idx = lane; idx < kTokPerWarp * kChunks; idx += 32) {
+                        const int lt = tok0 + idx / kChunks, ch = idx % kChunks;
+                        const uint32_t R = (uint32_t)(g * ST + lt);
+                        const uint32_t off = (uint32_t)(ch >> 3) * kBox + R * 128u +
+                                             ((((uint32_t)ch & 7u) ^ (R & 7u)) << 4);
+                        uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+                        if (lt < cnt) {
+                            const int64_t e = ((r + lt) * p.Hkv + g) * D + ch * 8;
+                            kv = *reinterpret_cast<const uint4 *>(kg + e);
+                            vv = *reinterpret_cast<const uint4 *>(vg + e);
                         }
+                        *reinterpret_cast<uint4 *>(smem + (kst - sbase) + off) = kv;
+                        *reinterpret_cast<uint4 *>(smem + (vst - sbase) + off) = vv;
                     }
+                    // these generic-proxy writes precede the copy engine's next
+                    // writes into this stage
+                    fence_proxy_async_smem();
                     __syncwarp();
                 }
 
                 float sc[2][4];
 #pragma unroll
                 for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-                {
-                    const int mat = lane >> 3, rr = lane & 7;
-                    const uint32_t rowa = kb + (uint32_t)(tok0 + 8 * (mat >> 1) + rr) * RS;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(rowa + (uint32_t)(2 * kk + (mat & 1)) * 16, b0, b1, b2, b3);
-                        mma_16816(sc[0], qa[kk][0], qa[kk][1], b0, b1);
-                        mma_16816(sc[1], qa[kk][0], qa[kk][1], b2, b3);
-                    }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kst + (uint32_t)(kk >> 2) * kBox + rowS + (((uint32_t)((kk & 3) << 1) ^ xs) << 4),
+                            b0, b1, b2, b3);
+                    mma_16816(sc[0], qa[kk][0], qa[kk][1], b0, b1);
+                    mma_16816(sc[1], qa[kk][0], qa[kk][1], b2, b3);
                 }
                 float pv[2][2];
                 float mx = -INFINITY;
@@ -522,19 +549,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_mma_kernel(const Dec
                 l += (p00 + p01) + (p10 + p11);
                 const uint32_t a0 = pack2_bf16(p00, p01);
                 const uint32_t a2 = pack2_bf16(p10, p11);
-                {
-                    const int mat = lane >> 3, rr = lane & 7;
-                    const uint32_t rowa = vb + (uint32_t)(tok0 + 8 * (mat & 1) + rr) * RS +
-                                          (uint32_t)(mat >> 1) * 16;
 #pragma unroll
-                    for (int n = 0; n < D / 8; n += 2) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4_t(rowa + (uint32_t)n * 16, b0, b1, b2, b3);
-                        mma_16816(o[n], a0, a2, b0, b1);
-                        mma_16816(o[n + 1], a0, a2, b2, b3);
-                    }
+                for (int n = 0; n < D / 8; n += 2) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vst + (uint32_t)(n >> 3) * kBox + rowP + ((((uint32_t)n & 7u) ^ xp) << 4),
+                              b0, b1, b2, b3);
+                    mma_16816(o[n], a0, a2, b0, b1);
+                    mma_16816(o[n + 1], a0, a2, b2, b3);
                 }
-                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
@@ -623,13 +645,13 @@ bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dt
     per = ((per + pl.stage_tokens - 1) / pl.stage_tokens) * pl.stage_tokens;
     pl.split = std::max(per, min_split);
     pl.n_split = (max_len + pl.split - 1) / pl.split;
-    // fp32: 128 packed rows of [D] per tensor; bf16 (tensor-core kernel): one
-    // padded row of [Hkv, D] + 16 bytes per token per tensor
-    const size_t stage_bytes =
-        dtype == kBF16 ? 2 * (size_t)pl.stage_tokens * ((size_t)Hkv * D * 2 + 16)
-                       : 2 * (size_t)kRowsPerStage * D * dtype_bytes(dtype);
-    pl.stages = (int)std::max<size_t>(1, std::min<size_t>(4, (200 * 1024) / stage_bytes));
-    pl.smem_bytes = pl.stages * stage_bytes + 2 * pl.stages * sizeof(uint64_t);
+    // a stage holds 128 token-head rows of K and of V; the bf16 kernel adds
+    // 1 KB so that its swizzled stages can start on a 1024-byte boundary
+    const size_t stage_bytes = 2 * (size_t)kRowsPerStage * D * dtype_bytes(dtype);
+    pl.stages = (int)std::max<size_t>(1, std::min<size_t>(dtype == kBF16 ? 6 : 4,
+                                                          (200 * 1024) / stage_bytes));
+    pl.smem_bytes = pl.stages * stage_bytes + 2 * pl.stages * sizeof(uint64_t) +
+                    (dtype == kBF16 ? 1024 : 0);
     const size_t entries = (size_t)B * pl.n_split * pl.sub * Hq;
     pl.ws_bytes = entries * D * sizeof(float) + entries * 2 * sizeof(float);
     *plan = pl;
@@ -644,13 +666,35 @@ int device_sm_count() {
     return n;
 }
 
+// TMA view of a packed cache [rows, Hkv, D]: dimensions {D, token, head, 1},
+// box {64, stage_tokens, Hkv, 1}.  The token extent only has to cover every
+// row a full stage reads (the kernel never asks for a box past a sequence's
+// end); it is set to a 1 TiB span, beyond any device's memory.
+static bool make_cache_map(CUtensorMap *m, const void *cache, int Hkv, int D, int64_t stage_tokens) {
+    const uint64_t row_bytes = (uint64_t)Hkv * D * 2;
+    const uint64_t rows = std::min<uint64_t>((uint64_t)INT32_MAX, (1ull << 40) / row_bytes);
+    const uint64_t dims[4] = {(uint64_t)D, rows, (uint64_t)Hkv, 1};
+    const uint64_t strides[3] = {row_bytes, (uint64_t)D * 2, row_bytes};
+    const uint32_t box[4] = {64, (uint32_t)stage_tokens, (uint32_t)Hkv, 1};
+    return encode_bf16_map_4d(m, cache, dims, strides, box);
+}
+
+template <int D, int G>
+static cudaError_t launch_decode_tma(const DecodeArgs &a, const DecodePlan &pl, const DecodeKParams &p,
+                                     int grid, cudaStream_t st) {
+    CUtensorMap mk, mv;
+    if (!make_cache_map(&mk, a.k, a.Hkv, D, p.stage_tokens) ||
+        !make_cache_map(&mv, a.v, a.Hkv, D, p.stage_tokens))
+        return cudaErrorNotSupported;
+    auto kern = decode_tma_kernel<D, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kDecodeThreads, pl.smem_bytes, st>>>(mk, mv, p);
+    return cudaGetLastError();
+}
+
 template <typename T, int D, int G>
 static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t st) {
-    auto kern = std::is_same<T, __nv_bfloat16>::value ? decode_mma_kernel<D, G>
-                                                      : decode_split_kernel<T, D, G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)pl.smem_bytes);
-    if (e != cudaSuccess) return e;
     DecodeKParams p;
     p.q = a.q; p.k = a.k; p.v = a.v;
     p.seq_start = a.seq_start; p.seq_len = a.seq_len;
@@ -664,9 +708,17 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
     p.ws_ml = p.ws_o + entries * D;
     const int64_t units = (int64_t)a.B * pl.n_split;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, device_sm_count()));
-    kern<<<grid, kDecodeThreads, pl.smem_bytes, st>>>(p);
+    cudaError_t e;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        e = launch_decode_tma<D, G>(a, pl, p, grid, st);
+    } else {
+        auto kern = decode_split_kernel<T, D, G>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kDecodeThreads, pl.smem_bytes, st>>>(p);
+        e = cudaGetLastError();
+    }
     note_launches(2);
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int mgrid = (int)(((int64_t)a.B * a.Hq + 3) / 4);
     decode_merge_kernel<T, D><<<mgrid, 128, 0, st>>>(p.ws_o, p.ws_ml, a.seq_len, a.window, a.B,

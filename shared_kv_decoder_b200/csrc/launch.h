@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+struct CUtensorMap_st;  // cuda.h's TMA descriptor (CUtensorMap)
+
 namespace yoco {
 
 enum Dtype { kBF16 = 0, kFP32 = 1 };
@@ -102,6 +104,11 @@ unsigned int read_and_clear_status_prefill_tc();
 unsigned int read_and_clear_status_project_tc();
 
 int device_sm_count();
+
+// A 4-D bf16 tensor map (innermost dimension first, strides of dimensions 1-3
+// in bytes) with the 128-byte swizzle; false when the driver rejects it.
+bool encode_bf16_map_4d(::CUtensorMap_st *m, const void *ptr, const uint64_t dims[4],
+                        const uint64_t strides_bytes[3], const uint32_t box[4]);
 
 // Host-side count of kernel launches (reported by yoco_launch_count()).
 void note_launches(int n);
