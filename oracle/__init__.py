@@ -54,6 +54,7 @@ def load(path):
     L.oracle_cache_bytes_yoco.restype = dbl
     L.oracle_cache_bytes_transformer.argtypes = [i64, i64, i64, i64, i64]
     L.oracle_cache_bytes_transformer.restype = dbl
+    L.oracle_visibility.argtypes = [i64, i64, i64, i64, ctypes.POINTER(ctypes.c_uint8)]
     L.oracle_num_threads.restype = i32
     L.oracle_set_num_threads.argtypes = [i32]
     return L
@@ -133,6 +134,14 @@ def kv_project_blend(x, w_kv, Hkv, D, k_base=None, v_base=None, w_k=0.0, w_v=0.0
     if v_base is not None:
         v = blend(v, _f64(v_base).reshape(n, Hkv, D), w_v)
     return k, v
+
+
+def visibility(Tq, Tkv, q_pos0=0, window=0):
+    """Boolean [Tq, Tkv]: key j visible to query row i at absolute position
+    q_pos0 + i (causal; within the window when window > 0)."""
+    out = np.zeros((Tq, Tkv), dtype=np.uint8)
+    lib().oracle_visibility(Tq, Tkv, q_pos0, window, out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return out.astype(bool)
 
 
 def attention(q, k, v, q_pos0=0, window=0, scale=None, rows=None):

@@ -111,6 +111,14 @@ static int visible(int64_t j, int64_t p, int64_t window) {
     return 1;
 }
 
+/* The visibility matrix itself: out[i * Tkv + j] = 1 when key j is visible to
+ * query row i (absolute position q_pos0 + i), by the rule above.  Used to
+ * check the kernels' tile plans, not by the attention functions below. */
+void oracle_visibility(int64_t Tq, int64_t Tkv, int64_t q_pos0, int64_t window, unsigned char *out) {
+    for (int64_t i = 0; i < Tq; ++i)
+        for (int64_t j = 0; j < Tkv; ++j) out[i * Tkv + j] = (unsigned char)visible(j, q_pos0 + i, window);
+}
+
 /* Softmax attention of one query vector over n_keys candidate key rows.
  * key(t) / val(t) are rows at (base + t * stride); mask[t] != 0 if visible.
  * Two passes: max of the visible scores, then exp-sum and weighted sum.

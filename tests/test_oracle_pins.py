@@ -227,6 +227,23 @@ def test_decode_step_equals_prefill_row():
         np.testing.assert_array_equal(lse[b], lfull[b, lens[b] - 1])
 
 
+# ---------------------------------------------------------------- visibility
+@pytest.mark.parametrize("Tq,Tkv,q_pos0,W", [(5, 5, 0, 0), (7, 12, 5, 0), (9, 9, 0, 3), (6, 20, 14, 4),
+                                             (4, 10, 6, 100), (1, 1, 0, 1)])
+def test_visibility_is_a_shifted_band(Tq, Tkv, q_pos0, W):
+    # causal: numpy's lower triangle shifted by the chunk offset; window W:
+    # that triangle minus the one W diagonals further down
+    m = oracle.visibility(Tq, Tkv, q_pos0, W)
+    expect = np.tril(np.ones((Tq, Tkv), dtype=bool), k=q_pos0)
+    if W > 0:
+        expect &= ~np.tril(np.ones((Tq, Tkv), dtype=bool), k=q_pos0 - W)
+    np.testing.assert_array_equal(m, expect)
+    # row counts: min(p + 1, W) keys for the query at absolute position p
+    p = np.arange(Tq) + q_pos0
+    cnt = np.minimum(p + 1, Tkv) if W <= 0 else np.minimum(np.minimum(p + 1, W), Tkv)
+    np.testing.assert_array_equal(m.sum(1), cnt)
+
+
 # ---------------------------------------------------------------------- ring
 @pytest.mark.parametrize("T,W", [(0, 4), (3, 4), (4, 4), (5, 4), (17, 4), (1000, 32), (31, 32)])
 def test_ring_slots_closed_form(T, W):
