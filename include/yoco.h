@@ -174,6 +174,34 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
                         int32_t apply_ln, float ln_eps, const void *base, float base_w,
                         void *out, int32_t dtype, cudaStream_t stream);
 
+/* Test-only, with no counterpart on the pages: the work plan the kernels
+ * follow, computed on the host by the kernels' own schedule functions, so
+ * that tests can check it against the visibility rule pair by pair.  Reads
+ * and writes host memory only; launches nothing.
+ *
+ * kind YOCO_SCHEDULE_PREFILL -- the bf16 tensor-core prefill of
+ * yoco_cross_prefill / yoco_swa_prefill for B, Tq, Tkv, q_pos0 (query row i at
+ * absolute position q_pos0 + i; q_pos0 + Tq <= Tkv) and window (0: causal).
+ * One record per (work tile, KV tile) visit, CTA by CTA, each CTA's visits in
+ * the order it makes them:
+ *   {cta, b, query head, query tile (128 rows), KV tile (128 keys), masked}
+ * where masked = 1 when the tile runs the per-element mask.
+ *
+ * kind YOCO_SCHEDULE_DECODE -- the split-KV plan of yoco_cross_decode for
+ * B sequences with HOST arrays seq_start [B] and seq_len [B], and max_len.
+ * One record per unit, CTA by CTA, in processing order:
+ *   {cta, b, split index, first cache row, tokens, pipeline stages}
+ *
+ * n_cta: the persistent grid's size, 0 = the current device's SM count.
+ * records: int64 [cap, 6] on the host (may be NULL when cap = 0); at most
+ * cap records are written and *n_records receives the full count. */
+enum { YOCO_SCHEDULE_PREFILL = 0, YOCO_SCHEDULE_DECODE = 1 };
+yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int32_t B, int64_t Tq,
+                                     int64_t Tkv, int64_t q_pos0, int32_t window,
+                                     const int64_t *seq_start, const int32_t *seq_len, int64_t max_len,
+                                     int32_t n_cta, int64_t *records, int64_t cap,
+                                     int64_t *n_records);
+
 /* KV-cache bytes of one sequence of N tokens (section 2: O(N + C L) for YOCO
  * versus N x L for a Transformer): one global K/V of N rows plus, per
  * self-decoder layer, a ring of min(window, N) rows.  Host only. */

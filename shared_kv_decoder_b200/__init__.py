@@ -9,7 +9,8 @@ importing a function fails loudly when libyoco.so is missing.
 
 Entry points (same names as the C ABI, without the ``yoco_`` prefix):
 kv_project_blend, swa_prefill, swa_decode, cross_prefill, cross_decode,
-plus linear, workspace sizes, cache_bytes and device_status.
+plus linear, workspace sizes, cache_bytes, device_status and the test-only
+debug_tile_schedule.
 """
 import ctypes
 import os
@@ -18,13 +19,15 @@ import torch
 
 __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_prefill",
            "swa_decode", "cross_prefill", "cross_decode", "cross_decode_workspace_size",
-           "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg"]
+           "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg",
+           "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT = range(6)
 BF16, FP32 = 0, 1
+SCHEDULE_PREFILL, SCHEDULE_DECODE = 0, 1
 _DT = {torch.bfloat16: BF16, torch.float32: FP32}
 
 
@@ -69,6 +72,8 @@ def load():
         "yoco_cross_decode_workspace_size": (sz, [i32, i64, cfgp]),
         "yoco_swa_decode_workspace_size": (sz, [i32, i32, cfgp]),
         "yoco_cache_bytes": (ctypes.c_double, [i32, i32, i64, cfgp]),
+        "yoco_debug_tile_schedule": (st, [i32, cfgp, i32, i64, i64, i64, i32, vp, vp, i64, i32, vp,
+                                          i64, ctypes.POINTER(ctypes.c_int64)]),
         "yoco_get_device_status": (st, [vp]),
         "yoco_status_string": (ctypes.c_char_p, [st]),
         "yoco_version": (ctypes.c_char_p, []),
@@ -241,3 +246,29 @@ def launch_count():
 def device_status():
     """Synchronise the current stream and return the device status code."""
     return int(load().yoco_get_device_status(_stream()))
+
+
+def debug_tile_schedule(kind, Hq, Hkv, D, dtype=torch.bfloat16, B=1, Tq=0, Tkv=0, q_pos0=0, window=0,
+                        seq_start=None, seq_len=None, max_len=1, n_cta=0):
+    """The kernels' work plan, computed on the host (test-only; see
+    yoco_debug_tile_schedule).  Returns an int64 numpy array [n, 6]:
+    prefill {cta, b, head, query tile, KV tile, masked};
+    decode {cta, b, split, first row, tokens, stages}.  seq_start / seq_len
+    are host sequences (decode only)."""
+    import numpy as np
+    L = load()
+    cfg = _cfg(Hq, Hkv, D, dtype)
+    ss = sl = None
+    if kind == SCHEDULE_DECODE:
+        ss = np.ascontiguousarray(np.asarray(seq_start, dtype=np.int64))
+        sl = np.ascontiguousarray(np.asarray(seq_len, dtype=np.int32))
+    n = ctypes.c_int64(0)
+    args = lambda rec, cap: (int(kind), ctypes.byref(cfg), int(B), int(Tq), int(Tkv), int(q_pos0),
+                             int(window), None if ss is None else ss.ctypes.data_as(ctypes.c_void_p),
+                             None if sl is None else sl.ctypes.data_as(ctypes.c_void_p), int(max_len),
+                             int(n_cta), rec, cap, ctypes.byref(n))
+    _check(L.yoco_debug_tile_schedule(*args(None, 0)), "yoco_debug_tile_schedule")
+    out = np.zeros((n.value, 6), dtype=np.int64)
+    _check(L.yoco_debug_tile_schedule(*args(out.ctypes.data_as(ctypes.c_void_p), n.value)),
+           "yoco_debug_tile_schedule")
+    return out

@@ -5,10 +5,12 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "../../include/yoco.h"
 #include "launch.h"
+#include "schedule.h"
 
 using namespace yoco;
 
@@ -224,6 +226,70 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = nullptr; a.ws = workspace;
     return from_cuda(launch_decode(a, pl, stream));
+}
+
+yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int32_t B, int64_t Tq,
+                                     int64_t Tkv, int64_t q_pos0, int32_t window,
+                                     const int64_t *seq_start, const int32_t *seq_len, int64_t max_len,
+                                     int32_t n_cta, int64_t *records, int64_t cap,
+                                     int64_t *n_records) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (!n_records || cap < 0 || (cap > 0 && !records) || B < 0 || n_cta < 0) return YOCO_ERR_INVALID;
+    const int sms = n_cta > 0 ? n_cta : device_sm_count();
+    int64_t n = 0;
+    auto put = [&](int64_t a, int64_t b, int64_t c, int64_t d, int64_t e, int64_t f) {
+        if (n < cap) {
+            int64_t *r = records + 6 * n;
+            r[0] = a; r[1] = b; r[2] = c; r[3] = d; r[4] = e; r[5] = f;
+        }
+        ++n;
+    };
+    if (kind == YOCO_SCHEDULE_PREFILL) {
+        if (Tq < 0 || Tkv < 0 || q_pos0 < 0 || q_pos0 + Tq > Tkv || window < 0) return YOCO_ERR_INVALID;
+        sched::PrefillShape s;
+        s.B = B; s.Hq = cfg->Hq; s.Hkv = cfg->Hkv;
+        s.Tq = Tq; s.Tkv = Tkv; s.q_pos0 = q_pos0; s.window = window;
+        const int64_t n_qtiles = (Tq + sched::kPrefillBM - 1) / sched::kPrefillBM;
+        const int64_t n_work = n_qtiles * cfg->Hq * B;
+        if (n_work > INT32_MAX / 2) return YOCO_ERR_UNSUPPORTED;
+        s.n_qtiles = (int32_t)n_qtiles;
+        const int grid = (int)(n_work < sms ? n_work : sms);
+        for (int c = 0; c < grid; ++c)
+            for (int r = 0;; ++r) {
+                const int w = sched::prefill_work_index(r, c, grid);
+                if (w >= n_work) break;
+                const sched::PrefillWork x = sched::prefill_work(s, w);
+                for (int t = 0; t < x.n_kv; ++t)
+                    put(c, x.b, x.h, x.qt, x.jt_lo + t, sched::prefill_tile_masked(s, x, t) ? 1 : 0);
+            }
+    } else if (kind == YOCO_SCHEDULE_DECODE) {
+        if (max_len < 1 || (B > 0 && (!seq_start || !seq_len))) return YOCO_ERR_INVALID;
+        DecodePlan pl;
+        if (!make_decode_plan(B, max_len, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl))
+            return YOCO_ERR_UNSUPPORTED;
+        // the compact unit list, sequence by sequence, as the kernel enumerates it
+        int64_t total = 0;
+        for (int b = 0; b < B; ++b) total += sched::decode_units(seq_len[b], pl.split, pl.n_split);
+        const int64_t slots = (int64_t)B * pl.n_split;
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(slots, sms));
+        for (int c = 0; c < grid; ++c) {
+            int b = 0;
+            int64_t before = 0;  // units of sequences < b
+            for (int64_t u = c; u < total; u += grid) {
+                while (before + sched::decode_units(seq_len[b], pl.split, pl.n_split) <= u)
+                    before += sched::decode_units(seq_len[b++], pl.split, pl.n_split);
+                const int64_t sidx = u - before;
+                const int64_t t0 = sidx * pl.split;
+                const int64_t n_tok = std::min<int64_t>(pl.split, seq_len[b] - t0);
+                put(c, b, sidx, seq_start[b] + t0, n_tok, (n_tok + pl.stage_tokens - 1) / pl.stage_tokens);
+            }
+        }
+    } else {
+        return YOCO_ERR_INVALID;
+    }
+    *n_records = n;
+    return YOCO_OK;
 }
 
 double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_attn_cfg *cfg) {

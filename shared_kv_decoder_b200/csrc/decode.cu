@@ -28,6 +28,7 @@
 //    a slot is visible when its stored position lies in (pos - window, pos].
 #include "common.cuh"
 #include "launch.h"
+#include "schedule.h"
 #include "tc.cuh"
 
 #include <algorithm>
@@ -74,7 +75,7 @@ static __device__ bool find_unit(const DecodeKParams &p, int64_t u, int *b_out, 
         if (b < p.B) len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
         // never more units than the workspace plan holds (lengths above max_len
         // are a caller error; their tail is not read)
-        const int64_t cnt = len > 0 ? min((len + p.split - 1) / p.split, p.n_split) : 0;
+        const int64_t cnt = sched::decode_units(len, p.split, p.n_split);
         int64_t incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

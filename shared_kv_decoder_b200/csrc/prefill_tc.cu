@@ -48,6 +48,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "schedule.h"
 #include "tc.cuh"
 
 namespace yoco {
@@ -77,13 +78,10 @@ struct Smem {
 };
 
 struct TcParams {
-    int32_t B, Hq, Hkv;
-    int64_t Tq, Tkv, q_pos0;
-    int32_t window;
+    sched::PrefillShape s;
     float scale_log2;
     void *o;
     float *lse;
-    int32_t n_qtiles;
     int32_t n_work;
 };
 
@@ -107,35 +105,6 @@ YOCO_DEV bool wait1(uint64_t *bar, uint32_t parity) {
 }
 YOCO_DEV bool waitw(uint64_t *bar, uint32_t parity) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, &g_status_prefill_tc));
-}
-
-// One work tile: its query tile, head, batch and KV tile range.
-struct Work {
-    int qt, h, b, g;               // query tile, query head, batch, KV head
-    int64_t i0, p_first, p_last;   // first row, absolute positions of first / last real row
-    int jt_lo, n_kv;               // first KV tile, number of KV tiles
-};
-
-// Work tile of round r for CTA c: rounds alternate direction (snake order), so
-// with the causal tiles sorted heaviest first every CTA gets a similar total.
-YOCO_DEV int work_index(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
-
-YOCO_DEV Work work_of(const TcParams &p, int w) {
-    Work x;
-    const int per = p.Hq * p.B;
-    x.qt = p.n_qtiles - 1 - w / per;  // heaviest causal tiles first
-    x.h = (w % per) % p.Hq;
-    x.b = (w % per) / p.Hq;
-    x.g = x.h / (p.Hq / p.Hkv);
-    x.i0 = (int64_t)x.qt * BM;
-    const int64_t i_last = min(x.i0 + BM, p.Tq) - 1;
-    x.p_first = p.q_pos0 + x.i0;
-    x.p_last = p.q_pos0 + i_last;
-    const int64_t j_lo = p.window > 0 ? max((int64_t)0, x.p_first - p.window + 1) : 0;
-    const int64_t j_hi = min(p.Tkv - 1, x.p_last);
-    x.jt_lo = (int)(j_lo / BN);
-    x.n_kv = (int)(j_hi / BN) - x.jt_lo + 1;
-    return x;
 }
 
 }  // namespace
@@ -195,9 +164,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int gk = 0, k = 0;  // K tiles issued, Q tiles issued
             for (int r = 0; !*abort_flag; ++r) {
-                const int w = work_index(r, blockIdx.x, gridDim.x);
+                const int w = sched::prefill_work_index(r, blockIdx.x, gridDim.x);
                 if (w >= p.n_work) break;
-                const Work x = work_of(p, w);
+                const sched::PrefillWork x = sched::prefill_work(p.s, w);
                 if (!wait1(&bars[kQEmpty + (k & 1)], ((k >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
                 mbar_arrive_expect_tx(&bars[kQFull + (k & 1)], BM * D * 2);
                 for (int kb = 0; kb < KB; ++kb)
@@ -223,9 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (lane == 1) {
             int gv = 0;
             for (int r = 0; !*abort_flag; ++r) {
-                const int w = work_index(r, blockIdx.x, gridDim.x);
+                const int w = sched::prefill_work_index(r, blockIdx.x, gridDim.x);
                 if (w >= p.n_work) break;
-                const Work x = work_of(p, w);
+                const sched::PrefillWork x = sched::prefill_work(p.s, w);
                 for (int t = 0; t < x.n_kv; ++t, ++gv) {
                     const int st = gv % L::VSTAGES;
                     if (!wait1(&bars[kVEmpty + st], ((gv / L::VSTAGES) & 1) ^ 1)) { *abort_flag = 1; break; }
@@ -271,9 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             int gk = 0;
             for (int k = 0; ok; ++k) {
-                const int w = work_index(k, blockIdx.x, gridDim.x);
+                const int w = sched::prefill_work_index(k, blockIdx.x, gridDim.x);
                 if (w >= p.n_work) break;
-                const Work x = work_of(p, w);
+                const sched::PrefillWork x = sched::prefill_work(p.s, w);
                 if (!wait1(&bars[kQFull + (k & 1)], (k >> 1) & 1)) { ok = false; break; }
                 const uint32_t qb = base + L::Q + (k & 1) * L::TILE;
                 for (int t = 0; t < x.n_kv; ++t, ++gk) {
@@ -311,11 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[BN / 2];
         int gk = 0;
         for (int k = 0; ok; ++k) {
-            const int w = work_index(k, blockIdx.x, gridDim.x);
+            const int w = sched::prefill_work_index(k, blockIdx.x, gridDim.x);
             if (w >= p.n_work) break;
-            const Work x = work_of(p, w);
+            const sched::PrefillWork x = sched::prefill_work(p.s, w);
             const int64_t i = x.i0 + r;
-            const int64_t pos = p.q_pos0 + i;
+            const int64_t pos = p.s.q_pos0 + i;
             const uint32_t tO = ((k & 1) ? tO1 : tO0) + lane_off;
             float m = -INFINITY, l = 0.f;
             for (int t = 0; t < x.n_kv; ++t, ++gk) {
@@ -327,14 +296,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < BN; c += 32) tc::tmem_ld32(tS + c, s + c);
                 tc::wait_ld();
                 const int64_t j0 = (int64_t)(x.jt_lo + t) * BN;
-                const bool need_mask = (j0 + BN - 1 > x.p_first) || (j0 + BN > p.Tkv) ||
-                                       (p.window > 0 && j0 <= x.p_last - p.window);
-                if (need_mask) {
+                if (sched::prefill_tile_masked(p.s, x, t)) {
                     // visible columns of this row form one range [c_lo, c_hi): one
                     // unsigned compare per element against 32-bit bounds
                     const int64_t dg = pos - j0;
-                    const int c_hi = (int)max((int64_t)0, min(min(dg + 1, p.Tkv - j0), (int64_t)BN));
-                    const int c_lo = p.window > 0 ? (int)max((int64_t)0, min(dg - p.window + 1, (int64_t)BN)) : 0;
+                    const int c_hi = (int)max((int64_t)0, min(min(dg + 1, p.s.Tkv - j0), (int64_t)BN));
+                    const int c_lo = p.s.window > 0 ? (int)max((int64_t)0, min(dg - p.s.window + 1, (int64_t)BN)) : 0;
                     const unsigned width = (unsigned)max(0, c_hi - c_lo);
 #pragma unroll
                     for (int c = 0; c < BN; ++c)
@@ -415,13 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
-                                 (((int64_t)x.b * p.Tq + i) * p.Hq + x.h) * D;
+                                 (((int64_t)x.b * p.s.Tq + i) * p.s.Hq + x.h) * D;
 #pragma unroll
             for (int c = 0; c < D; c += 32) {
                 float o[32];
                 tc::tmem_ld32(tO + c, o);
                 tc::wait_ld();
-                if (i < p.Tq) {
+                if (i < p.s.Tq) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
                         uint4 wv;
@@ -433,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (p.lse && i < p.Tq)
-                p.lse[((int64_t)x.b * p.Hq + x.h) * p.Tq + i] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+            if (p.lse && i < p.s.Tq)
+                p.lse[((int64_t)x.b * p.s.Hq + x.h) * p.s.Tq + i] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
             tc::fence_before_sync();
             mbar_arrive(&bars[kOFree + (k & 1)]);
         }
@@ -467,14 +434,14 @@ cudaError_t launch_tc_d(const PrefillArgs &a, cudaStream_t st) {
         !make_map(&mv, a.v, a.B, a.Tkv, a.Hkv, D))
         return cudaErrorNotSupported;
     TcParams p;
-    p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv;
-    p.Tq = a.Tq; p.Tkv = a.Tkv; p.q_pos0 = a.q_pos0; p.window = a.window;
+    p.s.B = a.B; p.s.Hq = a.Hq; p.s.Hkv = a.Hkv;
+    p.s.Tq = a.Tq; p.s.Tkv = a.Tkv; p.s.q_pos0 = a.q_pos0; p.s.window = a.window;
     p.scale_log2 = a.scale * kLog2e;
     p.o = a.o; p.lse = a.lse;
     const int64_t n_qtiles = (a.Tq + BM - 1) / BM;
     const int64_t n_work = n_qtiles * a.Hq * a.B;
     if (n_work > INT32_MAX / 2) return cudaErrorNotSupported;
-    p.n_qtiles = (int)n_qtiles;
+    p.s.n_qtiles = (int)n_qtiles;
     p.n_work = (int)n_work;
     auto kern = attn_prefill_tc_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

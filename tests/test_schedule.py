@@ -1,0 +1,128 @@
+"""The kernels' work plans (yoco_debug_tile_schedule), checked on the host
+against the oracle's visibility rule, bit-exact: the prefill visits exactly
+the KV tiles that hold a visible (query, key) pair, masks exactly the tiles
+that also hold an invisible pair or a key past the end, and covers every
+work tile once; the decode units partition every sequence.  No GPU needed:
+the plan is computed by the same schedule functions the kernels run."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import shared_kv_decoder_b200 as yoco
+
+BM = BN = 128
+
+PREFILL_CASES = [
+    # B, Hq, Hkv, Tq, Tkv, q_pos0, window, n_cta
+    (1, 4, 2, 300, 300, 0, 0, 5),        # causal, ragged last query tile
+    (2, 8, 2, 256, 256, 0, 0, 148),      # more CTAs than work tiles
+    (1, 2, 1, 200, 777, 577, 0, 3),      # chunk offset, tail KV tile
+    (1, 4, 4, 640, 640, 0, 100, 7),      # window smaller than a tile
+    (3, 2, 2, 513, 513, 0, 300, 4),      # window spanning tile edges, B > 1
+    (1, 2, 1, 129, 1000, 871, 256, 2),   # chunked window, tile-boundary offsets
+    (1, 1, 1, 1, 1, 0, 0, 1),            # a single query and key
+    (1, 2, 1, 384, 384, 0, 128, 3),      # window equal to the tile size
+]
+
+
+def _prefill(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta):
+    return yoco.debug_tile_schedule(yoco.SCHEDULE_PREFILL, Hq, Hkv, 64, B=B, Tq=Tq, Tkv=Tkv,
+                                    q_pos0=q_pos0, window=W, n_cta=n_cta)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Tq,Tkv,q_pos0,W,n_cta", PREFILL_CASES)
+def test_prefill_plan_matches_visibility(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta):
+    rec = _prefill(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta)
+    vis = oracle.visibility(Tq, Tkv, q_pos0, W)
+    n_qt = -(-Tq // BM)
+    n_kt = -(-Tkv // BN)
+    # expected per query tile: KV tiles with a visible pair, and which need a mask
+    want = {}
+    for qt in range(n_qt):
+        rows = vis[qt * BM:min((qt + 1) * BM, Tq)]
+        tiles = {}
+        for kt in range(n_kt):
+            blk = rows[:, kt * BN:(kt + 1) * BN]
+            if blk.any():
+                # masked: an invisible pair among real rows, or keys past Tkv
+                tiles[kt] = int((not blk.all()) or (kt + 1) * BN > Tkv)
+        want[qt] = tiles
+    seen = {}
+    for cta, b, h, qt, kt, masked in rec.tolist():
+        assert 0 <= cta < n_cta and 0 <= b < B and 0 <= h < Hq
+        seen.setdefault((b, h, qt), []).append((cta, kt, masked))
+    assert set(seen) == {(b, h, qt) for b in range(B) for h in range(Hq) for qt in range(n_qt)}
+    for (b, h, qt), visits in seen.items():
+        assert len({c for c, _, _ in visits}) == 1, "a work tile is split over CTAs"
+        kts = [kt for _, kt, _ in visits]
+        assert kts == sorted(want[qt]), (b, h, qt)      # exactly the visible tiles, in order
+        assert {kt: m for _, kt, m in visits} == want[qt], (b, h, qt)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Tq,Tkv,q_pos0,W,n_cta", PREFILL_CASES)
+def test_prefill_plan_order_and_balance(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta):
+    rec = _prefill(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta)
+    # the CTAs' visits form contiguous runs, one run per work tile
+    runs = []
+    for r in rec.tolist():
+        key = (r[0], r[1], r[2], r[3])
+        if not runs or runs[-1][0] != key:
+            runs.append([key, 0])
+        runs[-1][1] += 1
+    assert len(runs) == len({k for k, _ in runs})
+    # each CTA's first work tile is a heaviest one (the last query tile), and
+    # the per-CTA totals stay within one work tile's worth of each other
+    n_qt = -(-Tq // BM)
+    firsts = {}
+    for (cta, b, h, qt), _ in runs:
+        firsts.setdefault(cta, qt)
+    assert all(qt == n_qt - 1 for qt in firsts.values()) or len(firsts) > B * Hq
+    tot = np.zeros(max(firsts) + 1)
+    for (cta, _, _, _), n in runs:
+        tot[cta] += n
+    heaviest = max(n for _, n in runs)
+    if len(runs) >= 2 * len(tot):
+        assert tot.max() - tot.min() <= heaviest
+
+
+@pytest.mark.parametrize("lens,max_len,Hq,Hkv,D,n_cta", [
+    ([1000, 17, 3000], 3000, 32, 8, 128, 4),
+    ([1, 2, 3, 130, 4097], 5000, 8, 1, 64, 148),
+    ([65536, 70001, 131072, 100000], 131072, 32, 8, 128, 148),
+    ([0, 5, 0, 300], 300, 4, 2, 64, 3),
+])
+def test_decode_plan_partitions_sequences(lens, max_len, Hq, Hkv, D, n_cta):
+    starts = np.cumsum([0] + [l + 7 for l in lens[:-1]])
+    rec = yoco.debug_tile_schedule(yoco.SCHEDULE_DECODE, Hq, Hkv, D, B=len(lens), seq_start=starts,
+                                   seq_len=lens, max_len=max_len, n_cta=n_cta)
+    stage = 128 // Hkv
+    covered = {b: [] for b in range(len(lens))}
+    per_cta_units = {}
+    for cta, b, s, row0, n_tok, n_st in rec.tolist():
+        assert 0 <= cta < n_cta
+        assert n_tok >= 1 and n_st == -(-n_tok // stage)
+        covered[b].append((row0 - starts[b], n_tok, s))
+        per_cta_units[cta] = per_cta_units.get(cta, 0) + 1
+    for b, L in enumerate(lens):
+        segs = sorted(covered[b])
+        pos = 0
+        for k, (off, n, s) in enumerate(segs):
+            assert off == pos and s == k         # consecutive, no gap or overlap
+            pos += n
+        assert pos == L                          # the whole sequence, nothing past it
+        if len(segs) > 1:                        # equal splits, a multiple of the stage
+            split = segs[0][1]
+            assert split % stage == 0 and all(n == split for _, n, _ in segs[:-1])
+    # the compact unit list is dealt round-robin over the CTAs
+    if per_cta_units:
+        assert max(per_cta_units.values()) - min(per_cta_units.values()) <= 1
+
+
+def test_schedule_rejects_bad_arguments():
+    with pytest.raises(yoco.YocoError):
+        _prefill(1, 4, 2, 100, 50, 0, 0, 4)      # q_pos0 + Tq > Tkv
+    with pytest.raises(yoco.YocoError):
+        yoco.debug_tile_schedule(7, 4, 2, 64)
+    with pytest.raises(yoco.YocoError):
+        yoco.debug_tile_schedule(yoco.SCHEDULE_PREFILL, 3, 2, 64, Tq=1, Tkv=1)   # Hq % Hkv
