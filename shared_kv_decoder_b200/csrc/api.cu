@@ -54,11 +54,15 @@ yoco_status run_linear(const LinearArgs &a, cudaStream_t s) {
     return from_cuda(launch_linear_simt(a, s));
 }
 
-// Attention prefill dispatch: bf16 goes to the tcgen05 kernel; fp32 (and any
-// bf16 shape that kernel was not built for) to the CUDA-core kernel.
+// Attention prefill dispatch: bf16 goes to a tcgen05 kernel -- two query
+// heads per CTA when the group size is even, else one; fp32 (and any bf16
+// shape those kernels were not built for) to the CUDA-core kernel.
 yoco_status run_prefill(const PrefillArgs &a, cudaStream_t s) {
     if (a.dtype == kBF16) {
-        const cudaError_t e = launch_prefill_tc(a, s);
+        cudaError_t e = launch_prefill_pair(a, s);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();
+        e = launch_prefill_tc(a, s);
         if (e != cudaErrorNotSupported) return from_cuda(e);
         cudaGetLastError();
     }
@@ -302,7 +306,7 @@ double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_at
 yoco_status yoco_get_device_status(cudaStream_t stream) {
     const cudaError_t e = cudaStreamSynchronize(stream);
     const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc() |
-                           read_and_clear_status_project_tc();
+                           read_and_clear_status_prefill_pair() | read_and_clear_status_project_tc();
     if (s) return YOCO_ERR_TIMEOUT;
     return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;
 }

@@ -77,6 +77,9 @@ cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t s);
 // Tensor-core path (bf16): tcgen05 + TMEM + TMA.  Returns cudaErrorNotSupported
 // when the shape is outside what it was built for.
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s);
+// Tensor-core path for bf16 and an even group size: two query heads of one
+// KV group per CTA.  cudaErrorNotSupported for other shapes.
+cudaError_t launch_prefill_pair(const PrefillArgs &a, cudaStream_t s);
 
 // ------------------------------------------------------------ projection
 struct LinearArgs {
@@ -101,6 +104,7 @@ cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
 // Device status words of the translation units that hold bounded waits.
 unsigned int read_and_clear_status_decode();
 unsigned int read_and_clear_status_prefill_tc();
+unsigned int read_and_clear_status_prefill_pair();
 unsigned int read_and_clear_status_project_tc();
 
 int device_sm_count();

@@ -22,9 +22,8 @@ constexpr int kPrefillBN = 128;  // keys per KV tile
 YOCO_HD int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 YOCO_HD int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
-// Prefill work tile w of n_work = n_qtiles * Hq * B.  Works are numbered
-// heaviest causal tile first: all (head, batch) pairs of the last query tile,
-// then of the one before, and so on.
+// Prefill work tiles are numbered heaviest causal tile first: all (head,
+// batch) pairs of the last query tile, then of the one before, and so on.
 struct PrefillWork {
     int qt, h, b, g;              // query tile, query head, batch, KV head
     int64_t i0;                   // first query row
@@ -39,12 +38,12 @@ struct PrefillShape {
     int32_t n_qtiles;
 };
 
-YOCO_HD PrefillWork prefill_work(const PrefillShape &s, int w) {
+// The KV range of query tile qt of (batch b, query head h).
+YOCO_HD PrefillWork prefill_work_at(const PrefillShape &s, int qt, int h, int b) {
     PrefillWork x;
-    const int per = s.Hq * s.B;
-    x.qt = s.n_qtiles - 1 - w / per;
-    x.h = (w % per) % s.Hq;
-    x.b = (w % per) / s.Hq;
+    x.qt = qt;
+    x.h = h;
+    x.b = b;
     x.g = x.h / (s.Hq / s.Hkv);
     x.i0 = (int64_t)x.qt * kPrefillBM;
     const int64_t i_last = min64(x.i0 + kPrefillBM, s.Tq) - 1;
@@ -57,6 +56,23 @@ YOCO_HD PrefillWork prefill_work(const PrefillShape &s, int w) {
     x.n_kv = (int)(j_hi / kPrefillBN) - x.jt_lo + 1;
     return x;
 }
+
+// One query head per work tile (any group size).
+YOCO_HD PrefillWork prefill_work(const PrefillShape &s, int w) {
+    const int per = s.Hq * s.B;
+    return prefill_work_at(s, s.n_qtiles - 1 - w / per, (w % per) % s.Hq, (w % per) / s.Hq);
+}
+
+// Two query heads per work tile, 2hp and 2hp + 1, which share their KV head
+// when the group size Hq / Hkv is even: n_work = n_qtiles * (Hq / 2) * B.
+// The returned h is the first head of the pair.
+YOCO_HD PrefillWork prefill_pair_work(const PrefillShape &s, int w) {
+    const int hp = s.Hq / 2, per = hp * s.B;
+    return prefill_work_at(s, s.n_qtiles - 1 - w / per, 2 * ((w % per) % hp), (w % per) / hp);
+}
+
+// The paired kernel serves bf16 shapes whose group size is even.
+YOCO_HD bool prefill_pairs_heads(int Hq, int Hkv) { return (Hq / Hkv) % 2 == 0; }
 
 // Work tile of round r for CTA c of a G-CTA grid: rounds alternate direction
 // (snake order), so with the works sorted heaviest first every CTA gets a
