@@ -182,8 +182,9 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
  * kind YOCO_SCHEDULE_PREFILL -- the bf16 tensor-core prefill of
  * yoco_cross_prefill / yoco_swa_prefill for B, Tq, Tkv, q_pos0 (query row i at
  * absolute position q_pos0 + i; q_pos0 + Tq <= Tkv) and window (0: causal).
- * One record per (work tile, KV tile) visit, CTA by CTA, each CTA's visits in
- * the order it makes them:
+ * A work tile is one 128-row query tile of one query head, or of two heads
+ * (2hp, 2hp + 1) when Hq / Hkv is even.  One record per (query head, KV tile)
+ * visit, CTA by CTA, each CTA's visits in the order it makes them:
  *   {cta, b, query head, query tile (128 rows), KV tile (128 keys), masked}
  * where masked = 1 when the tile runs the per-element mask.
  *

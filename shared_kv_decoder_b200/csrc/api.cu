@@ -254,8 +254,12 @@ yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int
         sched::PrefillShape s;
         s.B = B; s.Hq = cfg->Hq; s.Hkv = cfg->Hkv;
         s.Tq = Tq; s.Tkv = Tkv; s.q_pos0 = q_pos0; s.window = window;
+        // the kernel run_prefill picks for bf16: two heads per work tile when
+        // the group size is even, else one
+        const bool pairs = cfg->dtype == YOCO_BF16 && sched::prefill_pairs_heads(cfg->Hq, cfg->Hkv);
+        const int heads = pairs ? 2 : 1;
         const int64_t n_qtiles = (Tq + sched::kPrefillBM - 1) / sched::kPrefillBM;
-        const int64_t n_work = n_qtiles * cfg->Hq * B;
+        const int64_t n_work = n_qtiles * (cfg->Hq / heads) * B;
         if (n_work > INT32_MAX / 2) return YOCO_ERR_UNSUPPORTED;
         s.n_qtiles = (int32_t)n_qtiles;
         const int grid = (int)(n_work < sms ? n_work : sms);
@@ -263,9 +267,10 @@ yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int
             for (int r = 0;; ++r) {
                 const int w = sched::prefill_work_index(r, c, grid);
                 if (w >= n_work) break;
-                const sched::PrefillWork x = sched::prefill_work(s, w);
+                const sched::PrefillWork x = pairs ? sched::prefill_pair_work(s, w) : sched::prefill_work(s, w);
                 for (int t = 0; t < x.n_kv; ++t)
-                    put(c, x.b, x.h, x.qt, x.jt_lo + t, sched::prefill_tile_masked(s, x, t) ? 1 : 0);
+                    for (int hh = 0; hh < heads; ++hh)
+                        put(c, x.b, x.h + hh, x.qt, x.jt_lo + t, sched::prefill_tile_masked(s, x, t) ? 1 : 0);
             }
     } else if (kind == YOCO_SCHEDULE_DECODE) {
         if (max_len < 1 || (B > 0 && (!seq_start || !seq_len))) return YOCO_ERR_INVALID;

@@ -23,6 +23,8 @@ PREFILL_CASES = [
     (1, 2, 1, 129, 1000, 871, 256, 2),   # chunked window, tile-boundary offsets
     (1, 1, 1, 1, 1, 0, 0, 1),            # a single query and key
     (1, 2, 1, 384, 384, 0, 128, 3),      # window equal to the tile size
+    (2, 8, 8, 300, 300, 0, 0, 5),        # group size 1: one head per work tile
+    (1, 16, 2, 520, 520, 0, 200, 6),     # group size 8
 ]
 
 
@@ -63,25 +65,32 @@ def test_prefill_plan_matches_visibility(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta):
 @pytest.mark.parametrize("B,Hq,Hkv,Tq,Tkv,q_pos0,W,n_cta", PREFILL_CASES)
 def test_prefill_plan_order_and_balance(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta):
     rec = _prefill(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta)
-    # the CTAs' visits form contiguous runs, one run per work tile
-    runs = []
-    for r in rec.tolist():
-        key = (r[0], r[1], r[2], r[3])
-        if not runs or runs[-1][0] != key:
-            runs.append([key, 0])
-        runs[-1][1] += 1
-    assert len(runs) == len({k for k, _ in runs})
-    # each CTA's first work tile is a heaviest one (the last query tile), and
-    # the per-CTA totals stay within one work tile's worth of each other
+    heads = 2 if (Hq // Hkv) % 2 == 0 else 1          # heads per work tile
     n_qt = -(-Tq // BM)
+    # work tiles: (cta, b, head pair, query tile); the heads of a pair visit
+    # the same KV tiles in lockstep, and each work tile's visits are one run
+    runs = []
+    for cta, b, h, qt, kt, _ in rec.tolist():
+        key = (cta, b, h // heads, qt)
+        if not runs or runs[-1][0] != key:
+            runs.append([key, []])
+        runs[-1][1].append((h, kt))
+    assert len(runs) == len({k for k, _ in runs})
+    for (cta, b, hp, qt), visits in runs:
+        per_head = [[kt for h, kt in visits if h == heads * hp + e] for e in range(heads)]
+        assert all(v == per_head[0] for v in per_head)
+        if heads == 2:
+            assert [h for h, _ in visits] == [2 * hp, 2 * hp + 1] * len(per_head[0])
+    # each CTA starts with a heaviest work tile (the last query tile), and the
+    # per-CTA totals stay within one work tile's worth of each other
     firsts = {}
-    for (cta, b, h, qt), _ in runs:
+    for (cta, _, _, qt), _ in runs:
         firsts.setdefault(cta, qt)
-    assert all(qt == n_qt - 1 for qt in firsts.values()) or len(firsts) > B * Hq
+    assert all(qt == n_qt - 1 for qt in firsts.values()) or len(firsts) > B * Hq // heads
     tot = np.zeros(max(firsts) + 1)
-    for (cta, _, _, _), n in runs:
-        tot[cta] += n
-    heaviest = max(n for _, n in runs)
+    for (cta, _, _, _), v in runs:
+        tot[cta] += len(v)
+    heaviest = max(len(v) for _, v in runs)
     if len(runs) >= 2 * len(tot):
         assert tot.max() - tot.min() <= heaviest
 
