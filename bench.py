@@ -74,29 +74,33 @@ def load_peaks():
 
 # DRAM bytes (read + write) per launch of the roofline kernels, from one ncu
 # capture of the benchmark's own launch shape (--case prefill_layer /
-# decode_layer).  Each figure is keyed by the SHA-256 of the kernel source it
-# was taken on: once that source changes the figure no longer describes the
-# kernel, and the report carries null instead.
+# decode_layer).  Each figure is keyed by the SHA-256 of the kernel's source
+# files (the .cu and the headers it includes) as they were when it was
+# taken: once any of them changes the figure no longer describes the kernel,
+# and the report carries null instead.
+_CSRC = "shared_kv_decoder_b200/csrc/"
 TRAFFIC = {
-    # attn_prefill_tc_kernel<128>, T=32768: 3.265428 GB read + 235.083008 MB written
-    "prefill": {"bytes": 3265428000 + 235083008, "source": "shared_kv_decoder_b200/csrc/prefill_tc.cu",
-                "sha256": "35d72ea4c3ff406b935bda52a94133bd2fe4550eebff1d60083be4627cf2341d"},
-    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416670 GB read + 25.219584 MB written
-    "decode": {"bytes": 6416670000 + 25219584, "source": "shared_kv_decoder_b200/csrc/decode.cu",
-               "sha256": "9080e46437d4985bd9cdcb257d678d3fb60a3ae388defc3e7d43c6a439bb0637"},
+    # attn_prefill_pair_kernel<128>, T=32768: 1.829333 GB read + 238.978304 MB written
+    "prefill": {"bytes": 1829333000 + 238978304,
+                "sources": ["prefill_pair.cu", "schedule.h", "tc.cuh", "common.cuh"],
+                "sha256": "fbaf62f0cc8dcc000c7d83c2a46392dd5909ea2890086fc6737808270a7a158c"},
+    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416114 GB read + 25.135360 MB written
+    "decode": {"bytes": 6416114000 + 25135360,
+               "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
+               "sha256": "d7d7875bc339ebb6d1a5591fe98c89c1f392bf916274f892be58e1618f647935"},
 }
 
 
 def traffic(kind):
     import hashlib
     t = TRAFFIC[kind]
-    if t["bytes"] is None:
-        return None
+    m = hashlib.sha256()
     try:
-        h = hashlib.sha256(open(os.path.join(ROOT, t["source"]), "rb").read()).hexdigest()
+        for f in t["sources"]:
+            m.update(open(os.path.join(ROOT, _CSRC, f), "rb").read())
     except OSError:
         return None
-    return float(t["bytes"]) if h == t["sha256"] else None
+    return float(t["bytes"]) if m.hexdigest() == t["sha256"] else None
 
 
 def reduce_max_over_ranks(values, device=None):
