@@ -246,6 +246,31 @@ def cache_bytes_transformer(L, N, Hkv, D, elem_bytes):
     return lib().oracle_cache_bytes_transformer(L, N, Hkv, D, elem_bytes)
 
 
+def _self_decoder(x, weights, Hq, Hkv, D, window, w_blend, eps, out):
+    """Self-decoder layers over every row of x, then the global K/V (see
+    tiny_stack); fills out and returns (x, k_g, v_g)."""
+    T = x.shape[0]
+    k_bottom = v_bottom = None
+    for l in range(len(weights["self_q"])):
+        q = project(x, weights["self_q"][l], True, eps).reshape(1, T, Hq, D)
+        if l == 0:
+            k, v = kv_project_blend(x, weights["self_kv"][l], Hkv, D, eps=eps)
+            k_bottom, v_bottom = k, v
+        else:
+            k, v = kv_project_blend(x, weights["self_kv"][l], Hkv, D, k_bottom, v_bottom,
+                                    w_blend[l], w_blend[l], eps=eps)
+        o, _ = attention(q, k.reshape(1, T, Hkv, D), v.reshape(1, T, Hkv, D), 0, window)
+        x = x + project(o.reshape(T, Hq * D), weights["self_o"][l], False)
+        out["self_q"].append(q.reshape(T, Hq, D))
+        out["self_k"].append(k)
+        out["self_v"].append(v)
+        out["self_o"].append(o.reshape(T, Hq, D))
+        out["x_self"].append(x.copy())
+    kg, vg = kv_project_blend(x, weights["g_kv"], Hkv, D, eps=eps)
+    out["k_g"], out["v_g"] = kg, vg
+    return x, kg, vg
+
+
 def tiny_stack(x, weights, Hq, Hkv, D, window, w_blend, eps=1e-5):
     """The small YOCO++ attention stack, end to end, for every row of x.
 
@@ -267,24 +292,7 @@ def tiny_stack(x, weights, Hq, Hkv, D, window, w_blend, eps=1e-5):
     T, d = x.shape
     out = {"self_q": [], "self_k": [], "self_v": [], "self_o": [], "x_self": [],
            "cross_q": [], "cross_o": [], "x_cross": []}
-    k_bottom = v_bottom = None
-    for l in range(len(weights["self_q"])):
-        q = project(x, weights["self_q"][l], True, eps).reshape(1, T, Hq, D)
-        if l == 0:
-            k, v = kv_project_blend(x, weights["self_kv"][l], Hkv, D, eps=eps)
-            k_bottom, v_bottom = k, v
-        else:
-            k, v = kv_project_blend(x, weights["self_kv"][l], Hkv, D, k_bottom, v_bottom,
-                                    w_blend[l], w_blend[l], eps=eps)
-        o, _ = attention(q, k.reshape(1, T, Hkv, D), v.reshape(1, T, Hkv, D), 0, window)
-        x = x + project(o.reshape(T, Hq * D), weights["self_o"][l], False)
-        out["self_q"].append(q.reshape(T, Hq, D))
-        out["self_k"].append(k)
-        out["self_v"].append(v)
-        out["self_o"].append(o.reshape(T, Hq, D))
-        out["x_self"].append(x.copy())
-    kg, vg = kv_project_blend(x, weights["g_kv"], Hkv, D, eps=eps)
-    out["k_g"], out["v_g"] = kg, vg
+    x, kg, vg = _self_decoder(x, weights, Hq, Hkv, D, window, w_blend, eps, out)
     for c in range(len(weights["cross_q"])):
         q = project(x, weights["cross_q"][c], True, eps).reshape(1, T, Hq, D)
         o, _ = attention(q, kg.reshape(1, T, Hkv, D), vg.reshape(1, T, Hkv, D), 0, 0)
@@ -294,3 +302,21 @@ def tiny_stack(x, weights, Hq, Hkv, D, window, w_blend, eps=1e-5):
         out["x_cross"].append(x.copy())
     out["x"] = x
     return out
+
+
+def tiny_stack_early_exit(x, weights, Hq, Hkv, D, window, w_blend, eps=1e-5):
+    """Early-exit prefill of the same stack ("You Only Cache Once", paperlayer
+    summary, section 2, and podcast transcript, the Figure 3 discussion): the
+    self-decoder runs over every prompt row and writes the global K/V, and only
+    the LAST row goes through the cross-decoder, each cross layer attending
+    from that row to the whole global K/V.  Returns the last row's final x [d]."""
+    x = _f64(x).copy()
+    T, d = x.shape
+    out = {"self_q": [], "self_k": [], "self_v": [], "self_o": [], "x_self": []}
+    x, kg, vg = _self_decoder(x, weights, Hq, Hkv, D, window, w_blend, eps, out)
+    xt = x[T - 1:T].copy()
+    for c in range(len(weights["cross_q"])):
+        q = project(xt, weights["cross_q"][c], True, eps).reshape(1, Hq, D)
+        o, _ = cross_decode(q, kg, vg, [0], [T])
+        xt = xt + project(o.reshape(1, Hq * D), weights["cross_o"][c], False)
+    return xt[0]

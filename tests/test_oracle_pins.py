@@ -338,3 +338,17 @@ def test_tiny_stack_cross_layers_share_one_kv():
         q = out["cross_q"][c][None]
         ref = _sdpa(q, out["k_g"][None], out["v_g"][None])
         np.testing.assert_allclose(out["cross_o"][c], ref[0], atol=1e-12)
+
+
+def test_tiny_stack_early_exit_is_exact():
+    # The pages: prefill may exit before the cross-decoder for all but the last
+    # prompt row without changing the output.  Row by row the oracle computes
+    # the same sums, so the early-exit row equals the full run's last row.
+    cfg = wl.TinyStack()
+    x, w = wl.tiny_stack_inputs(cfg, torch.float32)
+    T = cfg.T
+    full = oracle.tiny_stack(x[:T], w, cfg.Hq, cfg.Hkv, cfg.D, cfg.window, cfg.w_blend)
+    ee = oracle.tiny_stack_early_exit(x[:T], w, cfg.Hq, cfg.Hkv, cfg.D, cfg.window, cfg.w_blend)
+    np.testing.assert_allclose(ee, full["x"][T - 1], rtol=0, atol=1e-12)
+    # and it differs from the row before: the check is not vacuous
+    assert np.abs(ee - full["x"][T - 2]).max() > 1e-3
