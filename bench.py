@@ -45,6 +45,7 @@ WORKLOAD = ("cross-decoder causal prefill B=1 T=32768 32q/8kv D=128 x14 layers o
 P = dict(T=32768, Hq=32, Hkv=8, D=128, layers=14, d=4096)          # cross prefill
 DEC = dict(B=16, lo=65536, hi=131072, Hq=32, Hkv=8, D=128, layers=16, d=4096, seed=2000)
 SWA = dict(B=4, T=65536, W=1024, Hq=32, Hkv=8, D=128, d=4096)
+SELF_LAYERS = 14    # self-decoder depth of the early-exit measurement (half of a 28-layer stack)
 
 
 def parse_args():
@@ -55,6 +56,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["yoco", "reference"], default="yoco")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-early-exit", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer"],
                     default=None,
@@ -286,6 +288,80 @@ def new_events():
     mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     return {"swa": mk(2), "gkv": mk(2), "decode": mk(2), "prefill_l": mk(2 * P["layers"]),
             "decode_l": mk(2 * DEC["layers"]), "step": mk(2)}
+
+
+def early_exit(W, reps):
+    """Early-exit prefill against the full prefill of one prompt, attention core
+    only ("You Only Cache Once", paperlayer summary, section 2: the prompt rows
+    skip the cross-decoder, only the last row goes through it).  Both run the
+    self-decoder (SELF_LAYERS sliding-window layers: K/V projection with the
+    YOCO++ blend, then SWA prefill with the ring fill) and the global K/V
+    projection over the T=32768 prompt; then the full prefill runs the 14
+    cross layers over every row, the early exit one cross decode of the last
+    row per cross layer.  Query / output projections and feed-forward layers
+    are not part of the attention core and are left out of both.  Returns
+    device milliseconds per prompt (mean over reps after one warm-up)."""
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    import workloads as wl
+    bf, dev = torch.bfloat16, W["o"].device
+    T, Hq, Hkv, D, d, Wn = P["T"], P["Hq"], P["Hkv"], P["D"], P["d"], SWA["W"]
+    x = wl.normal((T, d), 4001, bf, dev)
+    ws_ = [wl.normal((2 * Hkv * D, d), 4100 + l, bf, dev, std=d ** -0.5) for l in range(SELF_LAYERS)]
+    w_l = [float(v) for v in wl.uniform((SELF_LAYERS,), 4002)]
+    k1, v1, kl, vl = (torch.empty((1, T, Hkv, D), dtype=bf, device=dev) for _ in range(4))
+    q = wl.normal((1, T, Hq, D), 4003, bf, dev)
+    o = torch.empty((1, T, Hq, D), dtype=bf, device=dev)
+    ring = (torch.empty((1, Wn, Hkv, D), dtype=bf, device=dev), torch.empty((1, Wn, Hkv, D), dtype=bf, device=dev),
+            torch.empty((1, Wn), dtype=torch.int32, device=dev))
+    qlast = [q_.view(T, Hq, D)[T - 1:].contiguous() for q_ in W["qs"]]
+    od = torch.empty((1, Hq, D), dtype=bf, device=dev)
+    ss = torch.zeros(1, dtype=torch.int64, device=dev)
+    sl = torch.full((1,), T, dtype=torch.int32, device=dev)
+    wsd = torch.empty(yoco.cross_decode_workspace_size(1, T, Hq, Hkv, D, bf), dtype=torch.uint8, device=dev)
+
+    def self_decoder():
+        for l in range(SELF_LAYERS):
+            if l == 0:
+                yoco.kv_project_blend(x, ws_[0], Hkv, D, k_out=k1.view(-1, Hkv, D), v_out=v1.view(-1, Hkv, D))
+                k, v = k1, v1
+            else:
+                yoco.kv_project_blend(x, ws_[l], Hkv, D, k1.view(-1, Hkv, D), v1.view(-1, Hkv, D), w_l[l], w_l[l],
+                                      k_out=kl.view(-1, Hkv, D), v_out=vl.view(-1, Hkv, D))
+                k, v = kl, vl
+            yoco.swa_prefill(q, k, v, Wn, ring=ring, o=o)
+        yoco.kv_project_blend(W["x_mid"], W["w_g"], Hkv, D, k_out=W["kg"].view(-1, Hkv, D),
+                              v_out=W["vg"].view(-1, Hkv, D))
+
+    def cross_full():
+        for l in range(P["layers"]):
+            yoco.cross_prefill(W["qs"][l], W["kg"], W["vg"], o=W["o"])
+
+    def cross_last_row():
+        for l in range(P["layers"]):
+            yoco.cross_decode(qlast[l], W["kg"].view(T, Hkv, D), W["vg"].view(T, Hkv, D), ss, sl, T,
+                              workspace=wsd, o=od)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 1):
+            W["flush"].zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(); fn(); e1.record()
+            torch.cuda.synchronize()
+            if i > 0:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.mean(ts)
+
+    t_self = timed(self_decoder)
+    t_full = timed(cross_full)
+    t_ee = timed(cross_last_row)
+    return {"T": T, "self_layers": SELF_LAYERS, "cross_layers": P["layers"], "window": Wn,
+            "self_decoder_ms": t_self, "cross_full_ms": t_full, "cross_last_row_ms": t_ee,
+            "prefill_full_ms": t_self + t_full, "prefill_early_exit_ms": t_self + t_ee,
+            "speedup": (t_self + t_full) / (t_self + t_ee),
+            "note": "attention core only (no Q/O projections, no feed-forward); self_decoder_ms "
+                    "includes the global K/V projection"}
 
 
 def e2e_prefill(W, steps, warmup):
@@ -551,6 +627,8 @@ def main():
         e2e_ms = reduce_max_over_ranks([sum(times)], dev)[0]
         out["e2e"] = {"value": world * len(times) * P["layers"] * f_layer / (e2e_ms * 1e-3) / 1e12,
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if not args.no_early_exit:
+        out["early_exit"] = early_exit(W, 3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(W, args.cpu_seconds)
     if world > 1:

@@ -583,32 +583,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (warp == kConsumerWarps && lane == 0) producer_drain(full, it, p.stages);
 }
 
+// Split merge: one CTA of kMergeWarps warps per (sequence, query head).  Warp
+// w takes the chunks of 32 partial entries w, w + kMergeWarps, ...; it forms
+// its own max, its lanes weight 32 entries at once and its weighted sum keeps
+// several partial rows in flight per lane; the warps' (max, sum, row) are then
+// combined through shared memory.  With one warp per (sequence, head), a
+// single long sequence left the merge with a few dozen warps to read
+// hundreds of partial rows each.
+constexpr int kMergeWarps = 8;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const float *ws_o, const float *ws_ml,
-                                                           const int32_t *seq_len, int32_t window,
-                                                           int32_t B, int32_t Hq, int64_t split,
-                                                           int64_t n_split, int32_t sub, T *o,
-                                                           float *lse) {
+__global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(
+    const float *ws_o, const float *ws_ml, const int32_t *seq_len, int32_t window, int32_t B, int32_t Hq,
+    int64_t split, int64_t n_split, int32_t sub, T *o, float *lse) {
+    constexpr int DPL = D / 32;
+    __shared__ float s_m[kMergeWarps], s_l[kMergeWarps];
+    __shared__ float s_acc[kMergeWarps][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t idx = (int64_t)blockIdx.x * 4 + warp;
-    if (idx >= (int64_t)B * Hq) return;
-    const int b = (int)(idx / Hq), h = (int)(idx % Hq);
+    const int b = (int)(blockIdx.x / Hq), h = (int)(blockIdx.x % Hq);
     const int64_t len = seq_len ? (int64_t)seq_len[b] : (int64_t)window;
-    const int64_t n_s = min(n_split, max((int64_t)0, (len + split - 1) / split));
+    const int64_t n_s = sched::decode_units(len, split, n_split);
     const int64_t n_e = n_s * sub;
     const int64_t e0 = (int64_t)b * n_split * sub;
 
     float M = -INFINITY;
-    for (int64_t e = lane; e < n_e; e += 32) M = fmaxf(M, ws_ml[((e0 + e) * Hq + h) * 2]);
+    for (int64_t c = (int64_t)warp * 32; c < n_e; c += 32 * kMergeWarps) {
+        const int64_t e = c + lane;
+        if (e < n_e) M = fmaxf(M, ws_ml[((e0 + e) * Hq + h) * 2]);
+    }
     M = warp_max(M);
-    // lanes compute the weights of 32 entries at a time; the weighted sum then
-    // walks those entries with several partial rows in flight per lane
     float Lp = 0.f;
-    constexpr int DPL = D / 32;
     float acc[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-    for (int64_t c = 0; c < n_e; c += 32) {
+    for (int64_t c = (int64_t)warp * 32; c < n_e; c += 32 * kMergeWarps) {
         const int64_t e = c + lane;
         float w = 0.f;
         if (e < n_e) {
@@ -626,11 +634,32 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *ws_o, co
         }
     }
     const float L = warp_sum(Lp);
-    const float inv = L > 0.f ? 1.f / L : 0.f;
+    if (lane == 0) {
+        s_m[warp] = M;
+        s_l[warp] = L;
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) s_acc[warp][lane + 32 * i] = acc[i];
+    __syncthreads();
+    if (warp != 0) return;
+    float Mg = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) Mg = fmaxf(Mg, s_m[w]);
+    float Lg = 0.f, out[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) out[i] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) {
+        const float f = (s_m[w] == -INFINITY) ? 0.f : exp2f(s_m[w] - Mg);
+        Lg = fmaf(s_l[w], f, Lg);
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) out[i] = fmaf(s_acc[w][lane + 32 * i], f, out[i]);
+    }
+    const float inv = Lg > 0.f ? 1.f / Lg : 0.f;
     T *dst = o + ((int64_t)b * Hq + h) * D;
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) dst[lane + 32 * i] = from_f32<T>(acc[i] * inv);
-    if (lse && lane == 0) lse[(int64_t)b * Hq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    for (int i = 0; i < DPL; ++i) dst[lane + 32 * i] = from_f32<T>(out[i] * inv);
+    if (lse && lane == 0) lse[(int64_t)b * Hq + h] = Lg > 0.f ? (Mg + log2f(Lg)) * kLn2 : -INFINITY;
 }
 
 bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dtype,
@@ -721,8 +750,8 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
     }
     note_launches(2);
     if (e != cudaSuccess) return e;
-    const int mgrid = (int)(((int64_t)a.B * a.Hq + 3) / 4);
-    decode_merge_kernel<T, D><<<mgrid, 128, 0, st>>>(p.ws_o, p.ws_ml, a.seq_len, a.window, a.B,
+    const int mgrid = (int)((int64_t)a.B * a.Hq);
+    decode_merge_kernel<T, D><<<mgrid, 32 * kMergeWarps, 0, st>>>(p.ws_o, p.ws_ml, a.seq_len, a.window, a.B,
                                                      a.Hq, pl.split, pl.n_split, pl.sub,
                                                      static_cast<T *>(a.o), a.lse);
     return cudaGetLastError();

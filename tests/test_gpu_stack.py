@@ -105,3 +105,52 @@ def test_tiny_stack_prefill_and_decode(cuda_lib, dtype):
         assert_close(got["cross_o"][c], ref["cross_o"][c][:T], dtype, f"cross_o{c}", **tol)
     assert_close(got["x_prefill"], ref["x"][:T], dtype, "x prefill", **tol)
     assert_close(got["x_decode"], ref["x"][T:], dtype, "x decode", **tol)
+
+
+def gpu_early_exit(yoco, x, w, cfg):
+    """Early-exit prefill on the GPU: the self-decoder and the global K/V over
+    all T prompt rows, then only row T-1 through the cross layers, each a
+    cross decode of that row over the whole global K/V."""
+    T, Hq, Hkv, D, W = cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.window
+    dev = x.device
+    xs = x[:T].contiguous()
+    kb = vb = None
+    for l in range(cfg.n_self):
+        q = yoco.linear(xs, w["self_q"][l], apply_ln=True)
+        if l == 0:
+            k, v = yoco.kv_project_blend(xs, w["self_kv"][l], Hkv, D)
+            kb, vb = k, v
+        else:
+            k, v = yoco.kv_project_blend(xs, w["self_kv"][l], Hkv, D, kb, vb,
+                                         cfg.w_blend[l], cfg.w_blend[l])
+        o = yoco.swa_prefill(q.view(1, T, Hq, D), k.view(1, T, Hkv, D), v.view(1, T, Hkv, D), W)
+        xs = yoco.linear(o.view(T, Hq * D), w["self_o"][l], base=xs, base_w=1.0)
+    kg, vg = yoco.kv_project_blend(xs, w["g_kv"], Hkv, D)
+    xt = xs[T - 1:T].contiguous()
+    seq_start = torch.zeros(1, dtype=torch.int64, device=dev)
+    seq_len = torch.tensor([T], dtype=torch.int32, device=dev)
+    for c in range(cfg.n_cross):
+        q = yoco.linear(xt, w["cross_q"][c], apply_ln=True)
+        o = yoco.cross_decode(q.view(1, Hq, D), kg, vg, seq_start, seq_len, T)
+        xt = yoco.linear(o.view(1, Hq * D), w["cross_o"][c], base=xt, base_w=1.0)
+    return xt[0]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_tiny_stack_early_exit(cuda_lib, dtype):
+    # the last prompt row through the cross layers alone equals the full
+    # prefill's last row: against the oracle's early exit, and against the
+    # GPU's own full prefill
+    cfg = wl.TinyStack()
+    x, w = wl.tiny_stack_inputs(cfg, dtype)
+    T = cfg.T
+    ref = oracle.tiny_stack_early_exit(x[:T], w, cfg.Hq, cfg.Hkv, cfg.D, cfg.window, cfg.w_blend)
+    wc = {k: ([t.cuda() for t in v] if isinstance(v, list) else v.cuda()) for k, v in w.items()}
+    got = gpu_early_exit(cuda_lib, x.cuda(), wc, cfg)
+    full = gpu_stack(cuda_lib, x.cuda(), wc, cfg)["x_prefill"][T - 1]
+    if dtype == torch.float32:
+        tol = dict(max_abs=2e-3, rel_l2=2e-5)
+    else:
+        tol = dict(max_abs=1e-1, rel_l2=1.5e-2)
+    assert_close(got, ref, dtype, "early exit vs oracle", **tol)
+    assert_close(got, full.float().cpu().numpy(), dtype, "early exit vs full prefill", **tol)
