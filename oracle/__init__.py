@@ -55,6 +55,10 @@ def load(path):
     L.oracle_cache_bytes_transformer.argtypes = [i64, i64, i64, i64, i64]
     L.oracle_cache_bytes_transformer.restype = dbl
     L.oracle_visibility.argtypes = [i64, i64, i64, i64, ctypes.POINTER(ctypes.c_uint8)]
+    L.oracle_gret_log_decay.argtypes = [_D, i64, dbl, _D]
+    L.oracle_gret_recurrent.argtypes = [_D, _D, _D, _D, i64, i64, i64, i64, dbl, _D, _D]
+    L.oracle_gret_parallel.argtypes = [_D, _D, _D, _D, i64, i64, i64, i64, dbl, _D, _D]
+    L.oracle_gret_chunkwise.argtypes = [_D, _D, _D, _D, i64, i64, i64, i64, dbl, i64, _D, _D]
     L.oracle_num_threads.restype = i32
     L.oracle_set_num_threads.argtypes = [i32]
     return L
@@ -244,6 +248,55 @@ def cache_bytes_yoco(L_self, window, N, Hkv, D, elem_bytes):
 
 def cache_bytes_transformer(L, N, Hkv, D, elem_bytes):
     return lib().oracle_cache_bytes_transformer(L, N, Hkv, D, elem_bytes)
+
+
+# ------------------------------------------------------------ gated retention
+def gret_log_decay(g, tau):
+    """log gamma = log(sigmoid(g)) / tau, elementwise (any shape)."""
+    g = _f64(g)
+    out = np.empty_like(g)
+    lib().oracle_gret_log_decay(_p(g), g.size, float(tau), _p(out))
+    return out
+
+
+def _gret_args(q, k, v, log_gamma, scale, state):
+    q, k, v, lg = _f64(q), _f64(k), _f64(v), _f64(log_gamma)
+    B, T, H, D = q.shape
+    assert k.shape == q.shape and v.shape == q.shape and lg.shape == (B, T, H)
+    if scale is None:
+        scale = default_scale(D)
+    st = None if state is None else _f64(state).reshape(B, H, D, D).copy()
+    return q, k, v, lg, B, T, H, D, scale, st
+
+
+def gret_recurrent(q, k, v, log_gamma, scale=None, state=None):
+    """Recurrent gated retention.  q, k, v [B, T, H, D]; log_gamma [B, T, H];
+    state [B, H, D, D] initial state (None: zero).  Returns (o, final state)."""
+    q, k, v, lg, B, T, H, D, scale, st = _gret_args(q, k, v, log_gamma, scale, state)
+    if st is None:
+        st = np.zeros((B, H, D, D))
+    o = np.empty_like(q)
+    lib().oracle_gret_recurrent(_p(q), _p(k), _p(v), _p(lg), B, T, H, D, scale, _p(st), _p(o))
+    return o, st
+
+
+def gret_parallel(q, k, v, log_gamma, scale=None, state=None):
+    """Parallel gated retention (the same function as gret_recurrent's o)."""
+    q, k, v, lg, B, T, H, D, scale, st = _gret_args(q, k, v, log_gamma, scale, state)
+    o = np.empty_like(q)
+    lib().oracle_gret_parallel(_p(q), _p(k), _p(v), _p(lg), B, T, H, D, scale, _p(st), _p(o))
+    return o
+
+
+def gret_chunkwise(q, k, v, log_gamma, chunk, scale=None, state=None):
+    """Chunkwise gated retention with chunks of `chunk` tokens.  Returns
+    (o, final state)."""
+    q, k, v, lg, B, T, H, D, scale, st = _gret_args(q, k, v, log_gamma, scale, state)
+    if st is None:
+        st = np.zeros((B, H, D, D))
+    o = np.empty_like(q)
+    lib().oracle_gret_chunkwise(_p(q), _p(k), _p(v), _p(lg), B, T, H, D, scale, int(chunk), _p(st), _p(o))
+    return o, st
 
 
 def _self_decoder(x, weights, Hq, Hkv, D, window, w_blend, eps, out):

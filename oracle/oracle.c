@@ -280,3 +280,160 @@ double oracle_cache_bytes_transformer(int64_t L, int64_t N, int64_t Hkv, int64_t
                                       int64_t elem_bytes) {
     return 2.0 * (double)Hkv * (double)D * (double)elem_bytes * (double)N * (double)L;
 }
+
+/* ---------------------------------------------------------------------------
+ * Gated retention, the alternative self-decoder ("You Only Cache Once",
+ * paperlayer summary, section 3 "Design Choices of Self-Decoder", bullets
+ * "Gated Retention", and Appendix B "Chunk-wise Representation of Gated
+ * Retention"; podcast transcript cue 16).  The pages state the mechanism in
+ * words: retention (no softmax) with a data-dependent, head-wise scalar decay
+ * gate, sigmoid of the input raised to one over a temperature; a d x d state
+ * per head for decoding; a parallel, a recurrent and a chunkwise form that
+ * give the same result.  Written out (the readings are in the design notes):
+ *
+ *   gamma_t = sigmoid(g_t)^(1/tau)                    (g: gate logits)
+ *   S_t     = gamma_t S_{t-1} + scale * k_t^T v_t     (S: D x D, S_{-1} given)
+ *   o_t     = q_t S_t
+ *
+ * Layouts: q, k, v [B, T, H, D]; log_gamma [B, T, H]; state [B, H, D, D]
+ * with S[d][e] multiplying q_d into o_e. */
+
+/* log gamma = log(sigmoid(g)) / tau, without overflow for large |g|. */
+void oracle_gret_log_decay(const double *g, int64_t n, double tau, double *out) {
+    for (int64_t i = 0; i < n; ++i) {
+        double x = g[i];
+        double ls = x >= 0.0 ? -log1p(exp(-x)) : x - log1p(exp(x));
+        out[i] = ls / tau;
+    }
+}
+
+/* Recurrent form: one token at a time through the state.  state: [B,H,D,D]
+ * initial state on entry and final state on return; NULL starts from zero
+ * and discards the final state. */
+void oracle_gret_recurrent(const double *q, const double *k, const double *v,
+                           const double *log_gamma, int64_t B, int64_t T, int64_t H, int64_t D,
+                           double scale, double *state, double *o) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            double *S = (double *)calloc((size_t)(D * D), sizeof(double));
+            if (state) memcpy(S, state + (b * H + h) * D * D, sizeof(double) * (size_t)(D * D));
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t row = (b * T + t) * H + h;
+                const double gam = exp(log_gamma[row]);
+                const double *kt = k + row * D, *vt = v + row * D, *qt = q + row * D;
+                for (int64_t d = 0; d < D; ++d)
+                    for (int64_t e = 0; e < D; ++e) S[d * D + e] = gam * S[d * D + e] + scale * kt[d] * vt[e];
+                for (int64_t e = 0; e < D; ++e) {
+                    double acc = 0.0;
+                    for (int64_t d = 0; d < D; ++d) acc += qt[d] * S[d * D + e];
+                    o[row * D + e] = acc;
+                }
+            }
+            if (state) memcpy(state + (b * H + h) * D * D, S, sizeof(double) * (size_t)(D * D));
+            free(S);
+        }
+    }
+}
+
+/* Parallel form: o_t = sum_{s <= t} (prod_{i=s+1..t} gamma_i) scale (q_t . k_s) v_s
+ *                    + (prod_{i=0..t} gamma_i) q_t S_init.
+ * The products are exp of differences of the running sum of log gamma.
+ * state0: [B,H,D,D] initial state or NULL (zero). */
+void oracle_gret_parallel(const double *q, const double *k, const double *v,
+                          const double *log_gamma, int64_t B, int64_t T, int64_t H, int64_t D,
+                          double scale, const double *state0, double *o) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            double *c = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+            double run = 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                run += log_gamma[(b * T + t) * H + h];
+                c[t] = run;
+            }
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t rt = (b * T + t) * H + h;
+                const double *qt = q + rt * D;
+                double *ot = o + rt * D;
+                for (int64_t e = 0; e < D; ++e) ot[e] = 0.0;
+                for (int64_t s = 0; s <= t; ++s) {
+                    const int64_t rs = (b * T + s) * H + h;
+                    double dot = 0.0;
+                    for (int64_t d = 0; d < D; ++d) dot += qt[d] * k[rs * D + d];
+                    const double w = exp(c[t] - c[s]) * scale * dot;
+                    for (int64_t e = 0; e < D; ++e) ot[e] += w * v[rs * D + e];
+                }
+                if (state0) {
+                    const double *S = state0 + (b * H + h) * D * D;
+                    const double f = exp(c[t]);
+                    for (int64_t e = 0; e < D; ++e) {
+                        double acc = 0.0;
+                        for (int64_t d = 0; d < D; ++d) acc += qt[d] * S[d * D + e];
+                        ot[e] += f * acc;
+                    }
+                }
+            }
+            free(c);
+        }
+    }
+}
+
+/* Chunkwise form (Appendix B): chunks of C tokens; inside a chunk the
+ * parallel form over the chunk's own tokens (the inner-chunk part) plus the
+ * state carried in from the chunks before, decayed to each row (the
+ * cross-chunk part); at the chunk's end the state is decayed over the whole
+ * chunk and the chunk's keys and values are added with their decay to the
+ * chunk's end.  state: as in the recurrent form. */
+void oracle_gret_chunkwise(const double *q, const double *k, const double *v,
+                           const double *log_gamma, int64_t B, int64_t T, int64_t H, int64_t D,
+                           double scale, int64_t C, double *state, double *o) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            double *S = (double *)calloc((size_t)(D * D), sizeof(double));
+            double *a = (double *)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1));
+            if (state) memcpy(S, state + (b * H + h) * D * D, sizeof(double) * (size_t)(D * D));
+            for (int64_t j0 = 0; j0 < T; j0 += C) {
+                const int64_t len = (T - j0) < C ? (T - j0) : C;
+                double run = 0.0;  /* a[r] = sum of log gamma over the chunk's rows 0..r */
+                for (int64_t r = 0; r < len; ++r) {
+                    run += log_gamma[(b * T + j0 + r) * H + h];
+                    a[r] = run;
+                }
+                for (int64_t r = 0; r < len; ++r) {
+                    const int64_t rt = (b * T + j0 + r) * H + h;
+                    const double *qt = q + rt * D;
+                    double *ot = o + rt * D;
+                    /* cross-chunk part: the carried state, decayed to row r */
+                    const double f = exp(a[r]);
+                    for (int64_t e = 0; e < D; ++e) {
+                        double acc = 0.0;
+                        for (int64_t d = 0; d < D; ++d) acc += qt[d] * S[d * D + e];
+                        ot[e] = f * acc;
+                    }
+                    /* inner-chunk part */
+                    for (int64_t u = 0; u <= r; ++u) {
+                        const int64_t ru = (b * T + j0 + u) * H + h;
+                        double dot = 0.0;
+                        for (int64_t d = 0; d < D; ++d) dot += qt[d] * k[ru * D + d];
+                        const double w = exp(a[r] - a[u]) * scale * dot;
+                        for (int64_t e = 0; e < D; ++e) ot[e] += w * v[ru * D + e];
+                    }
+                }
+                /* state to the chunk's end */
+                const double fe = exp(a[len - 1]);
+                for (int64_t i = 0; i < D * D; ++i) S[i] *= fe;
+                for (int64_t u = 0; u < len; ++u) {
+                    const int64_t ru = (b * T + j0 + u) * H + h;
+                    const double w = exp(a[len - 1] - a[u]) * scale;
+                    for (int64_t d = 0; d < D; ++d)
+                        for (int64_t e = 0; e < D; ++e) S[d * D + e] += w * k[ru * D + d] * v[ru * D + e];
+                }
+            }
+            if (state) memcpy(state + (b * H + h) * D * D, S, sizeof(double) * (size_t)(D * D));
+            free(a);
+            free(S);
+        }
+    }
+}

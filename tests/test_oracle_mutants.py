@@ -31,6 +31,16 @@ MUTANTS = {
     "ring_push_slot": ("int64_t s = pos % W;", "int64_t s = (pos + 1) % W;"),
     "decode_drops_newest": ("int64_t n = seq_len[b];", "int64_t n = seq_len[b] - 1;"),
     "accounting_no_window": ("(double)L_self * (double)c", "(double)L_self"),
+    "gret_decay_after_add": ("S[d * D + e] = gam * S[d * D + e] + scale * kt[d] * vt[e];",
+                             "S[d * D + e] = gam * (S[d * D + e] + scale * kt[d] * vt[e]);"),
+    "gret_scale_dropped": ("const double w = exp(c[t] - c[s]) * scale * dot;",
+                           "const double w = exp(c[t] - c[s]) * dot;"),
+    "gret_state_transposed": ("for (int64_t d = 0; d < D; ++d) acc += qt[d] * S[d * D + e];\n                    o[row * D + e] = acc;",
+                              "for (int64_t d = 0; d < D; ++d) acc += qt[d] * S[e * D + d];\n                    o[row * D + e] = acc;"),
+    "gret_chunk_cross_undecayed": ("const double f = exp(a[r]);", "const double f = 1.0;"),
+    "gret_chunk_state_off_by_one": ("const double w = exp(a[len - 1] - a[u]) * scale;",
+                                    "const double w = exp(a[len - 1] - a[u] + log_gamma[(b * T + j0 + u) * H + h]) * scale;"),
+    "gret_gate_no_temperature": ("out[i] = ls / tau;", "out[i] = ls;"),
 }
 
 

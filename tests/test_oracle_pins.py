@@ -352,3 +352,89 @@ def test_tiny_stack_early_exit_is_exact():
     np.testing.assert_allclose(ee, full["x"][T - 1], rtol=0, atol=1e-12)
     # and it differs from the row before: the check is not vacuous
     assert np.abs(ee - full["x"][T - 2]).max() > 1e-3
+
+
+# ----------------------------------------------------------- gated retention
+def _gret_inputs(B, T, H, D, seed, gate_mean=2.0, tau=4.0):
+    q = _rand((B, T, H, D), seed)
+    k = _rand((B, T, H, D), seed + 1)
+    v = _rand((B, T, H, D), seed + 2)
+    g = _rand((B, T, H), seed + 3) * 2.0 + gate_mean
+    return q, k, v, oracle.gret_log_decay(g, tau)
+
+
+def test_gret_log_decay_is_a_tempered_sigmoid():
+    g = np.array([-50.0, -3.0, -0.5, 0.0, 0.7, 4.0, 50.0])
+    for tau in (1.0, 4.0, 16.0):
+        got = oracle.gret_log_decay(g, tau)
+        # gamma^tau is the sigmoid itself
+        np.testing.assert_allclose(np.exp(got * tau), 1.0 / (1.0 + np.exp(-g)), rtol=1e-12, atol=0)
+        assert np.all(got <= 0.0)
+    assert oracle.gret_log_decay(np.array([0.0]), 1.0)[0] == pytest.approx(np.log(0.5), abs=1e-15)
+
+
+@pytest.mark.parametrize("chunk", [1, 4, 16, 37, 64])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_gret_three_forms_agree(chunk, with_state):
+    # the pages: the parallel, recurrent and chunkwise forms give the same result
+    B, T, H, D = 2, 37, 3, 8
+    q, k, v, lg = _gret_inputs(B, T, H, D, 900)
+    s0 = _rand((B, H, D, D), 950) if with_state else None
+    o_r, s_r = oracle.gret_recurrent(q, k, v, lg, state=s0)
+    o_p = oracle.gret_parallel(q, k, v, lg, state=s0)
+    o_c, s_c = oracle.gret_chunkwise(q, k, v, lg, chunk, state=s0)
+    np.testing.assert_allclose(o_p, o_r, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(o_c, o_r, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(s_c, s_r, rtol=1e-11, atol=1e-11)
+
+
+def test_gret_without_decay_is_cumulative_linear_attention():
+    # gamma = 1: o_t = scale * q_t (sum_{s<=t} k_s^T v_s), by numpy cumsum
+    B, T, H, D = 1, 20, 2, 6
+    q, k, v, _ = _gret_inputs(B, T, H, D, 910)
+    lg = np.zeros((B, T, H))
+    scale = 0.37
+    states = np.cumsum(np.einsum("bthd,bthe->bthde", k, v), axis=1)
+    expect = scale * np.einsum("bthd,bthde->bthe", q, states)
+    o, s = oracle.gret_recurrent(q, k, v, lg, scale=scale)
+    np.testing.assert_allclose(o, expect, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s, scale * states[:, -1], rtol=1e-12, atol=1e-12)
+
+
+def test_gret_full_decay_keeps_only_the_current_token():
+    # gamma -> 0: o_t = scale * (q_t . k_t) v_t
+    B, T, H, D = 2, 9, 2, 5
+    q, k, v, _ = _gret_inputs(B, T, H, D, 920)
+    lg = np.full((B, T, H), -1e4)
+    o = oracle.gret_parallel(q, k, v, lg, scale=0.5)
+    expect = 0.5 * np.einsum("bthd,bthd->bth", q, k)[..., None] * v
+    np.testing.assert_allclose(o, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_gret_constant_decay_is_geometric():
+    # constant gamma: weight gamma^(t-s) on token s, written as an explicit loop
+    B, T, H, D = 1, 12, 1, 4
+    q, k, v, _ = _gret_inputs(B, T, H, D, 930)
+    gam = 0.8
+    lg = np.full((B, T, H), np.log(gam))
+    expect = np.zeros_like(q)
+    for t in range(T):
+        for s in range(t + 1):
+            expect[0, t, 0] += gam ** (t - s) * 0.25 * np.dot(q[0, t, 0], k[0, s, 0]) * v[0, s, 0]
+    o, _ = oracle.gret_chunkwise(q, k, v, lg, 5, scale=0.25)
+    np.testing.assert_allclose(o, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_gret_state_continues_across_calls():
+    # prefill of T1 tokens, then T2 more from the carried state == one run of T1 + T2
+    B, T, H, D = 2, 30, 2, 6
+    q, k, v, lg = _gret_inputs(B, T, H, D, 940)
+    o_all, s_all = oracle.gret_recurrent(q, k, v, lg)
+    o1, s1 = oracle.gret_chunkwise(q[:, :17], k[:, :17], v[:, :17], lg[:, :17], 8)
+    o2, s2 = oracle.gret_recurrent(q[:, 17:], k[:, 17:], v[:, 17:], lg[:, 17:], state=s1)
+    np.testing.assert_allclose(np.concatenate([o1, o2], 1), o_all, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(s2, s_all, rtol=1e-11, atol=1e-11)
+    # and the decay applies to the state before the token's own k^T v is added
+    o_first, _ = oracle.gret_recurrent(q[:, :1], k[:, :1], v[:, :1], lg[:, :1])
+    np.testing.assert_allclose(o_first[:, 0], (1.0 / np.sqrt(D)) * np.einsum("bhd,bhd->bh", q[:, 0], k[:, 0])[..., None]
+                               * v[:, 0], rtol=1e-12, atol=1e-12)
