@@ -174,6 +174,29 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
                         int32_t apply_ln, float ln_eps, const void *base, float base_w,
                         void *out, int32_t dtype, cudaStream_t stream);
 
+/* Gated retention, the alternative self-decoder ("You Only Cache Once",
+ * paperlayer summary, section 3 "Gated Retention" and Appendix B; podcast
+ * transcript cue 16).  Per head h, with a D x D fp32 state S:
+ *   gamma_t = sigmoid(g_t)^(1/tau),  S_t = gamma_t S_{t-1} + scale k_t^T v_t,
+ *   o_t = q_t S_t,
+ * scale = cfg->scale (0: 1/sqrt(D)).  Query and key/value heads are the same
+ * heads: cfg->Hq == cfg->Hkv == H.
+ *
+ * yoco_gret_prefill: chunkwise over a prompt.  q, k, v, o [B, T, H, D] (bf16;
+ * fp32 returns YOCO_ERR_UNSUPPORTED); g [B, T, H] fp32 gate logits; tau > 0.
+ * state [B, H, D, D] fp32, S[d][e] multiplying q_d into o_e: the initial state
+ * on entry and the final state on return, or NULL to start from zero and
+ * drop the final state.  Caller-owned device memory; asynchronous on stream. */
+yoco_status yoco_gret_prefill(const void *q, const void *k, const void *v, const float *g, int32_t B,
+                              int64_t T, float tau, float *state, void *o, const yoco_attn_cfg *cfg,
+                              cudaStream_t stream);
+
+/* yoco_gret_decode: one recurrent step.  q, k, v, o [B, H, D] (bf16 or fp32);
+ * g [B, H] fp32; state [B, H, D, D] fp32, read and updated in place
+ * (required). */
+yoco_status yoco_gret_decode(const void *q, const void *k, const void *v, const float *g, int32_t B,
+                             float tau, float *state, void *o, const yoco_attn_cfg *cfg, cudaStream_t stream);
+
 /* Test-only, with no counterpart on the pages: the work plan the kernels
  * follow, computed on the host by the kernels' own schedule functions, so
  * that tests can check it against the visibility rule pair by pair.  Reads

@@ -9,6 +9,7 @@ importing a function fails loudly when libyoco.so is missing.
 
 Entry points (same names as the C ABI, without the ``yoco_`` prefix):
 kv_project_blend, swa_prefill, swa_decode, cross_prefill, cross_decode,
+gret_prefill, gret_decode,
 plus linear, workspace sizes, cache_bytes, device_status and the test-only
 debug_tile_schedule.
 """
@@ -20,7 +21,7 @@ import torch
 __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_prefill",
            "swa_decode", "cross_prefill", "cross_decode", "cross_decode_workspace_size",
            "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg",
-           "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE"]
+           "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE", "gret_prefill", "gret_decode"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -72,6 +73,8 @@ def load():
         "yoco_cross_decode_workspace_size": (sz, [i32, i64, cfgp]),
         "yoco_swa_decode_workspace_size": (sz, [i32, i32, cfgp]),
         "yoco_cache_bytes": (ctypes.c_double, [i32, i32, i64, cfgp]),
+        "yoco_gret_prefill": (st, [vp, vp, vp, vp, i32, i64, f32, vp, vp, cfgp, vp]),
+        "yoco_gret_decode": (st, [vp, vp, vp, vp, i32, f32, vp, vp, cfgp, vp]),
         "yoco_debug_tile_schedule": (st, [i32, cfgp, i32, i64, i64, i64, i32, vp, vp, i64, i32, vp,
                                           i64, ctypes.POINTER(ctypes.c_int64)]),
         "yoco_get_device_status": (st, [vp]),
@@ -272,3 +275,32 @@ def debug_tile_schedule(kind, Hq, Hkv, D, dtype=torch.bfloat16, B=1, Tq=0, Tkv=0
     _check(L.yoco_debug_tile_schedule(*args(out.ctypes.data_as(ctypes.c_void_p), n.value)),
            "yoco_debug_tile_schedule")
     return out
+
+
+def gret_prefill(q, k, v, g, tau, state=None, scale=0.0, o=None):
+    """Chunkwise gated retention over a prompt.  q, k, v [B, T, H, D] bf16;
+    g [B, T, H] fp32 gate logits; state [B, H, D, D] fp32 initial state,
+    overwritten with the final state (None: start from zero).  Returns o."""
+    L = load()
+    B, T, H, D = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    _dev(q, k, v, g, state, o)
+    cfg = _cfg(H, H, D, q.dtype, scale)
+    _check(L.yoco_gret_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, T, float(tau), _ptr(state), _ptr(o),
+                               ctypes.byref(cfg), _stream()), "yoco_gret_prefill")
+    return o
+
+
+def gret_decode(q, k, v, g, tau, state, scale=0.0, o=None):
+    """One recurrent gated-retention step.  q, k, v [B, H, D]; g [B, H] fp32;
+    state [B, H, D, D] fp32, updated in place.  Returns o [B, H, D]."""
+    L = load()
+    B, H, D = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    _dev(q, k, v, g, state, o)
+    cfg = _cfg(H, H, D, q.dtype, scale)
+    _check(L.yoco_gret_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, float(tau), _ptr(state), _ptr(o),
+                              ctypes.byref(cfg), _stream()), "yoco_gret_decode")
+    return o

@@ -232,6 +232,38 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     return from_cuda(launch_decode(a, pl, stream));
 }
 
+yoco_status yoco_gret_prefill(const void *q, const void *k, const void *v, const float *g, int32_t B,
+                              int64_t T, float tau, float *state, void *o, const yoco_attn_cfg *cfg,
+                              cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (cfg->Hq != cfg->Hkv || B < 0 || T < 0 || !(tau > 0.f) || isinf(tau)) return YOCO_ERR_INVALID;
+    if (B == 0 || T == 0) return YOCO_OK;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_opt(state) || !ok_ptr(o))
+        return YOCO_ERR_INVALID;
+    if (cfg->dtype != YOCO_BF16) return YOCO_ERR_UNSUPPORTED;
+    GretArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.state = state; a.o = o;
+    a.B = B; a.H = cfg->Hq; a.D = cfg->D; a.dtype = cfg->dtype; a.T = T;
+    a.tau = tau; a.scale = eff_scale(cfg);
+    return from_cuda(launch_gret_prefill(a, stream));
+}
+
+yoco_status yoco_gret_decode(const void *q, const void *k, const void *v, const float *g, int32_t B,
+                             float tau, float *state, void *o, const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (cfg->Hq != cfg->Hkv || B < 0 || !(tau > 0.f) || isinf(tau)) return YOCO_ERR_INVALID;
+    if (B == 0) return YOCO_OK;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(state) || !ok_ptr(o))
+        return YOCO_ERR_INVALID;
+    GretArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.state = state; a.o = o;
+    a.B = B; a.H = cfg->Hq; a.D = cfg->D; a.dtype = cfg->dtype; a.T = 1;
+    a.tau = tau; a.scale = eff_scale(cfg);
+    return from_cuda(launch_gret_decode(a, stream));
+}
+
 yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int32_t B, int64_t Tq,
                                      int64_t Tkv, int64_t q_pos0, int32_t window,
                                      const int64_t *seq_start, const int32_t *seq_len, int64_t max_len,

@@ -101,6 +101,21 @@ cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
 // LayerNorm folded into the epilogue.  cudaErrorNotSupported otherwise.
 cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
 
+// ------------------------------------------------------- gated retention
+struct GretArgs {
+    const void *q, *k, *v;  // prefill [B, T, H, D], decode [B, H, D]
+    const float *g;         // gate logits: prefill [B, T, H], decode [B, H]
+    float *state;           // [B, H, D, D] fp32: prefill in/out or null, decode in/out
+    void *o;                // like q
+    int32_t B, H, D, dtype;
+    int64_t T;              // prefill only
+    float tau, scale;
+};
+// Chunkwise prefill (bf16; cudaErrorNotSupported for other dtypes).
+cudaError_t launch_gret_prefill(const GretArgs &a, cudaStream_t s);
+// One recurrent decode step (bf16 or fp32).
+cudaError_t launch_gret_decode(const GretArgs &a, cudaStream_t s);
+
 // Device status words of the translation units that hold bounded waits.
 unsigned int read_and_clear_status_decode();
 unsigned int read_and_clear_status_prefill_tc();

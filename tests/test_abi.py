@@ -85,6 +85,26 @@ def test_bad_arguments_rejected_before_launch():
     assert L.yoco_kv_project_blend(FAKE, 0, 64, FAKE, 1, 1e-5, None, None, 0.0, 0.0, None, FAKE, FAKE, b, None) == yoco.OK
 
 
+def test_gret_arguments_rejected_before_launch():
+    L = yoco.load()
+    same = ctypes.byref(_cfg(Hq=8, Hkv=8))
+    grouped = ctypes.byref(_cfg(Hq=8, Hkv=2))
+    fp32 = ctypes.byref(_cfg(Hq=8, Hkv=8, dtype=1))
+    # heads must match, tau > 0, pointers valid
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, None, FAKE, grouped, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 0.0, None, FAKE, same, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, None, 1, 64, 4.0, None, FAKE, same, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, MISALIGNED, FAKE, same, None) == yoco.ERR_INVALID
+    # the chunkwise prefill is built for bf16 only
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, None, FAKE, fp32, None) == yoco.ERR_UNSUPPORTED
+    # decode needs its state
+    assert L.yoco_gret_decode(FAKE, FAKE, FAKE, FAKE, 1, 4.0, None, FAKE, same, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_decode(FAKE, FAKE, FAKE, FAKE, 1, -1.0, FAKE, FAKE, same, None) == yoco.ERR_INVALID
+    # empty inputs: successful no-op
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 0, 64, 4.0, None, FAKE, same, None) == yoco.OK
+    assert L.yoco_gret_decode(FAKE, FAKE, FAKE, FAKE, 0, 4.0, FAKE, FAKE, same, None) == yoco.OK
+
+
 def test_workspace_size_monotone_and_positive():
     sizes = [yoco.cross_decode_workspace_size(B, L, 32, 8, 128, torch.bfloat16)
              for B, L in [(1, 1), (1, 4096), (16, 131072), (16, 262144)]]
