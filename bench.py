@@ -46,6 +46,8 @@ P = dict(T=32768, Hq=32, Hkv=8, D=128, layers=14, d=4096)          # cross prefi
 DEC = dict(B=16, lo=65536, hi=131072, Hq=32, Hkv=8, D=128, layers=16, d=4096, seed=2000)
 SWA = dict(B=4, T=65536, W=1024, Hq=32, Hkv=8, D=128, d=4096)
 SELF_LAYERS = 14    # self-decoder depth of the early-exit measurement (half of a 28-layer stack)
+# gated-retention self-decoder layer (the sliding-window slice's shape with retention heads)
+GRET = dict(B=4, T=65536, H=32, D=128, tau=16.0, B_dec=16)
 
 
 def parse_args():
@@ -58,7 +60,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-early-exit", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer"],
+    ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer",
+                                       "gret", "gret_decode"],
                     default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
@@ -116,6 +119,16 @@ def reduce_max_over_ranks(values, device=None):
     t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(v) for v in t.tolist()]
+
+
+def gret_flops(B, T, H, D, chunk=64):
+    """Tensor FLOPs of chunkwise gated retention at the kernel's chunk size: per
+    chunk and head, Q K^T and P V over the chunk's causal pairs (counted in
+    full, C x C) plus the cross term Q S and the state update K^T V (D x D
+    each), 2 FLOP per multiply-add."""
+    n_chunks = -(-T // chunk)
+    per_chunk = 2 * (2.0 * chunk * chunk * D) + 2 * (2.0 * chunk * D * D)
+    return B * H * n_chunks * per_chunk
 
 
 def prefill_flops_per_layer(T, Hq, D, q_pos0=0, window=0):
@@ -364,6 +377,44 @@ def early_exit(W, reps):
                     "includes the global K/V projection"}
 
 
+def gret_layer(W, reps):
+    """The gated-retention self-decoder layer, measured beside the step (it is
+    not part of it): the chunkwise prefill over B=4 x T=65536 tokens with 32
+    heads, then one decode step for a batch of 16.  Device ms, mean over reps."""
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    import workloads as wl
+    bf, dev = torch.bfloat16, W["o"].device
+    B, T, H, D, tau, Bd = GRET["B"], GRET["T"], GRET["H"], GRET["D"], GRET["tau"], GRET["B_dec"]
+    q, k, v = (wl.normal((B, T, H, D), 5001 + i, bf, dev) for i in range(3))
+    g = wl.normal((B, T, H), 5004, torch.float32, dev) + 3.0
+    o = torch.empty_like(q)
+    st = torch.zeros((B, H, D, D), dtype=torch.float32, device=dev)
+    qd, kd, vd = (wl.normal((Bd, H, D), 5011 + i, bf, dev) for i in range(3))
+    gd = wl.normal((Bd, H), 5014, torch.float32, dev) + 3.0
+    sd = torch.zeros((Bd, H, D, D), dtype=torch.float32, device=dev)
+    od = torch.empty_like(qd)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 1):
+            W["flush"].zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(); fn(); e1.record()
+            torch.cuda.synchronize()
+            if i > 0:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.mean(ts)
+
+    t_pre = timed(lambda: yoco.gret_prefill(q, k, v, g, tau, state=st, o=o))
+    t_dec = timed(lambda: yoco.gret_decode(qd, kd, vd, gd, tau, sd, o=od))
+    return {"prefill_ms": t_pre, "prefill_tflops": gret_flops(B, T, H, D) / (t_pre * 1e-3) / 1e12,
+            "prefill_tokens_per_s": B * T / (t_pre * 1e-3),
+            "decode_ms": t_dec, "decode_gbs": Bd * H * D * D * 8.0 / (t_dec * 1e-3) / 1e9,
+            "shape": f"prefill B={B} T={T} H={H} D={D}; decode batch {Bd}",
+            "flops": "chunkwise at chunk 64: QK^T and PV over C x C, Q S and K^T V over D x D, per chunk and head"}
+
+
 def e2e_prefill(W, steps, warmup):
     """Prefill through the public API with HOST buffers: every step copies the
     step's Q (14 layers) and the shared K/V from pinned host memory and reads
@@ -470,6 +521,8 @@ def run_case(args):
       proj     K/V projection + blend, 32768 tokens, d=4096 (x 256 MB)
       prefill_layer / decode_layer  one launch of the full benchmark's own
                prefill layer (T=32768) / decode layer (batch 16, 64K-128K)
+      gret     gated-retention chunkwise prefill B=4, T=65536, 32 heads, D=128
+      gret_decode  one gated-retention decode step, batch 16, 32 heads (state 34 MB, L2 flushed)
     Prints one JSON line with the mean launch time and the work rate."""
     import torch
     import shared_kv_decoder_b200 as yoco
@@ -501,6 +554,21 @@ def run_case(args):
         v = wl.normal((1, T, Hkv, D), 9, bf, dev); o = torch.empty_like(q)
         fn = lambda: yoco.swa_prefill(q, k, v, Wn, o=o)
         work, unit = prefill_flops_per_layer(T, Hq, D, 0, Wn), "TFLOP/s"
+    elif args.case == "gret":
+        B, T, H = GRET["B"], GRET["T"], GRET["H"]
+        q = wl.normal((B, T, H, D), 14, bf, dev); k = wl.normal((B, T, H, D), 15, bf, dev)
+        v = wl.normal((B, T, H, D), 16, bf, dev); g = wl.normal((B, T, H), 17, torch.float32, dev) + 3.0
+        o = torch.empty_like(q)
+        fn = lambda: yoco.gret_prefill(q, k, v, g, GRET["tau"], o=o)
+        work, unit = gret_flops(B, T, H, D), "TFLOP/s"
+    elif args.case == "gret_decode":
+        B, H = GRET["B_dec"], GRET["H"]
+        q = wl.normal((B, H, D), 18, bf, dev); k = wl.normal((B, H, D), 19, bf, dev)
+        v = wl.normal((B, H, D), 20, bf, dev); g = wl.normal((B, H), 21, torch.float32, dev) + 3.0
+        st = torch.zeros((B, H, D, D), dtype=torch.float32, device=dev)
+        o = torch.empty_like(q)
+        fn = lambda: yoco.gret_decode(q, k, v, g, GRET["tau"], st, o=o)
+        work, unit = B * H * D * D * 4.0 * 2, "GB/s"
     else:
         n, d = 32768, 4096
         x = wl.normal((n, d), 10, bf, dev); w = wl.normal((2 * Hkv * D, d), 11, bf, dev, std=d ** -0.5)
@@ -629,6 +697,7 @@ def main():
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     if not args.no_early_exit:
         out["early_exit"] = early_exit(W, 3)
+        out["gret"] = gret_layer(W, 3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(W, args.cpu_seconds)
     if world > 1:
