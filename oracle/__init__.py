@@ -250,6 +250,34 @@ def cache_bytes_transformer(L, N, Hkv, D, elem_bytes):
     return lib().oracle_cache_bytes_transformer(L, N, Hkv, D, elem_bytes)
 
 
+# ------------------------------------------------------------- 8-bit K/V
+def quantize_kv_i8(x):
+    """Symmetric 8-bit quantisation of a K or V cache, one scale per (token,
+    KV head) (the pages' "8-bit cache quantization", podcast cue 1; the scheme
+    is not stated -- reading: absmax over the head's D values, scale =
+    absmax / 127, code = round-half-even(x / scale) in [-127, 127]).
+
+    x [rows, Hkv, D] (bf16 / fp32 tensor or array).  Every decision that
+    yields an integer is taken in fp32 (IEEE division, round-half-even), the
+    precision the kernel uses, so the codes are reproducible bit for bit.
+    Returns (codes int8 [rows, Hkv, D], scales float32 [rows, Hkv])."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().to("cpu", torch.float32).numpy()
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x), axis=-1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = np.rint((x / safe[..., None]).astype(np.float32))
+    q = np.where(scale[..., None] > 0, q, 0.0)
+    return np.clip(q, -127, 127).astype(np.int8), scale
+
+
+def dequantize_kv_i8(codes, scales):
+    """codes [rows, Hkv, D] int8, scales [rows, Hkv] -> fp64 values code * scale."""
+    return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
 # ------------------------------------------------------------ gated retention
 def gret_log_decay(g, tau):
     """log gamma = log(sigmoid(g)) / tau, elementwise (any shape)."""

@@ -438,3 +438,33 @@ def test_gret_state_continues_across_calls():
     o_first, _ = oracle.gret_recurrent(q[:, :1], k[:, :1], v[:, :1], lg[:, :1])
     np.testing.assert_allclose(o_first[:, 0], (1.0 / np.sqrt(D)) * np.einsum("bhd,bhd->bh", q[:, 0], k[:, 0])[..., None]
                                * v[:, 0], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------- 8-bit K/V
+def test_quantize_i8_worked_example():
+    # absmax 2.54 -> scale 0.02; 1.0 -> 50, -2.54 -> -127, 2.54 -> 127
+    x = np.array([[[1.0, -2.54, 0.01, 0.03, 2.54, -0.05]]], dtype=np.float32)
+    codes, scales = oracle.quantize_kv_i8(x)
+    s = np.float32(np.float32(2.54) / np.float32(127.0))
+    assert scales[0, 0] == s
+    expect = np.rint((x[0, 0] / s).astype(np.float32)).astype(np.int8)
+    np.testing.assert_array_equal(codes[0, 0], expect)
+    assert codes[0, 0, 1] == -127 and codes[0, 0, 4] == 127 and codes[0, 0, 0] == 50
+
+
+def test_quantize_i8_bounds_and_round_trip():
+    x = _rand((50, 8, 128), 960).astype(np.float32) * 3.0
+    x[3, 2] = 0.0                                    # an all-zero head row
+    codes, scales = oracle.quantize_kv_i8(x)
+    assert codes.dtype == np.int8 and codes.min() >= -127 and codes.max() <= 127
+    assert scales[3, 2] == 0 and not codes[3, 2].any()
+    # the largest magnitude of every head row maps to +-127
+    amax_idx = np.argmax(np.abs(x), axis=-1)
+    top = np.take_along_axis(codes, amax_idx[..., None], -1)[..., 0]
+    nz = scales > 0
+    assert np.all(np.abs(top[nz]) == 127)
+    # round trip within half a step (plus fp32 rounding of the step)
+    err = np.abs(oracle.dequantize_kv_i8(codes, scales) - x)
+    assert np.all(err <= 0.5 * scales[..., None] * (1 + 1e-6) + 1e-12)
+    # and the step really is absmax / 127
+    np.testing.assert_allclose(scales, np.abs(x).max(-1) / 127.0, rtol=1e-6)
