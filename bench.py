@@ -61,7 +61,7 @@ def parse_args():
     ap.add_argument("--no-early-exit", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer",
-                                       "gret", "gret_decode"],
+                                       "gret", "gret_decode", "decode_i8_layer"],
                     default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
@@ -523,6 +523,7 @@ def run_case(args):
                prefill layer (T=32768) / decode layer (batch 16, 64K-128K)
       gret     gated-retention chunkwise prefill B=4, T=65536, 32 heads, D=128
       gret_decode  one gated-retention decode step, batch 16, 32 heads (state 34 MB, L2 flushed)
+      decode_i8_layer  one decode layer over the 8-bit cache of the benchmark's decode shape
     Prints one JSON line with the mean launch time and the work rate."""
     import torch
     import shared_kv_decoder_b200 as yoco
@@ -554,6 +555,19 @@ def run_case(args):
         v = wl.normal((1, T, Hkv, D), 9, bf, dev); o = torch.empty_like(q)
         fn = lambda: yoco.swa_prefill(q, k, v, Wn, o=o)
         work, unit = prefill_flops_per_layer(T, Hq, D, 0, Wn), "TFLOP/s"
+    elif args.case == "decode_i8_layer":
+        lens = wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], DEC["seed"])
+        starts = torch.cumsum(torch.cat([torch.zeros(1, dtype=torch.int64), lens[:-1]]), 0)
+        rows = int(lens.sum())
+        kc = wl.normal((rows, Hkv, D), 4, bf, dev); vc = wl.normal((rows, Hkv, D), 5, bf, dev)
+        kq, vq = yoco.kv_quantize_i8(kc, vc)
+        del kc, vc
+        q = wl.normal((DEC["B"], Hq, D), 6, bf, dev); o = torch.empty_like(q)
+        ss, sl = starts.to(dev), lens.to(torch.int32).to(dev)
+        ws = torch.empty(yoco.cross_decode_workspace_size(DEC["B"], int(lens.max()), Hq, Hkv, D, bf),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: yoco.cross_decode_i8(q, kq, vq, Hkv, ss, sl, int(lens.max()), workspace=ws, o=o)
+        work, unit = rows * 2.0 * yoco.kv_i8_row_bytes(Hkv, D), "GB/s"
     elif args.case == "gret":
         B, T, H = GRET["B"], GRET["T"], GRET["H"]
         q = wl.normal((B, T, H, D), 14, bf, dev); k = wl.normal((B, T, H, D), 15, bf, dev)

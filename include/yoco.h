@@ -174,6 +174,29 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
                         int32_t apply_ln, float ln_eps, const void *base, float base_w,
                         void *out, int32_t dtype, cudaStream_t stream);
 
+/* 8-bit shared cache (podcast transcript, cue 1: the 65B example's "8-bit
+ * cache quantization"; the scheme is not stated).  Reading: symmetric int8,
+ * one fp32 scale per (token, KV head): scale = absmax / 127 over the head's D
+ * values, code = round-half-even(x / scale) (fp32, IEEE division), value =
+ * code * scale.  A cache row of an 8-bit K or V cache holds the token's
+ * Hkv x D codes, then its Hkv scales, padded to a multiple of 16 bytes:
+ * yoco_kv_i8_row_bytes(cfg) bytes (0 on bad arguments).
+ *
+ * yoco_kv_quantize_i8: k, v [n_tok, Hkv, D] (cfg->dtype) -> rows dst_rows[i]
+ * (a device int64 array, or NULL for rows 0..n_tok-1) of k_i8 / v_i8.
+ * Decode-time appends pass the new rows' indices, like yoco_kv_project_blend.
+ *
+ * yoco_cross_decode_i8: yoco_cross_decode over 8-bit caches (same q, o, lse,
+ * sequence and workspace arguments; the workspace size is
+ * yoco_cross_decode_workspace_size with the bf16 cfg).  Built for D = 128
+ * and bf16 q / o; other shapes return YOCO_ERR_UNSUPPORTED. */
+int64_t yoco_kv_i8_row_bytes(const yoco_attn_cfg *cfg);
+yoco_status yoco_kv_quantize_i8(const void *k, const void *v, int64_t n_tok, const int64_t *dst_rows, void *k_i8,
+                                void *v_i8, const yoco_attn_cfg *cfg, cudaStream_t stream);
+yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_i8, const int64_t *seq_start,
+                                 const int32_t *seq_len, int32_t B, int64_t max_len, void *o, float *lse,
+                                 void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream);
+
 /* Gated retention, the alternative self-decoder ("You Only Cache Once",
  * paperlayer summary, section 3 "Gated Retention" and Appendix B; podcast
  * transcript cue 16).  Per head h, with a D x D fp32 state S:

@@ -9,7 +9,7 @@ importing a function fails loudly when libyoco.so is missing.
 
 Entry points (same names as the C ABI, without the ``yoco_`` prefix):
 kv_project_blend, swa_prefill, swa_decode, cross_prefill, cross_decode,
-gret_prefill, gret_decode,
+gret_prefill, gret_decode, kv_quantize_i8, cross_decode_i8,
 plus linear, workspace sizes, cache_bytes, device_status and the test-only
 debug_tile_schedule.
 """
@@ -21,7 +21,8 @@ import torch
 __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_prefill",
            "swa_decode", "cross_prefill", "cross_decode", "cross_decode_workspace_size",
            "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg",
-           "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE", "gret_prefill", "gret_decode"]
+           "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE", "gret_prefill", "gret_decode",
+           "kv_i8_row_bytes", "kv_quantize_i8", "cross_decode_i8"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -74,6 +75,9 @@ def load():
         "yoco_swa_decode_workspace_size": (sz, [i32, i32, cfgp]),
         "yoco_cache_bytes": (ctypes.c_double, [i32, i32, i64, cfgp]),
         "yoco_gret_prefill": (st, [vp, vp, vp, vp, i32, i64, f32, vp, vp, cfgp, vp]),
+        "yoco_kv_i8_row_bytes": (i64, [cfgp]),
+        "yoco_kv_quantize_i8": (st, [vp, vp, i64, vp, vp, vp, cfgp, vp]),
+        "yoco_cross_decode_i8": (st, [vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
         "yoco_gret_decode": (st, [vp, vp, vp, vp, i32, f32, vp, vp, cfgp, vp]),
         "yoco_debug_tile_schedule": (st, [i32, cfgp, i32, i64, i64, i64, i32, vp, vp, i64, i32, vp,
                                           i64, ctypes.POINTER(ctypes.c_int64)]),
@@ -304,3 +308,45 @@ def gret_decode(q, k, v, g, tau, state, scale=0.0, o=None):
     _check(L.yoco_gret_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, float(tau), _ptr(state), _ptr(o),
                               ctypes.byref(cfg), _stream()), "yoco_gret_decode")
     return o
+
+
+def kv_i8_row_bytes(Hkv, D):
+    """Bytes of one row of an 8-bit K or V cache (codes, then padded scales)."""
+    return int(load().yoco_kv_i8_row_bytes(ctypes.byref(_cfg(Hkv, Hkv, D, torch.bfloat16))))
+
+
+def kv_quantize_i8(k, v, k_i8=None, v_i8=None, dst_rows=None):
+    """8-bit quantisation of K, V [n, Hkv, D] into cache rows (uint8 tensors
+    [rows, row_bytes]); dst_rows (int64, device) places row i at dst_rows[i].
+    Returns (k_i8, v_i8)."""
+    L = load()
+    n, Hkv, D = k.shape
+    rb = kv_i8_row_bytes(Hkv, D)
+    if k_i8 is None:
+        k_i8 = torch.empty((n, rb), dtype=torch.uint8, device=k.device)
+    if v_i8 is None:
+        v_i8 = torch.empty((n, rb), dtype=torch.uint8, device=k.device)
+    _dev(k, v, dst_rows, k_i8, v_i8)
+    cfg = _cfg(Hkv, Hkv, D, k.dtype)
+    _check(L.yoco_kv_quantize_i8(_ptr(k), _ptr(v), n, _ptr(dst_rows), _ptr(k_i8), _ptr(v_i8), ctypes.byref(cfg),
+                                 _stream()), "yoco_kv_quantize_i8")
+    return k_i8, v_i8
+
+
+def cross_decode_i8(q, k_i8, v_i8, Hkv, seq_start, seq_len, max_len, workspace=None, o=None, want_lse=False,
+                    scale=0.0):
+    """cross_decode over 8-bit caches (uint8 rows from kv_quantize_i8)."""
+    L = load()
+    B, Hq, D = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if want_lse else None
+    cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
+    if workspace is None:
+        n = L.yoco_cross_decode_workspace_size(B, int(max_len), ctypes.byref(cfg))
+        workspace = torch.empty(max(int(n), 16), dtype=torch.uint8, device=q.device)
+    _dev(q, k_i8, v_i8, seq_start, seq_len, o, lse, workspace)
+    _check(L.yoco_cross_decode_i8(_ptr(q), _ptr(k_i8), _ptr(v_i8), _ptr(seq_start), _ptr(seq_len), B,
+                                  int(max_len), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                  ctypes.byref(cfg), _stream()), "yoco_cross_decode_i8")
+    return (o, lse) if want_lse else o

@@ -232,6 +232,42 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     return from_cuda(launch_decode(a, pl, stream));
 }
 
+int64_t yoco_kv_i8_row_bytes(const yoco_attn_cfg *cfg) {
+    if (!cfg || cfg->Hkv < 1 || (cfg->D != 64 && cfg->D != 128)) return 0;
+    return i8_row_bytes(cfg->Hkv, cfg->D);
+}
+
+yoco_status yoco_kv_quantize_i8(const void *k, const void *v, int64_t n_tok, const int64_t *dst_rows, void *k_i8,
+                                void *v_i8, const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (n_tok < 0) return YOCO_ERR_INVALID;
+    if (n_tok == 0) return YOCO_OK;
+    if (!ok_ptr(k) || !ok_ptr(v) || !ok_opt(dst_rows) || !ok_ptr(k_i8) || !ok_ptr(v_i8)) return YOCO_ERR_INVALID;
+    return from_cuda(launch_kv_quantize_i8(k, v, n_tok, cfg->Hkv, cfg->D, cfg->dtype, dst_rows, k_i8, v_i8, stream));
+}
+
+yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_i8, const int64_t *seq_start,
+                                 const int32_t *seq_len, int32_t B, int64_t max_len, void *o, float *lse,
+                                 void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (B < 0 || max_len < 1) return YOCO_ERR_INVALID;
+    if (B == 0) return YOCO_OK;
+    if (!ok_ptr(q) || !ok_ptr(k_i8) || !ok_ptr(v_i8) || !ok_ptr(seq_start) || !seq_len || !ok_ptr(o) || !ok_opt(lse))
+        return YOCO_ERR_INVALID;
+    if (cfg->D != 128 || cfg->dtype != YOCO_BF16) return YOCO_ERR_UNSUPPORTED;
+    DecodePlan pl;
+    if (!make_decode_plan(B, max_len, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl)) return YOCO_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace) || ws_bytes < pl.ws_bytes) return YOCO_ERR_WORKSPACE;
+    DecodeArgs a;
+    a.q = q; a.k = k_i8; a.v = v_i8; a.seq_start = seq_start; a.seq_len = seq_len;
+    a.slot_pos = nullptr; a.pos = nullptr; a.window = 0;
+    a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
+    a.scale = eff_scale(cfg); a.o = o; a.lse = lse; a.ws = workspace;
+    return from_cuda(launch_decode_i8(a, pl, stream));
+}
+
 yoco_status yoco_gret_prefill(const void *q, const void *k, const void *v, const float *g, int32_t B,
                               int64_t T, float tau, float *state, void *o, const yoco_attn_cfg *cfg,
                               cudaStream_t stream) {

@@ -583,6 +583,337 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (warp == kConsumerWarps && lane == 0) producer_drain(full, it, p.stages);
 }
 
+// ---------------------------------------------------------------------------
+// Decode over an 8-bit cache (D = 128).  A cache row holds the Hkv x 128 int8
+// codes of one token, then its Hkv fp32 scales (padded to 16 bytes); a value
+// is code * scale.  A stage arrives as two 16 KB TMA boxes of codes ([head]
+// [token] rows of 128 bytes, 128-byte swizzle) and two small boxes of the
+// stage's scales -- half the bytes of the bf16 cache.  Each consumer warp
+// turns its head's 16 token rows of K and V into fp16 tiles in its own
+// shared-memory slice (exact: an int8 code fits fp16's mantissa; the byte is
+// placed under the exponent of 1024 and 1152 subtracted), then runs the same
+// mma.sync inner products in fp16.  The K scale multiplies the column of S
+// it belongs to, the V scale folds into P before P V, so the tensor cores see
+// integer-valued operands only.
+constexpr int kI8Stages = 4;
+constexpr int kI8TileLd = 136;  // fp16 elements per row of a warp's converted tile (272 bytes)
+
+struct DecodeI8Params {
+    DecodeKParams k;
+    int64_t row_bytes;   // bytes per cache row
+    int32_t scale_off;   // byte offset of the scales within a row
+    int32_t scale_bytes; // padded bytes of the scales per row
+};
+
+YOCO_DEV void mma_16816_f16(float *c, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+YOCO_DEV uint32_t pack2_f16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// four int8 codes -> two fp16x2 words, exactly
+YOCO_DEV void i8x4_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = w ^ 0x80808080u;  // code + 128, as unsigned bytes
+    const uint32_t bias = 0x64806480u;   // fp16 1152 = 1024 + 128, twice
+    uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);
+    uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(bias));
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    decode_i8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                     const DecodeI8Params pi) {
+    if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
+    constexpr int D = 128;
+    constexpr uint32_t kBox = kRowsPerStage * 128;  // one code box: 128 rows of 128 bytes
+    const DecodeKParams &p = pi.k;
+    const int ST = (int)p.stage_tokens;
+    const uint32_t sbox = (uint32_t)(ST * pi.scale_bytes);             // one scale box
+    const uint32_t stage_bytes = 2 * kBox + ((2 * sbox + 1023u) & ~1023u);
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - raw);
+    const uint32_t tiles = (uint32_t)kI8Stages * stage_bytes;           // converted fp16 tiles
+    const uint32_t tile_bytes = 2u * kTokPerWarp * kI8TileLd * 2u;      // K and V of one warp
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + tiles + kConsumerWarps * tile_bytes);
+    uint64_t *empty = full + kI8Stages;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kI8Stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const unsigned char *kg = static_cast<const unsigned char *>(p.k);
+    const unsigned char *vg = static_cast<const unsigned char *>(p.v);
+    uint32_t it = 0;
+
+    for (int64_t u = blockIdx.x;; u += gridDim.x) {
+        int b;
+        int64_t s;
+        if (!find_unit(p, u, &b, &s)) break;
+        const int64_t len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
+        const int64_t t0 = s * p.split;
+        const int64_t n_tok = min(p.split, len - t0);
+        const int64_t row0 = (p.seq_start ? p.seq_start[b] : (int64_t)b * p.window) + t0;
+        const int n_st = (int)((n_tok + ST - 1) / ST);
+
+        if (warp == kConsumerWarps) {
+            // ---------------------------------------------------- producer
+            for (int i = 0; i < n_st; ++i) {
+                const uint32_t itg = it + i;
+                const int st = (int)(itg % kI8Stages);
+                const uint32_t ph = (itg / kI8Stages) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u, &g_status_decode))) {
+                    if (lane == 0) producer_drain(full, it + i, kI8Stages);
+                    return;
+                }
+                const int64_t r = row0 + (int64_t)i * ST;
+                if (lane == 0) {
+                    if (n_tok - (int64_t)i * ST >= ST) {
+                        const uint32_t dst = sbase + (uint32_t)st * stage_bytes;
+                        mbar_arrive_expect_tx(&full[st], 2 * kBox + 2 * sbox);
+                        tc::tma_load_4d(dst, &tm_k, 0, (int)r, 0, 0, &full[st]);
+                        tc::tma_load_4d(dst + kBox, &tm_v, 0, (int)r, 0, 0, &full[st]);
+                        tc::tma_load_4d(dst + 2 * kBox, &tm_ks, 0, (int)r, 0, 0, &full[st]);
+                        tc::tma_load_4d(dst + 2 * kBox + sbox, &tm_vs, 0, (int)r, 0, 0, &full[st]);
+                    } else {
+                        mbar_arrive(&full[st]);  // short stage: the consumers load it
+                    }
+                }
+                __syncwarp();
+            }
+        } else {
+            // --------------------------------------------------- consumers
+            const int g = warp % p.Hkv;      // KV head
+            const int j = warp / p.Hkv;      // 16-token subset of every stage
+            const int gq = lane >> 2;
+            const int t = lane & 3;
+            const int64_t pos_b = p.pos ? p.pos[b] : 0;
+            const int32_t *sp = p.slot_pos ? p.slot_pos + (int64_t)b * p.window + t0 : nullptr;
+
+            uint32_t qa[D / 16][2];
+            if (gq < G) {
+                const __nv_bfloat16 *qr = static_cast<const __nv_bfloat16 *>(p.q) +
+                                          ((int64_t)b * p.Hq + (int64_t)g * G + gq) * D;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const __nv_bfloat162 x0 = *reinterpret_cast<const __nv_bfloat162 *>(qr + 16 * kk + 2 * t);
+                    const __nv_bfloat162 x1 = *reinterpret_cast<const __nv_bfloat162 *>(qr + 16 * kk + 8 + 2 * t);
+                    qa[kk][0] = pack2_f16(__bfloat162float(x0.x), __bfloat162float(x0.y));
+                    qa[kk][1] = pack2_f16(__bfloat162float(x1.x), __bfloat162float(x1.y));
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) qa[kk][0] = qa[kk][1] = 0u;
+            }
+            float o[D / 8][4];
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            float m = -INFINITY, l = 0.f;
+            const int tok0 = j * kTokPerWarp;
+            // this warp's converted tiles: K rows then V rows, 272 bytes each
+            unsigned char *kt = smem + tiles + warp * tile_bytes;
+            unsigned char *vt = kt + kTokPerWarp * kI8TileLd * 2;
+            const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt);
+            const int mat = lane >> 3, rr = lane & 7;
+
+            for (int i = 0; i < n_st; ++i) {
+                const uint32_t itg = it + i;
+                const int st = (int)(itg % kI8Stages);
+                const uint32_t ph = (itg / kI8Stages) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph, &g_status_decode))) return;
+                const unsigned char *stg = smem + (size_t)st * stage_bytes;
+                const int64_t base_tok = (int64_t)i * ST + tok0;
+                const int cnt = (int)min((int64_t)ST, n_tok - (int64_t)i * ST);
+                const int64_t r = row0 + (int64_t)i * ST;
+                // codes -> fp16 tiles (16 rows x 8 chunks of 16 codes, K and V)
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const int idx = c4 * 32 + lane;         // 0..255
+                    const int tsr = idx >> 7;               // 0: K, 1: V
+                    const int lt = (idx >> 3) & 15, ch = idx & 7;
+                    uint4 w;
+                    if (cnt == ST) {
+                        const uint32_t R = (uint32_t)(g * ST + tok0 + lt);
+                        w = *reinterpret_cast<const uint4 *>(stg + tsr * kBox + R * 128u + ((ch ^ (R & 7u)) << 4));
+                    } else if (tok0 + lt < cnt) {
+                        w = *reinterpret_cast<const uint4 *>((tsr ? vg : kg) + (r + tok0 + lt) * pi.row_bytes +
+                                                             g * D + ch * 16);
+                    } else {
+                        w = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    uint4 h0, h1;
+                    i8x4_to_f16(w.x, h0.x, h0.y);
+                    i8x4_to_f16(w.y, h0.z, h0.w);
+                    i8x4_to_f16(w.z, h1.x, h1.y);
+                    i8x4_to_f16(w.w, h1.z, h1.w);
+                    unsigned char *dst = (tsr ? vt : kt) + lt * (kI8TileLd * 2) + ch * 32;
+                    *reinterpret_cast<uint4 *>(dst) = h0;
+                    *reinterpret_cast<uint4 *>(dst + 16) = h1;
+                }
+                // the scales of this lane's S columns (tokens 8n + 2t + e of the warp's 16)
+                float ks[2][2], vsc[2][2];
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int lt = 8 * n + 2 * t + e;
+                        if (cnt == ST) {
+                            ks[n][e] = *reinterpret_cast<const float *>(stg + 2 * kBox + (tok0 + lt) * pi.scale_bytes + g * 4);
+                            vsc[n][e] = *reinterpret_cast<const float *>(stg + 2 * kBox + sbox + (tok0 + lt) * pi.scale_bytes + g * 4);
+                        } else if (tok0 + lt < cnt) {
+                            const int64_t row = r + tok0 + lt;
+                            ks[n][e] = *reinterpret_cast<const float *>(kg + row * pi.row_bytes + pi.scale_off + g * 4);
+                            vsc[n][e] = *reinterpret_cast<const float *>(vg + row * pi.row_bytes + pi.scale_off + g * 4);
+                        } else {
+                            ks[n][e] = vsc[n][e] = 0.f;
+                        }
+                    }
+                __syncwarp();
+
+                float sc[2][4];
+#pragma unroll
+                for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+                {
+                    const uint32_t rowa = kt_s + (uint32_t)((8 * (mat >> 1) + rr) * kI8TileLd * 2);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(rowa + (uint32_t)(2 * kk + (mat & 1)) * 16, b0, b1, b2, b3);
+                        mma_16816_f16(sc[0], qa[kk][0], qa[kk][1], b0, b1);
+                        mma_16816_f16(sc[1], qa[kk][0], qa[kk][1], b2, b3);
+                    }
+                }
+                float pv[2][2];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int n = 0; n < 2; ++n) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int lt = 8 * n + 2 * t + e;
+                        const int64_t tok = base_tok + lt;
+                        bool vld = tok < n_tok;
+                        if (vld && sp) {
+                            const int32_t sp_t = sp[tok];
+                            vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window;
+                        }
+                        const float v = vld ? sc[n][e] * ks[n][e] * p.scale_log2 : -INFINITY;
+                        pv[n][e] = v;
+                        mx = fmaxf(mx, v);
+                    }
+                }
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                if (mx > m + 8.f) {
+                    const float alpha = (m == -INFINITY) ? 0.f : ex2f(m - mx);
+                    m = mx;
+                    l *= alpha;
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n) {
+                        o[n][0] *= alpha;
+                        o[n][1] *= alpha;
+                    }
+                }
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                const float p00 = ex2f(pv[0][0] + neg_m), p01 = ex2f(pv[0][1] + neg_m);
+                const float p10 = ex2f(pv[1][0] + neg_m), p11 = ex2f(pv[1][1] + neg_m);
+                l += (p00 + p01) + (p10 + p11);
+                // the V scale of each token folds into its weight
+                const uint32_t a0 = pack2_f16(p00 * vsc[0][0], p01 * vsc[0][1]);
+                const uint32_t a2 = pack2_f16(p10 * vsc[1][0], p11 * vsc[1][1]);
+                {
+                    const uint32_t rowa = vt_s + (uint32_t)((8 * (mat & 1) + rr) * kI8TileLd * 2) +
+                                          (uint32_t)(mat >> 1) * 16;
+#pragma unroll
+                    for (int n = 0; n < D / 8; n += 2) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(rowa + (uint32_t)n * 16, b0, b1, b2, b3);
+                        mma_16816_f16(o[n], a0, a2, b0, b1);
+                        mma_16816_f16(o[n + 1], a0, a2, b2, b3);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
+
+            l += __shfl_xor_sync(0xffffffffu, l, 1);
+            l += __shfl_xor_sync(0xffffffffu, l, 2);
+            const int64_t entry = ((int64_t)b * p.n_split + s) * p.sub + j;
+            if (gq < G) {
+                const int64_t hq = (int64_t)g * G + gq;
+                float *dst = p.ws_o + (entry * p.Hq + hq) * D;
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n)
+                    *reinterpret_cast<float2 *>(dst + 8 * n + 2 * t) = make_float2(o[n][0], o[n][1]);
+                if (t == 0) {
+                    p.ws_ml[(entry * p.Hq + hq) * 2 + 0] = m;
+                    p.ws_ml[(entry * p.Hq + hq) * 2 + 1] = l;
+                }
+            }
+        }
+        it += (uint32_t)n_st;
+    }
+    if (warp == kConsumerWarps && lane == 0) producer_drain(full, it, kI8Stages);
+}
+
+// 8-bit quantisation of K and V rows: one warp per (token, head, tensor);
+// absmax over the head's D values, scale = absmax / 127, code = nearest
+// integer (half to even) of x / scale, all in fp32 with IEEE division.
+template <typename T, int D>
+__global__ void kv_quantize_i8_kernel(const T *k, const T *v, int64_t n, int Hkv, const int64_t *dst_rows,
+                                      unsigned char *kq, unsigned char *vq, int64_t row_bytes) {
+    constexpr int PER = D / 32;
+    const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (wid >= n * Hkv * 2) return;
+    const int tensor = (int)(wid & 1);
+    const int64_t th = wid >> 1, tok = th / Hkv;
+    const int h = (int)(th % Hkv);
+    const T *src = (tensor ? v : k) + (tok * Hkv + h) * D + lane * PER;
+    float x[PER];
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        x[e] = to_f32(src[e]);
+        amax = fmaxf(amax, fabsf(x[e]));
+    }
+    amax = warp_max(amax);
+    const float scale = __fdiv_rn(amax, 127.f);
+    const int64_t row = dst_rows ? dst_rows[tok] : tok;
+    unsigned char *dst = (tensor ? vq : kq) + row * row_bytes;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        int c = scale > 0.f ? __float2int_rn(__fdiv_rn(x[e], scale)) : 0;
+        c = max(-127, min(127, c));
+        packed |= (uint32_t)(c & 0xff) << (8 * e);
+    }
+    if (PER == 4)
+        *reinterpret_cast<uint32_t *>(dst + h * D + lane * 4) = packed;
+    else
+        *reinterpret_cast<uint16_t *>(dst + h * D + lane * 2) = (uint16_t)packed;
+    if (lane == 0) {
+        reinterpret_cast<float *>(dst + (int64_t)Hkv * D)[h] = scale;
+        if (h == 0)  // zero the padding after the scales
+            for (int64_t z = (int64_t)Hkv * (D + 4); z < row_bytes; ++z) dst[z] = 0;
+    }
+}
+
 // Split merge: one CTA of kMergeWarps warps per (sequence, query head).  Warp
 // w takes the chunks of 32 partial entries w, w + kMergeWarps, ...; it forms
 // its own max, its lanes weight 32 entries at once and its weighted sum keeps
@@ -778,6 +1109,102 @@ cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &pl, cudaStream_
         if (a.D == 64) return launch_decode_g<float, 64>(a, pl, st);
     }
     return cudaErrorNotSupported;
+}
+
+// ------------------------------------------------------------- 8-bit cache
+// TMA views of an 8-bit cache: the codes as {128, token, head, 1} bytes (token
+// stride row_bytes, head stride 128), box {128, stage_tokens, Hkv, 1} with the
+// 128-byte swizzle; the scales as {scale_bytes, token, 1, 1} starting at the
+// row's scale offset, box {scale_bytes, stage_tokens, 1, 1}.
+static bool make_i8_maps(CUtensorMap *codes, CUtensorMap *scales, const void *cache, int Hkv, int64_t ST) {
+    const uint64_t rb = (uint64_t)i8_row_bytes(Hkv, 128);
+    const uint64_t rows = std::min<uint64_t>((uint64_t)INT32_MAX, (1ull << 40) / rb);
+    const uint64_t dims[4] = {128, rows, (uint64_t)Hkv, 1};
+    const uint64_t strides[3] = {rb, 128, rb};
+    const uint32_t box[4] = {128, (uint32_t)ST, (uint32_t)Hkv, 1};
+    const uint64_t sdims[4] = {(uint64_t)i8_scale_bytes(Hkv), rows, 1, 1};
+    const uint64_t sstrides[3] = {rb, rb, rb};
+    const uint32_t sbox[4] = {(uint32_t)i8_scale_bytes(Hkv), (uint32_t)ST, 1, 1};
+    const unsigned char *sp = static_cast<const unsigned char *>(cache) + (int64_t)Hkv * 128;
+    return encode_map_4d(codes, cache, true, true, dims, strides, box) &&
+           encode_map_4d(scales, sp, true, false, sdims, sstrides, sbox);
+}
+
+template <int G>
+static cudaError_t launch_decode_i8_g(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t st) {
+    CUtensorMap mk, mks, mv, mvs;
+    if (!make_i8_maps(&mk, &mks, a.k, a.Hkv, pl.stage_tokens) || !make_i8_maps(&mv, &mvs, a.v, a.Hkv, pl.stage_tokens))
+        return cudaErrorNotSupported;
+    DecodeI8Params pi;
+    DecodeKParams &p = pi.k;
+    p.q = a.q; p.k = a.k; p.v = a.v;
+    p.seq_start = a.seq_start; p.seq_len = a.seq_len;
+    p.slot_pos = a.slot_pos; p.pos = a.pos; p.window = a.window;
+    p.B = a.B; p.Hkv = a.Hkv; p.Hq = a.Hq;
+    p.stage_tokens = pl.stage_tokens; p.split = pl.split; p.n_split = pl.n_split;
+    p.sub = pl.sub; p.stages = kI8Stages;
+    p.scale_log2 = a.scale * kLog2e;
+    const size_t entries = (size_t)a.B * pl.n_split * pl.sub * a.Hq;
+    p.ws_o = static_cast<float *>(a.ws);
+    p.ws_ml = p.ws_o + entries * 128;
+    pi.row_bytes = i8_row_bytes(a.Hkv, 128);
+    pi.scale_off = a.Hkv * 128;
+    pi.scale_bytes = (int32_t)i8_scale_bytes(a.Hkv);
+    const uint32_t sbox = (uint32_t)(pl.stage_tokens * pi.scale_bytes);
+    const size_t stage_bytes = 2 * (size_t)kRowsPerStage * 128 + ((2 * sbox + 1023u) & ~1023u);
+    const size_t smem = 1024 + kI8Stages * stage_bytes + (size_t)kConsumerWarps * 2 * kTokPerWarp * kI8TileLd * 2 +
+                        2 * kI8Stages * sizeof(uint64_t);
+    auto kern = decode_i8_kernel<G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t units = (int64_t)a.B * pl.n_split;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, device_sm_count()));
+    kern<<<grid, kDecodeThreads, smem, st>>>(mk, mv, mks, mvs, pi);
+    note_launches(2);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    decode_merge_kernel<__nv_bfloat16, 128><<<(int)((int64_t)a.B * a.Hq), 32 * kMergeWarps, 0, st>>>(
+        p.ws_o, p.ws_ml, a.seq_len, a.window, a.B, a.Hq, pl.split, pl.n_split, pl.sub,
+        static_cast<__nv_bfloat16 *>(a.o), a.lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_i8(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t st) {
+    if (a.B == 0) return cudaSuccess;
+    if (a.D != 128 || a.dtype != kBF16) return cudaErrorNotSupported;
+    switch (a.Hq / a.Hkv) {
+        case 1: return launch_decode_i8_g<1>(a, pl, st);
+        case 2: return launch_decode_i8_g<2>(a, pl, st);
+        case 4: return launch_decode_i8_g<4>(a, pl, st);
+        case 8: return launch_decode_i8_g<8>(a, pl, st);
+    }
+    return cudaErrorNotSupported;
+}
+
+cudaError_t launch_kv_quantize_i8(const void *k, const void *v, int64_t n, int Hkv, int D, int dtype,
+                                  const int64_t *dst_rows, void *kq, void *vq, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    const int64_t warps = n * Hkv * 2;
+    const int grid = (int)((warps + 7) / 8);
+    const int64_t rb = i8_row_bytes(Hkv, D);
+    unsigned char *kb = static_cast<unsigned char *>(kq), *vb = static_cast<unsigned char *>(vq);
+    note_launches(1);
+    if (dtype == kBF16) {
+        if (D == 128)
+            kv_quantize_i8_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), n, Hkv, dst_rows, kb, vb, rb);
+        else
+            kv_quantize_i8_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), n, Hkv, dst_rows, kb, vb, rb);
+    } else {
+        if (D == 128)
+            kv_quantize_i8_kernel<float, 128><<<grid, 256, 0, st>>>(static_cast<const float *>(k),
+                                                                   static_cast<const float *>(v), n, Hkv, dst_rows, kb, vb, rb);
+        else
+            kv_quantize_i8_kernel<float, 64><<<grid, 256, 0, st>>>(static_cast<const float *>(k),
+                                                                  static_cast<const float *>(v), n, Hkv, dst_rows, kb, vb, rb);
+    }
+    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ ring

@@ -128,6 +128,21 @@ int device_sm_count();
 // in bytes) with the 128-byte swizzle; false when the driver rejects it.
 bool encode_bf16_map_4d(::CUtensorMap_st *m, const void *ptr, const uint64_t dims[4],
                         const uint64_t strides_bytes[3], const uint32_t box[4]);
+// The same for bf16 or byte elements, with or without the 128-byte swizzle.
+bool encode_map_4d(::CUtensorMap_st *m, const void *ptr, bool bytes, bool swizzle128, const uint64_t dims[4],
+                   const uint64_t strides_bytes[3], const uint32_t box[4]);
+
+// ------------------------------------------------------------- 8-bit cache
+// One row of an 8-bit K or V cache: Hkv x D int8 codes, then the Hkv fp32
+// scales, padded to a multiple of 16 bytes.
+inline int64_t i8_scale_bytes(int Hkv) { return 16 * ((Hkv * 4 + 15) / 16); }
+inline int64_t i8_row_bytes(int Hkv, int D) { return (int64_t)Hkv * D + i8_scale_bytes(Hkv); }
+// Quantise n rows of K and V ([n, Hkv, D], bf16 or fp32) into 8-bit rows,
+// row dst_rows[i] (or i) of kq / vq.
+cudaError_t launch_kv_quantize_i8(const void *k, const void *v, int64_t n, int Hkv, int D, int dtype,
+                                  const int64_t *dst_rows, void *kq, void *vq, cudaStream_t s);
+// Split-KV decode over 8-bit caches (D = 128); a.k / a.v point at the 8-bit rows.
+cudaError_t launch_decode_i8(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t s);
 
 // Host-side count of kernel launches (reported by yoco_launch_count()).
 void note_launches(int n);

@@ -1,5 +1,5 @@
-// Host-side TMA descriptor encoding for the bf16 kernels (prefill, K/V
-// projection, decode).  The driver's cuTensorMapEncodeTiled is reached
+// Host-side TMA descriptor encoding for the TMA-fed kernels (prefill, K/V
+// projection, decode of bf16 and 8-bit caches).  The driver's cuTensorMapEncodeTiled is reached
 // through the runtime's driver entry-point query, so the library links only
 // the CUDA runtime.
 #include <cuda.h>
@@ -30,8 +30,8 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool encode_bf16_map_4d(CUtensorMap *m, const void *ptr, const uint64_t dims[4],
-                        const uint64_t strides_bytes[3], const uint32_t box[4]) {
+bool encode_map_4d(CUtensorMap *m, const void *ptr, bool bytes, bool swizzle128, const uint64_t dims[4],
+                   const uint64_t strides_bytes[3], const uint32_t box[4]) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t d[4], s[3];
@@ -41,9 +41,15 @@ bool encode_bf16_map_4d(CUtensorMap *m, const void *ptr, const uint64_t dims[4],
         b[i] = box[i];
     }
     for (int i = 0; i < 3; ++i) s[i] = strides_bytes[i];
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), d, s, b, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return enc(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+               const_cast<void *>(ptr), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_bf16_map_4d(CUtensorMap *m, const void *ptr, const uint64_t dims[4],
+                        const uint64_t strides_bytes[3], const uint32_t box[4]) {
+    return encode_map_4d(m, ptr, false, true, dims, strides_bytes, box);
 }
 
 }  // namespace yoco

@@ -105,6 +105,22 @@ def test_gret_arguments_rejected_before_launch():
     assert L.yoco_gret_decode(FAKE, FAKE, FAKE, FAKE, 0, 4.0, FAKE, FAKE, same, None) == yoco.OK
 
 
+def test_i8_cache_arguments_rejected_before_launch():
+    L = yoco.load()
+    c = _cfg()
+    b = ctypes.byref(c)
+    assert L.yoco_kv_i8_row_bytes(b) == 8 * 128 + 32
+    assert L.yoco_kv_i8_row_bytes(ctypes.byref(_cfg(Hq=8, Hkv=1))) == 128 + 16
+    # the 8-bit decode is built for D = 128 and bf16
+    assert L.yoco_cross_decode_i8(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, FAKE, None, FAKE, 1 << 30,
+                                  ctypes.byref(_cfg(D=64)), None) == yoco.ERR_UNSUPPORTED
+    assert L.yoco_cross_decode_i8(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, FAKE, None, None, 0, b, None) == yoco.ERR_WORKSPACE
+    assert L.yoco_cross_decode_i8(FAKE, MISALIGNED, FAKE, FAKE, FAKE, 2, 100, FAKE, None, FAKE, 1 << 30, b,
+                                  None) == yoco.ERR_INVALID
+    assert L.yoco_kv_quantize_i8(FAKE, FAKE, -1, None, FAKE, FAKE, b, None) == yoco.ERR_INVALID
+    assert L.yoco_kv_quantize_i8(FAKE, FAKE, 0, None, FAKE, FAKE, b, None) == yoco.OK
+
+
 def test_workspace_size_monotone_and_positive():
     sizes = [yoco.cross_decode_workspace_size(B, L, 32, 8, 128, torch.bfloat16)
              for B, L in [(1, 1), (1, 4096), (16, 131072), (16, 262144)]]
