@@ -74,6 +74,7 @@ struct ProjParams {
     float w0, w1;
     const int64_t *dst_rows;
     int32_t chunks_per_cta;
+    int32_t groups;  // CTAs per row tile (column groups), adjacent in launch order
 };
 
 YOCO_DEV bool wait1(uint64_t *bar, uint32_t parity) {
@@ -100,8 +101,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *colsum = reinterpret_cast<float *>(sbase + kSmemColsum);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row0 = (int64_t)blockIdx.x * kRowsA;
-    const int chunk0 = blockIdx.y * p.chunks_per_cta;
+    // the column groups of one row tile are adjacent CTAs, so they run at the
+    // same time and their reads of the row tile's x are shared through L2
+    const int64_t row0 = (int64_t)(blockIdx.x / p.groups) * kRowsA;
+    const int chunk0 = (int)(blockIdx.x % p.groups) * p.chunks_per_cta;
     const int n_chunks = min(p.chunks_per_cta, p.m / kBN - chunk0);
     const int kblocks = (p.d + kBK - 1) / kBK;
 
@@ -333,16 +336,17 @@ cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t st) {
     p.base1 = a.base1; p.w0 = a.w0; p.w1 = a.w1; p.dst_rows = a.dst_rows;
     const int64_t mtiles = (a.n + kRowsA - 1) / kRowsA;
     const int nchunks = a.d_out / kBN;
-    const int sms = device_sm_count();
-    int groups = (int)std::min<int64_t>(nchunks, std::max<int64_t>(1, (2 * sms + mtiles - 1) / mtiles));
-    p.chunks_per_cta = (nchunks + groups - 1) / groups;
-    groups = (nchunks + p.chunks_per_cta - 1) / p.chunks_per_cta;
-    if (mtiles > 0x7fffffff) return cudaErrorNotSupported;
+    // four 256-column chunks per CTA: the measured best of 1, 2, 4 and all 8 at
+    // 32K and 256K tokens (the epilogue of one chunk overlaps the next chunk's
+    // MMAs, and the few CTAs of a row tile share its x reads in L2)
+    p.chunks_per_cta = std::min(nchunks, 4);
+    p.groups = (nchunks + p.chunks_per_cta - 1) / p.chunks_per_cta;
+    if (mtiles * p.groups > 0x7fffffff) return cudaErrorNotSupported;
     cudaError_t e = cudaFuncSetAttribute(project_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemAlloc);
     if (e != cudaSuccess) return e;
     note_launches(1);
-    project_tc_kernel<<<dim3((unsigned)mtiles, groups), kThreads, kSmemAlloc, st>>>(mx, mw, p);
+    project_tc_kernel<<<(unsigned)(mtiles * p.groups), kThreads, kSmemAlloc, st>>>(mx, mw, p);
     return cudaGetLastError();
 }
 
