@@ -61,7 +61,7 @@ def parse_args():
     ap.add_argument("--no-early-exit", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer",
-                                       "gret", "gret_decode", "decode_i8_layer"],
+                                       "gret", "gret_decode", "decode_i8_layer", "gret1", "decode_i8"],
                     default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
@@ -89,10 +89,10 @@ TRAFFIC = {
     "prefill": {"bytes": 1829333000 + 238978304,
                 "sources": ["prefill_pair.cu", "schedule.h", "tc.cuh", "common.cuh"],
                 "sha256": "fbaf62f0cc8dcc000c7d83c2a46392dd5909ea2890086fc6737808270a7a158c"},
-    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416114 GB read + 25.135360 MB written
-    "decode": {"bytes": 6416114000 + 25135360,
+    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416178 GB read + 25.136896 MB written
+    "decode": {"bytes": 6416178000 + 25136896,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
-               "sha256": "d7d7875bc339ebb6d1a5591fe98c89c1f392bf916274f892be58e1618f647935"},
+               "sha256": "0640a8bac4919705a237a4213a7148d9feaabe0de312872db81dc6ac67504119"},
 }
 
 
@@ -524,6 +524,7 @@ def run_case(args):
       gret     gated-retention chunkwise prefill B=4, T=65536, 32 heads, D=128
       gret_decode  one gated-retention decode step, batch 16, 32 heads (state 34 MB, L2 flushed)
       decode_i8_layer  one decode layer over the 8-bit cache of the benchmark's decode shape
+      gret1 / decode_i8  the same at batch 1 / at the decode case's shape (for profiling)
     Prints one JSON line with the mean launch time and the work rate."""
     import torch
     import shared_kv_decoder_b200 as yoco
@@ -555,8 +556,9 @@ def run_case(args):
         v = wl.normal((1, T, Hkv, D), 9, bf, dev); o = torch.empty_like(q)
         fn = lambda: yoco.swa_prefill(q, k, v, Wn, o=o)
         work, unit = prefill_flops_per_layer(T, Hq, D, 0, Wn), "TFLOP/s"
-    elif args.case == "decode_i8_layer":
-        lens = wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], DEC["seed"])
+    elif args.case in ("decode_i8_layer", "decode_i8"):
+        lens = (wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], DEC["seed"]) if args.case == "decode_i8_layer"
+                else wl.ragged_lengths(16, 16384, 32768, 9))
         starts = torch.cumsum(torch.cat([torch.zeros(1, dtype=torch.int64), lens[:-1]]), 0)
         rows = int(lens.sum())
         kc = wl.normal((rows, Hkv, D), 4, bf, dev); vc = wl.normal((rows, Hkv, D), 5, bf, dev)
@@ -568,8 +570,8 @@ def run_case(args):
                          dtype=torch.uint8, device=dev)
         fn = lambda: yoco.cross_decode_i8(q, kq, vq, Hkv, ss, sl, int(lens.max()), workspace=ws, o=o)
         work, unit = rows * 2.0 * yoco.kv_i8_row_bytes(Hkv, D), "GB/s"
-    elif args.case == "gret":
-        B, T, H = GRET["B"], GRET["T"], GRET["H"]
+    elif args.case in ("gret", "gret1"):
+        B, T, H = (GRET["B"] if args.case == "gret" else 1), GRET["T"], GRET["H"]
         q = wl.normal((B, T, H, D), 14, bf, dev); k = wl.normal((B, T, H, D), 15, bf, dev)
         v = wl.normal((B, T, H, D), 16, bf, dev); g = wl.normal((B, T, H), 17, torch.float32, dev) + 3.0
         o = torch.empty_like(q)

@@ -114,8 +114,107 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const LinearArgs a) {
     }
 }
 
+// A few rows (decode-step projections): the weight is read once, from HBM,
+// by warps that each own four output columns and every row; x (a few KB per
+// row) comes from L2.  LayerNorm statistics per row first, then each x value
+// is normalised as it is loaded.
+constexpr int kSmallRows = 16, kSmallCols = 4, kSmallWarps = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(32 * kSmallWarps, 1) linear_small_kernel(const LinearArgs a) {
+    constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
+    __shared__ float mu[kSmallRows], rs[kSmallRows];
+    const T *x = static_cast<const T *>(a.x);
+    const T *w = static_cast<const T *>(a.w);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = (int)a.n;
+    for (int r = warp; r < n; r += kSmallWarps) {
+        float mean = 0.f, rstd = 1.f;
+        if (a.apply_ln) {
+            const T *xr = x + (int64_t)r * a.d_in;
+            float s1 = 0.f;
+            for (int c = lane; c < a.d_in; c += 32) s1 += to_f32(xr[c]);
+            mean = warp_sum(s1) / (float)a.d_in;
+            float q = 0.f;
+            for (int c = lane; c < a.d_in; c += 32) {
+                const float t = to_f32(xr[c]) - mean;
+                q = fmaf(t, t, q);
+            }
+            rstd = rsqrtf(warp_sum(q) / (float)a.d_in + a.eps);
+        }
+        if (lane == 0) {
+            mu[r] = a.apply_ln ? mean : 0.f;
+            rs[r] = a.apply_ln ? rstd : 1.f;
+        }
+    }
+    __syncthreads();
+    const int c0 = (blockIdx.x * kSmallWarps + warp) * kSmallCols;
+    if (c0 >= a.d_out) return;
+    float acc[kSmallRows][kSmallCols];
+#pragma unroll
+    for (int r = 0; r < kSmallRows; ++r)
+#pragma unroll
+        for (int j = 0; j < kSmallCols; ++j) acc[r][j] = 0.f;
+    for (int d0 = lane * VEC; d0 < a.d_in; d0 += 32 * VEC) {
+        float wv[kSmallCols][VEC];
+#pragma unroll
+        for (int j = 0; j < kSmallCols; ++j) {
+            const int c = min(c0 + j, a.d_out - 1);
+            const uint4 raw = *reinterpret_cast<const uint4 *>(w + (int64_t)c * a.d_in + d0);
+            const T *e = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+            for (int u = 0; u < VEC; ++u) wv[j][u] = to_f32(e[u]);
+        }
+#pragma unroll
+        for (int r = 0; r < kSmallRows; ++r) {
+            if (r >= n) break;
+            const uint4 raw = *reinterpret_cast<const uint4 *>(x + (int64_t)r * a.d_in + d0);
+            const T *e = reinterpret_cast<const T *>(&raw);
+            const float m = mu[r], sc = rs[r];
+#pragma unroll
+            for (int u = 0; u < VEC; ++u) {
+                const float xv = (to_f32(e[u]) - m) * sc;
+#pragma unroll
+                for (int j = 0; j < kSmallCols; ++j) acc[r][j] = fmaf(xv, wv[j][u], acc[r][j]);
+            }
+        }
+    }
+    const int w1 = a.d_out - a.split_col;
+#pragma unroll
+    for (int r = 0; r < kSmallRows; ++r) {
+        if (r >= n) break;
+#pragma unroll
+        for (int j = 0; j < kSmallCols; ++j) {
+            const float tot = warp_sum(acc[r][j]);
+            const int c = c0 + j;
+            if (lane != ((r * kSmallCols + j) & 31) || c >= a.d_out) continue;
+            const int64_t dr = a.dst_rows ? a.dst_rows[r] : r;
+            float val = tot;
+            if (c < a.split_col) {
+                if (a.base0) val = fmaf(a.w0, to_f32(static_cast<const T *>(a.base0)[(int64_t)r * a.split_col + c]), val);
+                static_cast<T *>(a.out0)[dr * a.split_col + c] = from_f32<T>(val);
+            } else {
+                const int cc = c - a.split_col;
+                if (a.base1) val = fmaf(a.w1, to_f32(static_cast<const T *>(a.base1)[(int64_t)r * w1 + cc]), val);
+                static_cast<T *>(a.out1)[dr * w1 + cc] = from_f32<T>(val);
+            }
+        }
+    }
+}
+
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t st) {
     if (a.n == 0 || a.d_out == 0) return cudaSuccess;
+    const int vec = a.dtype == kBF16 ? 8 : 4;
+    if (a.n <= kSmallRows && a.d_in % vec == 0) {
+        const int cols_per_cta = kSmallWarps * kSmallCols;
+        note_launches(1);
+        const int grid = (a.d_out + cols_per_cta - 1) / cols_per_cta;
+        if (a.dtype == kBF16)
+            linear_small_kernel<__nv_bfloat16><<<grid, 32 * kSmallWarps, 0, st>>>(a);
+        else
+            linear_small_kernel<float><<<grid, 32 * kSmallWarps, 0, st>>>(a);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)((a.d_out + kLinBN - 1) / kLinBN), (unsigned)((a.n + kLinBM - 1) / kLinBM));
     note_launches(1);
     if (a.dtype == kBF16)

@@ -177,7 +177,8 @@ def test_cross_decode_large_values_needle(cuda_lib):
 
 # --------------------------------------------------------- projection + blend
 @pytest.mark.parametrize("dtype", [BF, F32])
-@pytest.mark.parametrize("n,d,Hkv,D", [(1, 256, 2, 64), (77, 512, 2, 128), (300, 256, 8, 64), (4, 1024, 8, 128)])
+@pytest.mark.parametrize("n,d,Hkv,D", [(1, 256, 2, 64), (77, 512, 2, 128), (300, 256, 8, 64), (4, 1024, 8, 128),
+                                       (16, 512, 8, 128), (17, 512, 2, 64)])
 def test_kv_project_blend_matches_oracle(cuda_lib, dtype, n, d, Hkv, D):
     x = wl.normal((n, d), 700 + n, dtype)
     w = wl.normal((2 * Hkv * D, d), 701 + n, dtype, std=d ** -0.5)
