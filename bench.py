@@ -418,33 +418,63 @@ def gret_layer(W, reps):
 def e2e_prefill(W, steps, warmup):
     """Prefill through the public API with HOST buffers: every step copies the
     step's Q (14 layers) and the shared K/V from pinned host memory and reads
-    every layer's output back, inside the timed region."""
+    every layer's output back into its own pinned host buffer, all inside the
+    timed region.  The copies run on their own streams and overlap the
+    kernels as a caller would arrange them: layer l+1's Q goes up while layer
+    l computes, and layer l-1's O comes down (two device buffers each, events
+    for the hand-offs)."""
     import torch
     import shared_kv_decoder_b200 as yoco
+    L = P["layers"]
     hq = [q.cpu().pin_memory() for q in W["qs"]]
     hk = W["kg"].cpu().pin_memory()
     hv = W["vg"].cpu().pin_memory()
-    ho = torch.empty(W["o"].shape, dtype=W["o"].dtype).pin_memory()
-    dq = torch.empty_like(W["qs"][0])
+    ho = [torch.empty(W["o"].shape, dtype=W["o"].dtype).pin_memory() for _ in range(L)]
+    dq = [torch.empty_like(W["qs"][0]) for _ in range(2)]
+    do = [torch.empty_like(W["o"]) for _ in range(2)]
     dk, dv = torch.empty_like(W["kg"]), torch.empty_like(W["vg"])
-    s = torch.cuda.current_stream()
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
     times = []
     for it in range(warmup + steps):
         W["flush"].zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        for l in range(P["layers"]):
-            dq.copy_(hq[l], non_blocking=True)
-            yoco.cross_prefill(dq, dk, dv, o=W["o"])
-            ho.copy_(W["o"], non_blocking=True)
-        e1.record()
-        s.synchronize()
+        e0.record(comp)
+        in_ready = [ev() for _ in range(L)]
+        comp_done = [ev() for _ in range(L)]
+        out_done = [ev() for _ in range(L)]
+        s_in.wait_stream(comp)
+        s_out.wait_stream(comp)
+        with torch.cuda.stream(s_in):
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dq[0].copy_(hq[0], non_blocking=True)
+            in_ready[0].record(s_in)
+        for l in range(L):
+            if l + 1 < L:
+                with torch.cuda.stream(s_in):
+                    if l >= 1:
+                        s_in.wait_event(comp_done[l - 1])     # dq[(l+1)%2] is free again
+                    dq[(l + 1) % 2].copy_(hq[l + 1], non_blocking=True)
+                    in_ready[l + 1].record(s_in)
+            comp.wait_event(in_ready[l])
+            if l >= 2:
+                comp.wait_event(out_done[l - 2])              # do[l%2] has been read out
+            yoco.cross_prefill(dq[l % 2], dk, dv, o=do[l % 2])
+            comp_done[l].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[l])
+                ho[l].copy_(do[l % 2], non_blocking=True)
+                out_done[l].record(s_out)
+        comp.wait_event(out_done[L - 1])
+        comp.wait_stream(s_in)
+        e1.record(comp)
+        torch.cuda.synchronize()
         if it >= warmup:
             times.append(e0.elapsed_time(e1))
     h2d = sum(q.numel() * q.element_size() for q in hq) + 2 * hk.numel() * hk.element_size()
-    d2h = P["layers"] * ho.numel() * ho.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in ho)
     return times, h2d, d2h
 
 
@@ -707,7 +737,7 @@ def main():
         "clocks": clk,
     }
     if not args.no_e2e:
-        times, h2d, d2h = e2e_prefill(W, args.steps, 1)
+        times, h2d, d2h = e2e_prefill(W, args.steps, args.warmup)
         e2e_ms = reduce_max_over_ranks([sum(times)], dev)[0]
         out["e2e"] = {"value": world * len(times) * P["layers"] * f_layer / (e2e_ms * 1e-3) / 1e12,
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
