@@ -161,6 +161,20 @@ yoco_status yoco_cross_decode_static(const void *q, const void *k_cache, const v
                                      int64_t max_len, void *o, float *lse,
                                      const yoco_attn_cfg *cfg, cudaStream_t stream);
 
+/* General attention prefill over a key range that may start before the query
+ * rows: query row i sits at position q_pos0 + i of the key buffer and sees
+ * keys j <= q_pos0 + i, and j > q_pos0 + i - window when window > 0 (0:
+ * causal).  It is the call of a chunk of a longer sequence: the
+ * cross-decoder chunk over the gathered global K/V (window 0, q_pos0 = the
+ * chunk's start), and the self-decoder chunk over its keys preceded by a halo
+ * of the previous window - 1 keys ("You Only Cache Once", paperlayer summary,
+ * Appendix A: the self-decoder only exchanges with neighbouring devices).
+ * Layouts as yoco_cross_prefill; requires 0 <= q_pos0, q_pos0 + Tq <= Tkv,
+ * window >= 0. */
+yoco_status yoco_attention_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t Tq,
+                                   int64_t Tkv, int64_t q_pos0, int32_t window, void *o, float *lse,
+                                   const yoco_attn_cfg *cfg, cudaStream_t stream);
+
 /* Workspace bytes for yoco_cross_decode / yoco_swa_decode (0 on bad args). */
 size_t yoco_cross_decode_workspace_size(int32_t B, int64_t max_len, const yoco_attn_cfg *cfg);
 size_t yoco_swa_decode_workspace_size(int32_t B, int32_t window, const yoco_attn_cfg *cfg);
@@ -258,6 +272,14 @@ double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_at
  * YOCO_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call,
  * YOCO_ERR_CUDA if the stream reports an error, else YOCO_OK. */
 yoco_status yoco_get_device_status(cudaStream_t stream);
+
+/* Test-only, with no counterpart on the pages: launches one kernel that waits,
+ * through the same bounded mbarrier wait as the library's kernels, on a phase
+ * that nothing completes.  The wait gives up after its limit (about 0.1 s),
+ * the status word records it, and the next yoco_get_device_status returns
+ * YOCO_ERR_TIMEOUT; nothing faults and the context stays usable.  Until the
+ * status is read, the library's kernels exit at once (their first check). */
+yoco_status yoco_debug_wait_timeout_probe(cudaStream_t stream);
 
 /* Static description of a status code. */
 const char *yoco_status_string(yoco_status s);

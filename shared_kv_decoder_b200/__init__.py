@@ -9,6 +9,7 @@ importing a function fails loudly when libyoco.so is missing.
 
 Entry points (same names as the C ABI, without the ``yoco_`` prefix):
 kv_project_blend, swa_prefill, swa_decode, cross_prefill, cross_decode,
+attention_prefill,
 gret_prefill, gret_decode, kv_quantize_i8, cross_decode_i8,
 plus linear, workspace sizes, cache_bytes, device_status and the test-only
 debug_tile_schedule.
@@ -22,7 +23,8 @@ __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_p
            "swa_decode", "cross_prefill", "cross_decode", "cross_decode_workspace_size",
            "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg",
            "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE", "gret_prefill", "gret_decode",
-           "kv_i8_row_bytes", "kv_quantize_i8", "cross_decode_i8"]
+           "kv_i8_row_bytes", "kv_quantize_i8", "cross_decode_i8",
+           "attention_prefill"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -70,6 +72,7 @@ def load():
         "yoco_swa_prefill": (st, [vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, cfgp, vp]),
         "yoco_swa_decode": (st, [vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, sz, cfgp, vp]),
         "yoco_cross_prefill": (st, [vp, vp, vp, i32, i64, i64, i64, vp, vp, cfgp, vp]),
+        "yoco_attention_prefill": (st, [vp, vp, vp, i32, i64, i64, i64, i32, vp, vp, cfgp, vp]),
         "yoco_cross_decode": (st, [vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
         "yoco_cross_decode_workspace_size": (sz, [i32, i64, cfgp]),
         "yoco_swa_decode_workspace_size": (sz, [i32, i32, cfgp]),
@@ -82,6 +85,7 @@ def load():
         "yoco_debug_tile_schedule": (st, [i32, cfgp, i32, i64, i64, i64, i32, vp, vp, i64, i32, vp,
                                           i64, ctypes.POINTER(ctypes.c_int64)]),
         "yoco_get_device_status": (st, [vp]),
+        "yoco_debug_wait_timeout_probe": (st, [vp]),
         "yoco_status_string": (ctypes.c_char_p, [st]),
         "yoco_version": (ctypes.c_char_p, []),
         "yoco_launch_count": (ctypes.c_uint64, []),
@@ -349,4 +353,20 @@ def cross_decode_i8(q, k_i8, v_i8, Hkv, seq_start, seq_len, max_len, workspace=N
     _check(L.yoco_cross_decode_i8(_ptr(q), _ptr(k_i8), _ptr(v_i8), _ptr(seq_start), _ptr(seq_len), B,
                                   int(max_len), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(),
                                   ctypes.byref(cfg), _stream()), "yoco_cross_decode_i8")
+    return (o, lse) if want_lse else o
+
+
+def attention_prefill(q, k, v, q_pos0=0, window=0, o=None, want_lse=False, scale=0.0):
+    """Causal (window 0) or windowed attention of q [B, Tq, Hq, D] over keys
+    k, v [B, Tkv, Hkv, D], query row i at key position q_pos0 + i."""
+    L = load()
+    B, Tq, Hq, D = q.shape
+    Tkv, Hkv = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if want_lse else None
+    _dev(q, k, v, o, lse)
+    cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
+    _check(L.yoco_attention_prefill(_ptr(q), _ptr(k), _ptr(v), B, Tq, Tkv, int(q_pos0), int(window), _ptr(o),
+                                    _ptr(lse), ctypes.byref(cfg), _stream()), "yoco_attention_prefill")
     return (o, lse) if want_lse else o

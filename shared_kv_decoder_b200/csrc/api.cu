@@ -172,6 +172,22 @@ yoco_status yoco_cross_prefill(const void *q, const void *k, const void *v, int3
     return run_prefill(a, stream);
 }
 
+yoco_status yoco_attention_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t Tq,
+                                   int64_t Tkv, int64_t q_pos0, int32_t window, void *o, float *lse,
+                                   const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (B < 0 || Tq < 0 || Tkv < 0 || q_pos0 < 0 || q_pos0 + Tq > Tkv || window < 0) return YOCO_ERR_INVALID;
+    if (B == 0 || Tq == 0) return YOCO_OK;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_opt(lse)) return YOCO_ERR_INVALID;
+    PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.Tq = Tq; a.Tkv = Tkv; a.q_pos0 = q_pos0; a.window = window;
+    a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
+    a.scale = eff_scale(cfg);
+    return run_prefill(a, stream);
+}
+
 size_t yoco_cross_decode_workspace_size(int32_t B, int64_t max_len, const yoco_attn_cfg *cfg) {
     if (check_cfg(cfg) != YOCO_OK) return 0;
     DecodePlan pl;
@@ -374,6 +390,10 @@ double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_at
     const double row = 2.0 * cfg->Hkv * cfg->D * (cfg->dtype == YOCO_BF16 ? 2.0 : 4.0);
     const int64_t c = window < N ? window : N;
     return row * ((double)N + (double)L_self * (double)c);
+}
+
+yoco_status yoco_debug_wait_timeout_probe(cudaStream_t stream) {
+    return from_cuda(launch_wait_timeout_probe(stream));
 }
 
 yoco_status yoco_get_device_status(cudaStream_t stream) {

@@ -1207,6 +1207,27 @@ cudaError_t launch_kv_quantize_i8(const void *k, const void *v, int64_t n, int H
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------- test probe
+// Test-only: one thread waits, through the kernels' own bounded wait, on an
+// mbarrier phase that nothing completes.  The wait gives up after its limit,
+// records the timeout in the status word and returns: nothing faults, nothing
+// hangs, and the context stays usable.
+__global__ void wait_timeout_probe_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &g_status_decode);  // phase 0 never completes
+}
+
+cudaError_t launch_wait_timeout_probe(cudaStream_t st) {
+    note_launches(1);
+    wait_timeout_probe_kernel<<<1, 32, 0, st>>>();
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ ring
 template <typename T>
 __global__ void ring_write_kernel(const T *k_new, const T *v_new, const int64_t *pos, int32_t window,

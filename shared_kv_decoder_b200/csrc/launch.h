@@ -116,6 +116,9 @@ cudaError_t launch_gret_prefill(const GretArgs &a, cudaStream_t s);
 // One recurrent decode step (bf16 or fp32).
 cudaError_t launch_gret_decode(const GretArgs &a, cudaStream_t s);
 
+// Test-only: a kernel whose bounded wait is never satisfied (see decode.cu).
+cudaError_t launch_wait_timeout_probe(cudaStream_t s);
+
 // Device status words of the translation units that hold bounded waits.
 unsigned int read_and_clear_status_decode();
 unsigned int read_and_clear_status_prefill_tc();
