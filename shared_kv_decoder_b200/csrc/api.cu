@@ -399,7 +399,8 @@ yoco_status yoco_debug_wait_timeout_probe(cudaStream_t stream) {
 yoco_status yoco_get_device_status(cudaStream_t stream) {
     const cudaError_t e = cudaStreamSynchronize(stream);
     const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc() |
-                           read_and_clear_status_prefill_pair() | read_and_clear_status_project_tc();
+                           read_and_clear_status_prefill_pair() | read_and_clear_status_project_tc() |
+                           read_and_clear_status_gret_tc();
     if (s) return YOCO_ERR_TIMEOUT;
     return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;
 }

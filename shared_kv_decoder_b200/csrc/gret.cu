@@ -387,6 +387,10 @@ static cudaError_t launch_gret_prefill_d(const GretArgs &a, cudaStream_t st) {
 cudaError_t launch_gret_prefill(const GretArgs &a, cudaStream_t st) {
     if (a.dtype != kBF16) return cudaErrorNotSupported;
     if (a.B == 0 || a.T == 0 || a.H == 0) return cudaSuccess;
+    // D = 128: the tcgen05 kernel (gret_tc.cu); otherwise the mma.sync kernel here
+    const cudaError_t e = launch_gret_prefill_tc(a, st);
+    if (e != cudaErrorNotSupported) return e;
+    cudaGetLastError();
     if ((int64_t)a.B * a.H > INT32_MAX) return cudaErrorNotSupported;
     if (a.D == 128) return launch_gret_prefill_d<128>(a, st);
     if (a.D == 64) return launch_gret_prefill_d<64>(a, st);

@@ -115,6 +115,8 @@ struct GretArgs {
 cudaError_t launch_gret_prefill(const GretArgs &a, cudaStream_t s);
 // One recurrent decode step (bf16 or fp32).
 cudaError_t launch_gret_decode(const GretArgs &a, cudaStream_t s);
+// Chunkwise prefill on the tensor cores (bf16, D = 128; cudaErrorNotSupported otherwise).
+cudaError_t launch_gret_prefill_tc(const GretArgs &a, cudaStream_t s);
 
 // Test-only: a kernel whose bounded wait is never satisfied (see decode.cu).
 cudaError_t launch_wait_timeout_probe(cudaStream_t s);
@@ -123,6 +125,7 @@ cudaError_t launch_wait_timeout_probe(cudaStream_t s);
 unsigned int read_and_clear_status_decode();
 unsigned int read_and_clear_status_prefill_tc();
 unsigned int read_and_clear_status_prefill_pair();
+unsigned int read_and_clear_status_gret_tc();
 unsigned int read_and_clear_status_project_tc();
 
 int device_sm_count();
