@@ -588,15 +588,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 // codes of one token, then its Hkv fp32 scales (padded to 16 bytes); a value
 // is code * scale.  A stage arrives as two 16 KB TMA boxes of codes ([head]
 // [token] rows of 128 bytes, 128-byte swizzle) and two small boxes of the
-// stage's scales -- half the bytes of the bf16 cache.  Each consumer warp
-// turns its head's 16 token rows of K and V into fp16 tiles in its own
-// shared-memory slice (exact: an int8 code fits fp16's mantissa; the byte is
-// placed under the exponent of 1024 and 1152 subtracted), then runs the same
-// mma.sync inner products in fp16.  The K scale multiplies the column of S
-// it belongs to, the V scale folds into P before P V, so the tensor cores see
-// integer-valued operands only.
-constexpr int kI8Stages = 4;
-constexpr int kI8TileLd = 136;  // fp16 elements per row of a warp's converted tile (272 bytes)
+// stage's scales -- half the bytes of the bf16 cache.
+//
+// The tensor-core tiles read the codes where the TMA put them, with the
+// stage's 16 tokens of a head as the 16 MMA rows and the group's query heads
+// as the 8 columns (transposed against the bf16 kernel, so no row of an MMA
+// is padding when G < 16):
+//  * S^T = K q^T is an integer MMA (m16n8k32, s8 x s8 -> s32) straight on the
+//    K codes.  q is held as 15-bit fixed point per head (q ~ s_q * x, |x| <=
+//    16256) split into two int8 parts x = 128 hi + lo, so S^T = 128 K hi^T +
+//    K lo^T exactly in int32; the fixed-point step of q is 2^-14 of its
+//    largest element, far below bf16's own rounding of q.  The K scale, s_q
+//    and the softmax scale multiply the int32 result.
+//  * O^T += V^T P^T is an fp16 MMA: V's codes are turned into fp16 in
+//    registers (exact: the byte goes under the exponent of 1024 and 1152 is
+//    subtracted), P^T comes from the S^T accumulators by one register
+//    transpose (movmatrix) and carries each token's V scale.
+// A stage that a sequence's end cuts short is copied by each warp from
+// global memory into its own rows of the stage, zero-filled past the end.
+constexpr int kI8Stages = 6;
 
 struct DecodeI8Params {
     DecodeKParams k;
@@ -605,26 +615,46 @@ struct DecodeI8Params {
     int32_t scale_bytes; // padded bytes of the scales per row
 };
 
-YOCO_DEV void mma_16816_f16(float *c, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+YOCO_DEV void mma_16816_f16_t(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                              uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+YOCO_DEV void mma_16832_s8(int *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+YOCO_DEV uint32_t movmatrix_t(uint32_t x) {
+    uint32_t r;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    return r;
 }
 YOCO_DEV uint32_t pack2_f16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-// four int8 codes -> two fp16x2 words, exactly
-YOCO_DEV void i8x4_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+// Four int8 codes of a transposed ldmatrix word (bytes: token 2t at dims 2g,
+// 2g+1, then token 2t+1 at dims 2g, 2g+1) -> fp16x2 (token 2t, token 2t+1) of
+// dim 2g (even) and of dim 2g+1 (odd), exactly.
+YOCO_DEV void i8t_to_f16(uint32_t w, uint32_t &even, uint32_t &odd) {
     const uint32_t u = w ^ 0x80808080u;  // code + 128, as unsigned bytes
     const uint32_t bias = 0x64806480u;   // fp16 1152 = 1024 + 128, twice
-    uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);
-    uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(bias));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(bias));
+    const uint32_t a = __byte_perm(u, 0x64646464u, 0x4240);
+    const uint32_t b = __byte_perm(u, 0x64646464u, 0x4341);
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(even) : "r"(a), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(odd) : "r"(b), "r"(bias));
+}
+// four int8 values -> one word (byte i = v[i])
+YOCO_DEV uint32_t pack_s8x4(float v0, float v1, float v2, float v3) {
+    return ((uint32_t)(int)v0 & 0xffu) | (((uint32_t)(int)v1 & 0xffu) << 8) | (((uint32_t)(int)v2 & 0xffu) << 16) |
+           (((uint32_t)(int)v3 & 0xffu) << 24);
 }
 
 template <int G>
@@ -632,6 +662,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_i8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const DecodeI8Params pi) {
+    static_assert(G >= 1 && G <= 8, "the query heads of a group are the 8 columns of an MMA");
     if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
     constexpr int D = 128;
     constexpr uint32_t kBox = kRowsPerStage * 128;  // one code box: 128 rows of 128 bytes
@@ -643,9 +674,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     unsigned char *smem = smem_raw + (sbase - raw);
-    const uint32_t tiles = (uint32_t)kI8Stages * stage_bytes;           // converted fp16 tiles
-    const uint32_t tile_bytes = 2u * kTokPerWarp * kI8TileLd * 2u;      // K and V of one warp
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + tiles + kConsumerWarps * tile_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)kI8Stages * stage_bytes);
     uint64_t *empty = full + kI8Stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -699,170 +728,216 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             }
         } else {
             // --------------------------------------------------- consumers
-            const int g = warp % p.Hkv;      // KV head
+            const int kvh = warp % p.Hkv;    // KV head
             const int j = warp / p.Hkv;      // 16-token subset of every stage
-            const int gq = lane >> 2;
+            const int gq = lane >> 2;        // S^T row (token) / P^T column (query head)
             const int t = lane & 3;
             const int64_t pos_b = p.pos ? p.pos[b] : 0;
             const int32_t *sp = p.slot_pos ? p.slot_pos + (int64_t)b * p.window + t0 : nullptr;
-
-            uint32_t qa[D / 16][2];
-            if (gq < G) {
-                const __nv_bfloat16 *qr = static_cast<const __nv_bfloat16 *>(p.q) +
-                                          ((int64_t)b * p.Hq + (int64_t)g * G + gq) * D;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const __nv_bfloat162 x0 = *reinterpret_cast<const __nv_bfloat162 *>(qr + 16 * kk + 2 * t);
-                    const __nv_bfloat162 x1 = *reinterpret_cast<const __nv_bfloat162 *>(qr + 16 * kk + 8 + 2 * t);
-                    qa[kk][0] = pack2_f16(__bfloat162float(x0.x), __bfloat162float(x0.y));
-                    qa[kk][1] = pack2_f16(__bfloat162float(x1.x), __bfloat162float(x1.y));
-                }
-            } else {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) qa[kk][0] = qa[kk][1] = 0u;
-            }
-            float o[D / 8][4];
-#pragma unroll
-            for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-            float m = -INFINITY, l = 0.f;
             const int tok0 = j * kTokPerWarp;
-            // this warp's converted tiles: K rows then V rows, 272 bytes each
-            unsigned char *kt = smem + tiles + warp * tile_bytes;
-            unsigned char *vt = kt + kTokPerWarp * kI8TileLd * 2;
-            const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt);
-            const int mat = lane >> 3, rr = lane & 7;
+
+            // q of head gq as two int8 parts (B operand: dims 32kb + 4t.. and
+            // 32kb + 16 + 4t..), and per head column 2t + e the factor s_q *
+            // softmax scale * log2(e)
+            uint32_t qh[4][2], ql[4][2];
+            float qs[2];
+            {
+                float x[4][2][4];
+                float amax = 0.f;
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        if (gq < G) {
+                            const __nv_bfloat16 *qr = static_cast<const __nv_bfloat16 *>(p.q) +
+                                                      ((int64_t)b * p.Hq + (int64_t)kvh * G + gq) * D +
+                                                      32 * kb + 16 * hf + 4 * t;
+                            const uint2 w = *reinterpret_cast<const uint2 *>(qr);
+                            x[kb][hf][0] = __uint_as_float(w.x << 16);
+                            x[kb][hf][1] = __uint_as_float(w.x & 0xffff0000u);
+                            x[kb][hf][2] = __uint_as_float(w.y << 16);
+                            x[kb][hf][3] = __uint_as_float(w.y & 0xffff0000u);
+                        } else {
+                            x[kb][hf][0] = x[kb][hf][1] = x[kb][hf][2] = x[kb][hf][3] = 0.f;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(x[kb][hf][i]));
+                    }
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                const float inv = amax > 0.f ? 16256.f / amax : 0.f;
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float hi[4], lo[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float xi = fminf(fmaxf(rintf(x[kb][hf][i] * inv), -16256.f), 16256.f);
+                            hi[i] = rintf(xi * (1.f / 128.f));
+                            lo[i] = xi - 128.f * hi[i];
+                        }
+                        qh[kb][hf] = pack_s8x4(hi[0], hi[1], hi[2], hi[3]);
+                        ql[kb][hf] = pack_s8x4(lo[0], lo[1], lo[2], lo[3]);
+                    }
+                const float sq = amax * (1.f / 16256.f);
+                qs[0] = __shfl_sync(0xffffffffu, sq, 8 * t) * p.scale_log2;
+                qs[1] = __shfl_sync(0xffffffffu, sq, 8 * t + 4) * p.scale_log2;
+            }
+            float oe[4][4], oo[4][4];  // O^T of dims 32c + 2g (+16) and 32c + 2g + 1 (+16)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) oe[c][i] = oo[c][i] = 0.f;
+            float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+            // ldmatrix rows of this lane: K (matrix mi: tokens 8(mi&1).., 16-byte
+            // chunk mi>>1 of a 32-dim block), V (tokens 8(mi>>1).., chunk mi&1)
+            const int mi = lane >> 3, rr = lane & 7;
+            const uint32_t Rk = (uint32_t)(kvh * ST + tok0 + 8 * (mi & 1) + rr);
+            const uint32_t Rv = (uint32_t)(kvh * ST + tok0 + 8 * (mi >> 1) + rr);
 
             for (int i = 0; i < n_st; ++i) {
                 const uint32_t itg = it + i;
                 const int st = (int)(itg % kI8Stages);
                 const uint32_t ph = (itg / kI8Stages) & 1u;
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph, &g_status_decode))) return;
-                const unsigned char *stg = smem + (size_t)st * stage_bytes;
+                unsigned char *stg = smem + (size_t)st * stage_bytes;
+                const uint32_t stg_s = sbase + (uint32_t)st * stage_bytes;
                 const int64_t base_tok = (int64_t)i * ST + tok0;
                 const int cnt = (int)min((int64_t)ST, n_tok - (int64_t)i * ST);
                 const int64_t r = row0 + (int64_t)i * ST;
-                // codes -> fp16 tiles (16 rows x 8 chunks of 16 codes, K and V)
+                float ks[2], vs[2];  // scales of tokens gq and gq + 8
+                if (cnt == ST) {
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    const int idx = c4 * 32 + lane;         // 0..255
-                    const int tsr = idx >> 7;               // 0: K, 1: V
-                    const int lt = (idx >> 3) & 15, ch = idx & 7;
-                    uint4 w;
-                    if (cnt == ST) {
-                        const uint32_t R = (uint32_t)(g * ST + tok0 + lt);
-                        w = *reinterpret_cast<const uint4 *>(stg + tsr * kBox + R * 128u + ((ch ^ (R & 7u)) << 4));
-                    } else if (tok0 + lt < cnt) {
-                        w = *reinterpret_cast<const uint4 *>((tsr ? vg : kg) + (r + tok0 + lt) * pi.row_bytes +
-                                                             g * D + ch * 16);
-                    } else {
-                        w = make_uint4(0u, 0u, 0u, 0u);
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int lt = tok0 + gq + 8 * h8;
+                        ks[h8] = *reinterpret_cast<const float *>(stg + 2 * kBox + lt * pi.scale_bytes + kvh * 4);
+                        vs[h8] = *reinterpret_cast<const float *>(stg + 2 * kBox + sbox + lt * pi.scale_bytes + kvh * 4);
                     }
-                    uint4 h0, h1;
-                    i8x4_to_f16(w.x, h0.x, h0.y);
-                    i8x4_to_f16(w.y, h0.z, h0.w);
-                    i8x4_to_f16(w.z, h1.x, h1.y);
-                    i8x4_to_f16(w.w, h1.z, h1.w);
-                    unsigned char *dst = (tsr ? vt : kt) + lt * (kI8TileLd * 2) + ch * 32;
-                    *reinterpret_cast<uint4 *>(dst) = h0;
-                    *reinterpret_cast<uint4 *>(dst + 16) = h1;
-                }
-                // the scales of this lane's S columns (tokens 8n + 2t + e of the warp's 16)
-                float ks[2][2], vsc[2][2];
+                } else {
+                    // short stage: this warp's 16 rows of K and V codes into
+                    // their swizzled places, zeros past the end
 #pragma unroll
-                for (int n = 0; n < 2; ++n)
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        const int idx = c8 * 32 + lane;  // 0..255
+                        const int tsr = idx >> 7, lt = (idx >> 3) & 15, ch = idx & 7;
+                        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                        if (tok0 + lt < cnt)
+                            w = *reinterpret_cast<const uint4 *>((tsr ? vg : kg) + (r + tok0 + lt) * pi.row_bytes +
+                                                                 kvh * D + ch * 16);
+                        const uint32_t R = (uint32_t)(kvh * ST + tok0 + lt);
+                        *reinterpret_cast<uint4 *>(stg + tsr * kBox + R * 128u + ((ch ^ (R & 7u)) << 4)) = w;
+                    }
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int lt = 8 * n + 2 * t + e;
-                        if (cnt == ST) {
-                            ks[n][e] = *reinterpret_cast<const float *>(stg + 2 * kBox + (tok0 + lt) * pi.scale_bytes + g * 4);
-                            vsc[n][e] = *reinterpret_cast<const float *>(stg + 2 * kBox + sbox + (tok0 + lt) * pi.scale_bytes + g * 4);
-                        } else if (tok0 + lt < cnt) {
-                            const int64_t row = r + tok0 + lt;
-                            ks[n][e] = *reinterpret_cast<const float *>(kg + row * pi.row_bytes + pi.scale_off + g * 4);
-                            vsc[n][e] = *reinterpret_cast<const float *>(vg + row * pi.row_bytes + pi.scale_off + g * 4);
-                        } else {
-                            ks[n][e] = vsc[n][e] = 0.f;
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int lt = tok0 + gq + 8 * h8;
+                        ks[h8] = vs[h8] = 0.f;
+                        if (lt < cnt) {
+                            const int64_t row = r + lt;
+                            ks[h8] = *reinterpret_cast<const float *>(kg + row * pi.row_bytes + pi.scale_off + kvh * 4);
+                            vs[h8] = *reinterpret_cast<const float *>(vg + row * pi.row_bytes + pi.scale_off + kvh * 4);
                         }
                     }
-                __syncwarp();
-
-                float sc[2][4];
-#pragma unroll
-                for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-                {
-                    const uint32_t rowa = kt_s + (uint32_t)((8 * (mat >> 1) + rr) * kI8TileLd * 2);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(rowa + (uint32_t)(2 * kk + (mat & 1)) * 16, b0, b1, b2, b3);
-                        mma_16816_f16(sc[0], qa[kk][0], qa[kk][1], b0, b1);
-                        mma_16816_f16(sc[1], qa[kk][0], qa[kk][1], b2, b3);
-                    }
+                    fence_proxy_async_smem();  // before the next TMA write into this stage
+                    __syncwarp();
                 }
-                float pv[2][2];
-                float mx = -INFINITY;
+                uint32_t kr[4][4], vr[4][4];
 #pragma unroll
-                for (int n = 0; n < 2; ++n) {
+                for (int kb = 0; kb < 4; ++kb)
+                    ldsm_x4(stg_s + Rk * 128u + ((((uint32_t)(2 * kb + (mi >> 1))) ^ (Rk & 7u)) << 4), kr[kb][0],
+                            kr[kb][1], kr[kb][2], kr[kb][3]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    ldsm_x4_t(stg_s + kBox + Rv * 128u + ((((uint32_t)(2 * c + (mi & 1))) ^ (Rv & 7u)) << 4), vr[c][0],
+                              vr[c][1], vr[c][2], vr[c][3]);
+                // S^T (16 tokens x 8 heads) in int32: hi and lo parts of q
+                int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    mma_16832_s8(ah, kr[kb][0], kr[kb][1], kr[kb][2], kr[kb][3], qh[kb][0], qh[kb][1]);
+                    mma_16832_s8(al, kr[kb][0], kr[kb][1], kr[kb][2], kr[kb][3], ql[kb][0], ql[kb][1]);
+                }
+                // scores (log2 domain): element 2 h8 + e = token gq + 8 h8, head 2t + e
+                float sv[4];
+#pragma unroll
+                for (int h8 = 0; h8 < 2; ++h8) {
+                    const int64_t tok = base_tok + gq + 8 * h8;
+                    bool vld = tok < n_tok;
+                    if (vld && sp) {
+                        const int32_t sp_t = sp[tok];
+                        vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window;
+                    }
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int lt = 8 * n + 2 * t + e;
-                        const int64_t tok = base_tok + lt;
-                        bool vld = tok < n_tok;
-                        if (vld && sp) {
-                            const int32_t sp_t = sp[tok];
-                            vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window;
+                        const float acc = (float)(128 * ah[2 * h8 + e] + al[2 * h8 + e]);
+                        sv[2 * h8 + e] = vld ? acc * ks[h8] * qs[e] : -INFINITY;
+                    }
+                }
+                float pr[4];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float mx = fmaxf(sv[e], sv[2 + e]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    if (mx > m[e] + 8.f) {
+                        const float alpha = (m[e] == -INFINITY) ? 0.f : ex2f(m[e] - mx);
+                        m[e] = mx;
+                        l[e] *= alpha;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            oe[c][e] *= alpha;
+                            oe[c][2 + e] *= alpha;
+                            oo[c][e] *= alpha;
+                            oo[c][2 + e] *= alpha;
                         }
-                        const float v = vld ? sc[n][e] * ks[n][e] * p.scale_log2 : -INFINITY;
-                        pv[n][e] = v;
-                        mx = fmaxf(mx, v);
                     }
+                    const float neg_m = (m[e] == -INFINITY) ? 0.f : -m[e];
+                    pr[e] = ex2f(sv[e] + neg_m);
+                    pr[2 + e] = ex2f(sv[2 + e] + neg_m);
+                    l[e] += pr[e] + pr[2 + e];
                 }
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                if (mx > m + 8.f) {
-                    const float alpha = (m == -INFINITY) ? 0.f : ex2f(m - mx);
-                    m = mx;
-                    l *= alpha;
+                // P^T with each token's V scale: transpose the [token][head]
+                // fp16 pairs into the B fragments (head gq; tokens 2t, 2t+1 and
+                // 2t+8, 2t+9)
+                const uint32_t b0 = movmatrix_t(pack2_f16(pr[0] * vs[0], pr[1] * vs[0]));
+                const uint32_t b1 = movmatrix_t(pack2_f16(pr[2] * vs[1], pr[3] * vs[1]));
 #pragma unroll
-                    for (int n = 0; n < D / 8; ++n) {
-                        o[n][0] *= alpha;
-                        o[n][1] *= alpha;
-                    }
-                }
-                const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                const float p00 = ex2f(pv[0][0] + neg_m), p01 = ex2f(pv[0][1] + neg_m);
-                const float p10 = ex2f(pv[1][0] + neg_m), p11 = ex2f(pv[1][1] + neg_m);
-                l += (p00 + p01) + (p10 + p11);
-                // the V scale of each token folds into its weight
-                const uint32_t a0 = pack2_f16(p00 * vsc[0][0], p01 * vsc[0][1]);
-                const uint32_t a2 = pack2_f16(p10 * vsc[1][0], p11 * vsc[1][1]);
-                {
-                    const uint32_t rowa = vt_s + (uint32_t)((8 * (mat & 1) + rr) * kI8TileLd * 2) +
-                                          (uint32_t)(mat >> 1) * 16;
-#pragma unroll
-                    for (int n = 0; n < D / 8; n += 2) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4_t(rowa + (uint32_t)n * 16, b0, b1, b2, b3);
-                        mma_16816_f16(o[n], a0, a2, b0, b1);
-                        mma_16816_f16(o[n + 1], a0, a2, b2, b3);
-                    }
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
+                    i8t_to_f16(vr[c][0], e0, o0);
+                    i8t_to_f16(vr[c][1], e1, o1);
+                    i8t_to_f16(vr[c][2], e2, o2);
+                    i8t_to_f16(vr[c][3], e3, o3);
+                    mma_16816_f16_t(oe[c], e0, e1, e2, e3, b0, b1);
+                    mma_16816_f16_t(oo[c], o0, o1, o2, o3, b0, b1);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
 
-            l += __shfl_xor_sync(0xffffffffu, l, 1);
-            l += __shfl_xor_sync(0xffffffffu, l, 2);
-            const int64_t entry = ((int64_t)b * p.n_split + s) * p.sub + j;
-            if (gq < G) {
-                const int64_t hq = (int64_t)g * G + gq;
-                float *dst = p.ws_o + (entry * p.Hq + hq) * D;
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n)
-                    *reinterpret_cast<float2 *>(dst + 8 * n + 2 * t) = make_float2(o[n][0], o[n][1]);
-                if (t == 0) {
-                    p.ws_ml[(entry * p.Hq + hq) * 2 + 0] = m;
-                    p.ws_ml[(entry * p.Hq + hq) * 2 + 1] = l;
+            for (int e = 0; e < 2; ++e) {
+                l[e] += __shfl_xor_sync(0xffffffffu, l[e], 4);
+                l[e] += __shfl_xor_sync(0xffffffffu, l[e], 8);
+                l[e] += __shfl_xor_sync(0xffffffffu, l[e], 16);
+            }
+            const int64_t entry = ((int64_t)b * p.n_split + s) * p.sub + j;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int hh = 2 * t + e;
+                if (hh < G) {
+                    const int64_t hq = (int64_t)kvh * G + hh;
+                    float *dst = p.ws_o + (entry * p.Hq + hq) * D;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        *reinterpret_cast<float2 *>(dst + 32 * c + 2 * gq) = make_float2(oe[c][e], oo[c][e]);
+                        *reinterpret_cast<float2 *>(dst + 32 * c + 16 + 2 * gq) = make_float2(oe[c][2 + e], oo[c][2 + e]);
+                    }
+                    if (gq == 0) {
+                        p.ws_ml[(entry * p.Hq + hq) * 2 + 0] = m[e];
+                        p.ws_ml[(entry * p.Hq + hq) * 2 + 1] = l[e];
+                    }
                 }
             }
         }
@@ -1152,8 +1227,7 @@ static cudaError_t launch_decode_i8_g(const DecodeArgs &a, const DecodePlan &pl,
     pi.scale_bytes = (int32_t)i8_scale_bytes(a.Hkv);
     const uint32_t sbox = (uint32_t)(pl.stage_tokens * pi.scale_bytes);
     const size_t stage_bytes = 2 * (size_t)kRowsPerStage * 128 + ((2 * sbox + 1023u) & ~1023u);
-    const size_t smem = 1024 + kI8Stages * stage_bytes + (size_t)kConsumerWarps * 2 * kTokPerWarp * kI8TileLd * 2 +
-                        2 * kI8Stages * sizeof(uint64_t);
+    const size_t smem = 1024 + kI8Stages * stage_bytes + 2 * kI8Stages * sizeof(uint64_t);
     auto kern = decode_i8_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
