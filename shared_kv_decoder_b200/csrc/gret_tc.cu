@@ -6,27 +6,47 @@
 // in chunks of 128 tokens.  With c_r the running sum of log gamma over the
 // chunk's rows 0..r (base-2 units here):
 //   o_r   = sum_{u<=r} 2^{c_r - c_u} scale (q_r . k_u) v_u   +  2^{c_r} q_r S_prev
-//   S_new = 2^{c_last} S_prev + sum_u 2^{c_last - c_u} scale k_u^T v_u
+//   S_new = 2^{c_last} S_prev + sum_u K_w[u]^T v_u,  K_w[u] = 2^{c_last - c_u} scale k_u
 // Every exponent is <= 0.
 //
+// The decayed scores reuse K_w: Q K_w^T = scale 2^{c_last - c_u} (q_r . k_u),
+// so 2^{c_r - c_last} (Q K_w^T)[r][u] is the decayed score, one multiply per
+// element instead of an exponential.  That needs 2^{c_last - c_u} and
+// 2^{c_r - c_last} to stay normal fp32 / bf16 numbers: it is used when the
+// chunk's total decay 2^{c_last} is at least 2^-60; a chunk that decays more
+// takes the scores from Q K^T with one exponential per element.
+//
 // One CTA per (batch, head) walks the chunks in order.  TMEM (512 columns):
-//   A/P [0,128)   Q K^T of the chunk, then the decayed, masked P (bf16, first 64)
+//   A/P [0,128)   the scores of the chunk, then the decayed, masked P (bf16, first 64)
 //   O   [128,256) P V
 //   X   [256,384) Q S_prev
 //   S   [384,512) the fp32 state (row d = lane d)
-// Shared memory: the chunk's Q, K and V tiles (TMA, 128-byte swizzle), K_w
-// (K scaled by scale * 2^{c_last - c_u}), and S_prev split into bf16 high and
-// low parts laid out like a V tile (about 16 mantissa bits for the cross term).
-// Warp roles (320 threads):
-//   warps 0-3  output: P from A (decay mask), then o = O + 2^{c_r} X -> global
-//   warps 4-7  state: K_w, S *= 2^{c_last} in TMEM, and after the update the
-//              high / low split of S into shared memory for the next chunk
-//   warp 8     TMA: lane 0 Q tiles, lane 1 K tiles, lane 2 V tiles
-//   warp 9     MMA issuer: A = Q K^T; X = Q S_hi + Q S_lo; O = P V;
-//              S += K_w^T V (A operand MN-major from the K_w tile)
-// Every mbarrier wait is bounded; a wait that gives up sets the status word,
-// and all roles fall through to the common exit, which waits for issued
-// copies and MMAs before freeing TMEM.
+// Shared memory (224 KB): Q, K, V (two buffers), K_w, S_prev rounded to bf16
+// and laid out like a V tile for the cross term, and the bf16 output tile
+// that the TMA stores.  The cross term's rounding is of the same order as the
+// bf16 rounding of P in P V and of K_w in the update (an fp64 emulation of
+// the chunk loop: rel-L2 2.7e-3 against 2.3e-3 with a two-part bf16 split of
+// S, both dominated by those other roundings); the state itself stays fp32
+// in TMEM.  The running log-decay sums live in registers and are exchanged
+// by warp shuffles.
+// Warp roles (352 threads):
+//   warps 0-3  output: P, then o = O + 2^{c_r} X into the output tile (warp 0
+//              lane 0 issues its TMA store)
+//   warps 4-7  state: K_w; one pass over S that writes S_prev in bf16 for this
+//              chunk's cross term and leaves 2^{c_last} S_prev in TMEM for the
+//              update
+//   warp 8     TMA: lane 0 Q tiles, lane 1 K tiles, lane 2 V tiles; each also
+//              asks L2 for its next tile
+//   warp 9     output MMAs: scores = Q K_w^T (or Q K^T); X = Q S_prev; O = P V
+//   warp 10    state MMA: S += K_w^T V (A operand MN-major from the K_w tile)
+// The recurrence S -> S' runs on warps 4-7 and 10 alone, so it never queues
+// behind the output side's MMAs; the two sides meet at K_w (read by both
+// MMAs), at the bf16 copy of S_prev (the cross term of a chunk must have read
+// it before the next chunk's copy overwrites it) and at the K and V tiles.
+// Every warp reads the gate logits of the next chunk while it works on this
+// one.  Every mbarrier wait is bounded; a wait that gives up sets the status
+// word, and all roles fall through to the common exit, which waits for
+// issued copies and MMAs before freeing TMEM.
 #include <cuda.h>
 
 #include <algorithm>
@@ -44,41 +64,50 @@ namespace {
 
 constexpr int kC = 128;            // chunk length
 constexpr int kD = 128;            // head dim
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr uint32_t kBlk = 128 * 128;      // one [128 rows x 128 bytes] swizzled block
 constexpr uint32_t kTile = 2 * kBlk;      // a [128, 128] bf16 tile (two 64-column blocks)
+constexpr float kFoldMinLog2 = -60.f;     // smallest chunk decay (log2) that folds into K_w
 
 enum Smem : uint32_t {
     kQ = 0,
     kK = kQ + kTile,
-    kV = kK + kTile,
-    kKw = kV + kTile,
-    kShi = kKw + kTile,
-    kSlo = kShi + kTile,
-    kC2 = kSlo + kTile,                   // 8 warps x 128 floats of running sums
-    kBars = kC2 + 8 * kC * 4,
+    kV0 = kK + kTile,
+    kV1 = kV0 + kTile,
+    kKw = kV1 + kTile,
+    kSb = kKw + kTile,                    // S_prev in bf16
+    kOt = kSb + kTile,                    // output tile
+    kBars = kOt + kTile,
     kBytes = kBars + 256,
     kAlloc = kBytes + 1024,
 };
+static_assert(kAlloc <= 227 * 1024, "shared memory per block");
 
 enum Bar {
-    kQFull = 0, kKFull, kVFull,
-    kQEmpty, kKEmpty, kVEmpty,
-    kAFull,       // Q K^T done
+    kQFull = 0,
+    kKFull,
+    kVFull,       // two: V buffers
+    kQEmpty = kVFull + 2,  // the scores and the cross term done (Q and the bf16 S_prev free)
+    kKEmpty,      // the scores done (commit) and K_w written (arrive): 2 arrivals
+    kVEmpty,      // two: P V and the state update done (2 commits each)
+    kAFull = kVEmpty + 2,  // the scores done (K_w free for the next chunk's)
     kPFull,       // P written (128 arrivals)
-    kOFull,       // P V (and the cross term before it) done
-    kOFree,       // O and X read out (128 arrivals)
-    kSScaled,     // K_w written and S decayed (128 arrivals)
+    kOFull,       // the cross term and P V done
+    kOFree,       // O and X read out of TMEM (128 arrivals)
+    kOStaged,     // the output tile written (128 arrivals)
+    kOtFree,      // the previous output tile's store has read it
+    kSReady,      // K_w, the bf16 S_prev and the decayed S in place (128 arrivals)
     kSUpdated,    // S += K_w^T V done
-    kSplit,       // S_hi / S_lo ready for the next chunk (128 arrivals)
-    kDrain,
+    kDrainO, kDrainS,
     kNumBars
 };
+// after the barriers: TMEM address, abort flag, fold flag of the chunk (two)
+constexpr uint32_t kMisc = kBars + kNumBars * 8;
+static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
 
 struct GretTcParams {
     const float *g;
     float *state;
-    __nv_bfloat16 *o;
     int32_t B, H;
     int64_t T;
     float lg_scale;   // log2(e) / tau
@@ -107,22 +136,28 @@ YOCO_DEV uint32_t sw_off(int row, int col) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     gret_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const GretTcParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const GretTcParams p) {
     if (*(volatile unsigned int *)&g_status_gret_tc) return;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *sb = smem_raw + (base - raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sb + kBars);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sb + kBars + kNumBars * 8);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sb + kBars + kNumBars * 8 + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sb + kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sb + kMisc + 4);
+    volatile int *fold_flag = reinterpret_cast<volatile int *>(sb + kMisc + 8);  // [2]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int NC = p.n_chunks;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNumBars; ++i)
-            mbar_init(&bars[i], (i == kPFull || i == kOFree || i == kSScaled || i == kSplit) ? 128 : 1);
+        for (int i = 0; i < kNumBars; ++i) {
+            int cnt = 1;
+            if (i == kPFull || i == kOFree || i == kOStaged || i == kSReady) cnt = 128;
+            if (i == kKEmpty || i == kVEmpty || i == kVEmpty + 1) cnt = 2;
+            mbar_init(&bars[i], cnt);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -138,88 +173,108 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------ TMA producer
+        // lane 0: Q, lane 1: K, lane 2: V (two buffers)
         if (lane < 3) {
             const CUtensorMap *map = lane == 0 ? &tm_q : lane == 1 ? &tm_k : &tm_v;
-            const uint32_t dst = base + (lane == 0 ? kQ : lane == 1 ? kK : kV);
-            uint64_t *full = &bars[kQFull + lane], *empty = &bars[kQEmpty + lane];
+            const int nb = lane == 2 ? 2 : 1;
+            const uint32_t dst0 = base + (lane == 0 ? kQ : lane == 1 ? kK : kV0);
+            uint64_t *full = &bars[lane == 0 ? kQFull : lane == 1 ? kKFull : kVFull];
+            uint64_t *empty = &bars[lane == 0 ? kQEmpty : lane == 1 ? kKEmpty : kVEmpty];
             int j = 0;
             for (; j < NC && !*abort_flag; ++j) {
-                if (j > 0 && !wait1(empty, (j - 1) & 1)) { *abort_flag = 1; break; }
-                mbar_arrive_expect_tx(full, kC * kD * 2);
+                const int bi = j % nb, use = j / nb;
+                if (use > 0 && !wait1(&empty[bi], (use - 1) & 1)) { *abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&full[bi], kC * kD * 2);
                 for (int kb = 0; kb < 2; ++kb)
-                    tc::tma_load_4d(dst + kb * kBlk, map, kb * 64, h, j * kC, b, full);
+                    tc::tma_load_4d(dst0 + bi * kTile + kb * kBlk, map, kb * 64, h, j * kC, b, &full[bi]);
+                if (j + nb < NC)
+                    for (int kb = 0; kb < 2; ++kb) tc::tma_prefetch_4d(map, kb * 64, h, (j + nb) * kC, b);
             }
-            if (j > 0) wait1(full, (j - 1) & 1);  // the last copy has landed before exit
+            // the last copy into each buffer has landed before exit
+            for (int jj = j - 1; jj >= 0 && jj >= j - nb; --jj) wait1(&full[jj % nb], (jj / nb) & 1);
         }
     } else if (warp == 9) {
-        // ---------------------------------------------------------- MMA issue
+        // ------------------------------------------------ output-side MMAs
         if (lane == 0) {
             constexpr uint32_t idQK = tc::idesc_bf16(128, 128, false, false);
             constexpr uint32_t idMNB = tc::idesc_bf16(128, 128, false, true);
-            constexpr uint32_t idUpd = tc::idesc_bf16(128, 128, true, true);
             bool ok = true;
             for (int j = 0; ok && j < NC; ++j) {
-                const uint32_t ph = j & 1;
-                // A = Q K^T
-                if (!wait1(&bars[kQFull], ph) || !wait1(&bars[kKFull], ph) || *abort_flag) { ok = false; break; }
+                const uint32_t ph = j & 1, bi = j & 1, ph2 = (j >> 1) & 1;
+                const uint32_t v_s = base + kV0 + bi * kTile;
+                // scores: Q K_w^T when the chunk folds, else Q K^T
+                if (!wait1(&bars[kSReady], ph) || !wait1(&bars[kQFull], ph) || !wait1(&bars[kKFull], ph) ||
+                    *abort_flag) {
+                    ok = false;
+                    break;
+                }
                 tc::fence_after_sync();
+                const uint32_t kb_s = base + (fold_flag[bi] ? kKw : kK);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
                     tc::mma_bf16_ss(tA, tc::smem_desc_sw128(base + kQ + off, 16, 1024),
-                                    tc::smem_desc_sw128(base + kK + off, 16, 1024), idQK, kk > 0 ? 1u : 0u);
+                                    tc::smem_desc_sw128(kb_s + off, 16, 1024), idQK, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(&bars[kAFull]);
-                // X = Q S_prev (high and low parts); X and O must have been read out
-                if (!wait1(&bars[kSplit], ph)) { ok = false; break; }
+                tc::mma_commit(&bars[kKEmpty]);
+                // X = Q S_prev; X and O must have been read out
                 if (j > 0 && !wait1(&bars[kOFree], (j - 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t sm = base + (part == 0 ? kShi : kSlo);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
-                        tc::mma_bf16_ss(tX, tc::smem_desc_sw128(base + kQ + off, 16, 1024),
-                                        tc::smem_desc_sw128(sm + kk * 2048, kBlk, 1024), idMNB,
-                                        (part > 0 || kk > 0) ? 1u : 0u);
-                    }
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tX, tc::smem_desc_sw128(base + kQ + off, 16, 1024),
+                                    tc::smem_desc_sw128(base + kSb + kk * 2048, kBlk, 1024), idMNB, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(&bars[kQEmpty]);
                 // O = P V
-                if (!wait1(&bars[kPFull], ph) || !wait1(&bars[kVFull], ph)) { ok = false; break; }
+                if (!wait1(&bars[kPFull], ph) || !wait1(&bars[kVFull + bi], ph2)) { ok = false; break; }
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    tc::mma_bf16_ts(tO, tA + kk * 8, tc::smem_desc_sw128(base + kV + kk * 2048, kBlk, 1024), idMNB,
+                    tc::mma_bf16_ts(tO, tA + kk * 8, tc::smem_desc_sw128(v_s + kk * 2048, kBlk, 1024), idMNB,
                                     kk > 0 ? 1u : 0u);
                 tc::mma_commit(&bars[kOFull]);
-                // S += K_w^T V
-                if (!wait1(&bars[kSScaled], ph)) { ok = false; break; }
+                tc::mma_commit(&bars[kVEmpty + bi]);
+            }
+            if (!ok) *abort_flag = 1;
+            tc::mma_commit(&bars[kDrainO]);
+            wait1(&bars[kDrainO], 0);
+        }
+    } else if (warp == 10) {
+        // -------------------------------------------------------- state MMA
+        if (lane == 0) {
+            constexpr uint32_t idUpd = tc::idesc_bf16(128, 128, true, true);
+            bool ok = true;
+            for (int j = 0; ok && j < NC; ++j) {
+                const uint32_t ph = j & 1, bi = j & 1, ph2 = (j >> 1) & 1;
+                if (!wait1(&bars[kSReady], ph) || *abort_flag) { ok = false; break; }
+                mbar_arrive(&bars[kKEmpty]);  // the state warps are done reading K
+                if (!wait1(&bars[kVFull + bi], ph2)) { ok = false; break; }
                 tc::fence_after_sync();
-                tc::mma_commit(&bars[kKEmpty]);   // the state warps are done reading K
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
                     tc::mma_bf16_ss(tS, tc::smem_desc_sw128(base + kKw + kk * 2048, kBlk, 1024),
-                                    tc::smem_desc_sw128(base + kV + kk * 2048, kBlk, 1024), idUpd, 1u);
-                tc::mma_commit(&bars[kVEmpty]);
+                                    tc::smem_desc_sw128(base + kV0 + bi * kTile + kk * 2048, kBlk, 1024), idUpd, 1u);
+                tc::mma_commit(&bars[kVEmpty + bi]);
                 tc::mma_commit(&bars[kSUpdated]);
             }
             if (!ok) *abort_flag = 1;
-            tc::mma_commit(&bars[kDrain]);
-            wait1(&bars[kDrain], 0);
+            tc::mma_commit(&bars[kDrainS]);
+            wait1(&bars[kDrainS], 0);
         }
     } else {
         // ------------------------------------------- output and state warps
         const bool state_role = warp >= 4;
         const int r = (warp & 3) * 32 + lane;                 // TMEM lane = chunk row / state row
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        float *c2w = reinterpret_cast<float *>(sb + kC2) + warp * kC;
         const float *gb = p.g + (int64_t)b * p.T * p.H + h;
+        const bool store_thread = warp == 0 && lane == 0;   // issues the output tile's TMA store
         bool ok = true;
 
         if (state_role) {
-            // initial state: TMEM rows, then the high / low split for chunk 0
+            // initial state into TMEM rows
             const float *s0 = p.state ? p.state + ((int64_t)b * p.H + h) * kD * kD + (int64_t)r * kD : nullptr;
 #pragma unroll
             for (int c = 0; c < kD; c += 32) {
@@ -231,19 +286,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::wait_st();
         }
 
+        // gate logits of the chunk after the current one (lane l: rows 4l..4l+3)
+        float gn[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t t = 4 * lane + i;
+            gn[i] = t < p.T ? gb[t * p.H] : 0.f;
+        }
+
         for (int j = 0; ok && j < NC; ++j) {
             const uint32_t ph = j & 1;
             const int64_t t0 = (int64_t)j * kC;
-            // running base-2 log-decay sums of the chunk, computed by every warp
-            // for itself (lane l: rows 4l..4l+3; padded rows decay by 1)
-            __syncwarp();  // the previous chunk's reads of this warp's copy are done
+            // running base-2 log-decay sums of the chunk in registers: lane l
+            // holds c_u for u = 4l..4l+3 (padded rows decay by 1)
+            float x[4];
             {
-                float x[4], run = 0.f;
+                float run = 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int64_t t = t0 + 4 * lane + i;
-                    run += t < p.T ? log2_decay(gb[t * p.H], p.lg_scale) : 0.f;
+                    run += t0 + 4 * lane + i < p.T ? log2_decay(gn[i], p.lg_scale) : 0.f;
                     x[i] = run;
+                }
+                if (j + 1 < NC) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int64_t t = t0 + kC + 4 * lane + i;
+                        gn[i] = t < p.T ? gb[t * p.H] : 0.f;
+                    }
                 }
                 float incl = run;
 #pragma unroll
@@ -253,89 +322,104 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float excl = incl - run;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) c2w[4 * lane + i] = excl + x[i];
-                __syncwarp();
+                for (int i = 0; i < 4; ++i) x[i] += excl;
             }
-            const float c_r = c2w[r], c_last = c2w[kC - 1];
+            // c_r of this thread's row r (held by lane r / 4) and c_last
+            float c_r;
+            {
+                const int src = r >> 2;
+                const float y0 = __shfl_sync(0xffffffffu, x[0], src), y1 = __shfl_sync(0xffffffffu, x[1], src);
+                const float y2 = __shfl_sync(0xffffffffu, x[2], src), y3 = __shfl_sync(0xffffffffu, x[3], src);
+                const int sel = r & 3;
+                c_r = sel == 0 ? y0 : sel == 1 ? y1 : sel == 2 ? y2 : y3;
+            }
+            const float c_last = __shfl_sync(0xffffffffu, x[3], 31);
+            const bool fold = c_last >= kFoldMinLog2;   // the same in every warp
 
             if (!state_role) {
-                // ---- P = scale * 2^{c_r - c_u} A for u <= r, else 0
+                // ---- P: 2^{c_r - c_last} (Q K_w^T) or scale 2^{c_r - c_u} (Q K^T),
+                // for u <= r, else 0
                 if (!waitw(&bars[kAFull], ph)) { ok = false; break; }
                 tc::fence_after_sync();
+                const float fr = tc::ex2(c_r - c_last);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float a[64];
-                    tc::tmem_ld32(tA + lane_off + half * 64, a);
-                    tc::tmem_ld32(tA + lane_off + half * 64 + 32, a + 32);
+                for (int qt = 0; qt < 4; ++qt) {
+                    float a[32];
+                    tc::tmem_ld32(tA + lane_off + qt * 32, a);
                     tc::wait_ld();
-                    uint32_t pk[32];
+                    uint32_t pk[16];
+                    if (fold) {
 #pragma unroll
-                    for (int u2 = 0; u2 < 64; u2 += 2) {
-                        const int u = half * 64 + u2;
-                        const float w0 = u <= r ? p.scale * tc::ex2(c_r - c2w[u]) : 0.f;
-                        const float w1 = u + 1 <= r ? p.scale * tc::ex2(c_r - c2w[u + 1]) : 0.f;
-                        pk[u2 / 2] = tc::pack_bf16x2(a[u2] * w0, a[u2 + 1] * w1);
+                        for (int u2 = 0; u2 < 32; u2 += 2) {
+                            const int u = qt * 32 + u2;
+                            pk[u2 / 2] = tc::pack_bf16x2(u <= r ? a[u2] * fr : 0.f, u + 1 <= r ? a[u2 + 1] * fr : 0.f);
+                        }
+                    } else {
+#pragma unroll
+                        for (int u2 = 0; u2 < 32; u2 += 2) {
+                            const int u = qt * 32 + u2;
+                            const float cu0 = __shfl_sync(0xffffffffu, x[u & 3], u >> 2);
+                            const float cu1 = __shfl_sync(0xffffffffu, x[(u + 1) & 3], (u + 1) >> 2);
+                            const float w0 = u <= r ? p.scale * tc::ex2(c_r - cu0) : 0.f;
+                            const float w1 = u + 1 <= r ? p.scale * tc::ex2(c_r - cu1) : 0.f;
+                            pk[u2 / 2] = tc::pack_bf16x2(a[u2] * w0, a[u2 + 1] * w1);
+                        }
                     }
-                    tc::tmem_st32u(tA + lane_off + half * 32, pk);
+                    tc::tmem_st16u(tA + lane_off + qt * 16, pk);
                 }
                 tc::wait_st();
                 tc::fence_before_sync();
                 mbar_arrive(&bars[kPFull]);
-                // ---- o = O + 2^{c_r} X
+                // ---- o = O + 2^{c_r} X into the output tile, then its TMA store
                 if (!waitw(&bars[kOFull], ph)) { ok = false; break; }
                 tc::fence_after_sync();
+                // the previous chunk's store has read the tile
+                if (j > 0) {
+                    if (store_thread) {
+                        tc::bulk_wait_read_all();
+                        mbar_arrive(&bars[kOtFree]);
+                    }
+                    if (!waitw(&bars[kOtFree], (j - 1) & 1)) { ok = false; break; }
+                }
                 const float f = tc::ex2(c_r);
-                __nv_bfloat16 *dst = p.o + (((int64_t)b * p.T + t0 + r) * p.H + h) * kD;
 #pragma unroll
                 for (int c = 0; c < kD; c += 32) {
                     float ov[32], xv[32];
                     tc::tmem_ld32(tO + lane_off + c, ov);
                     tc::tmem_ld32(tX + lane_off + c, xv);
                     tc::wait_ld();
-                    if (t0 + r < p.T) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 w;
-                            w.x = tc::pack_bf16x2(fmaf(f, xv[e], ov[e]), fmaf(f, xv[e + 1], ov[e + 1]));
-                            w.y = tc::pack_bf16x2(fmaf(f, xv[e + 2], ov[e + 2]), fmaf(f, xv[e + 3], ov[e + 3]));
-                            w.z = tc::pack_bf16x2(fmaf(f, xv[e + 4], ov[e + 4]), fmaf(f, xv[e + 5], ov[e + 5]));
-                            w.w = tc::pack_bf16x2(fmaf(f, xv[e + 6], ov[e + 6]), fmaf(f, xv[e + 7], ov[e + 7]));
-                            *reinterpret_cast<uint4 *>(dst + c + e) = w;
-                        }
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 w;
+                        w.x = tc::pack_bf16x2(fmaf(f, xv[e], ov[e]), fmaf(f, xv[e + 1], ov[e + 1]));
+                        w.y = tc::pack_bf16x2(fmaf(f, xv[e + 2], ov[e + 2]), fmaf(f, xv[e + 3], ov[e + 3]));
+                        w.z = tc::pack_bf16x2(fmaf(f, xv[e + 4], ov[e + 4]), fmaf(f, xv[e + 5], ov[e + 5]));
+                        w.w = tc::pack_bf16x2(fmaf(f, xv[e + 6], ov[e + 6]), fmaf(f, xv[e + 7], ov[e + 7]));
+                        *reinterpret_cast<uint4 *>(sb + kOt + sw_off(r, c + e)) = w;
                     }
                 }
                 tc::fence_before_sync();
                 mbar_arrive(&bars[kOFree]);
-            } else {
-                // ---- the state's split for this chunk's cross term (chunk 0: the
-                // initial state; later: done at the end of the previous chunk)
-                if (j == 0) {
-#pragma unroll
-                    for (int c = 0; c < kD; c += 32) {
-                        float v[32];
-                        tc::tmem_ld32(tS + lane_off + c, v);
-                        tc::wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 hi, lo;
-                            uint32_t *hp = &hi.x, *lp = &lo.x;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float x0 = v[e + 2 * q], x1 = v[e + 2 * q + 1];
-                                hp[q] = tc::pack_bf16x2(x0, x1);
-                                lp[q] = tc::pack_bf16x2(x0 - __uint_as_float(hp[q] << 16),
-                                                        x1 - __uint_as_float(hp[q] & 0xffff0000u));
-                            }
-                            *reinterpret_cast<uint4 *>(sb + kShi + sw_off(r, c + e)) = hi;
-                            *reinterpret_cast<uint4 *>(sb + kSlo + sw_off(r, c + e)) = lo;
+                fence_proxy_async_smem();
+                mbar_arrive(&bars[kOStaged]);
+                if (warp == 0) {
+                    bool sok = true;
+                    if (lane == 0) {
+                        sok = wait1(&bars[kOStaged], ph);
+                        if (sok) {
+                            // rows past the sequence's end are not written
+                            tc::tma_store_4d(&tm_o, base + kOt, 0, h, (int)t0, b);
+                            tc::tma_store_4d(&tm_o, base + kOt + kBlk, 64, h, (int)t0, b);
+                            tc::bulk_commit_group();
                         }
                     }
-                    fence_proxy_async_smem();
-                    tc::fence_before_sync();
-                    mbar_arrive(&bars[kSplit]);
+                    if (!__shfl_sync(0xffffffffu, (int)sok, 0)) { ok = false; break; }
                 }
-                // ---- K_w = K * scale * 2^{c_last - c_u} (row u = r of the K tile)
+            } else {
+                // ---- K_w = K * scale * 2^{c_last - c_u} (row u = r of the K tile);
+                // the previous update and the previous scores have read K_w
                 if (!waitw(&bars[kKFull], ph)) { ok = false; break; }
+                if (j > 0 && !waitw(&bars[kAFull], (j - 1) & 1)) { ok = false; break; }
                 {
                     const float w = p.scale * tc::ex2(c_last - c_r);
 #pragma unroll
@@ -352,7 +436,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint4 *>(sb + kKw + off) = out;
                     }
                 }
-                // ---- S *= 2^{c_last} in TMEM (row d = r)
+                // ---- one pass over S_prev: its bf16 copy for this chunk's cross
+                // term (once the previous cross term has read the last copy),
+                // and S *= 2^{c_last} in TMEM
+                if (j > 0 && !waitw(&bars[kQEmpty], (j - 1) & 1)) { ok = false; break; }
                 {
                     const float f = tc::ex2(c_last);
                     tc::fence_after_sync();
@@ -362,54 +449,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::tmem_ld32(tS + lane_off + c, v);
                         tc::wait_ld();
 #pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            uint4 hv;
+                            hv.x = tc::pack_bf16x2(v[e], v[e + 1]);
+                            hv.y = tc::pack_bf16x2(v[e + 2], v[e + 3]);
+                            hv.z = tc::pack_bf16x2(v[e + 4], v[e + 5]);
+                            hv.w = tc::pack_bf16x2(v[e + 6], v[e + 7]);
+                            *reinterpret_cast<uint4 *>(sb + kSb + sw_off(r, c + e)) = hv;
+                        }
+#pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] *= f;
                         tc::tmem_st32(tS + lane_off + c, v);
                     }
                     tc::wait_st();
                 }
+                if (warp == 4 && lane == 0) fold_flag[j & 1] = fold ? 1 : 0;
                 fence_proxy_async_smem();
                 tc::fence_before_sync();
-                mbar_arrive(&bars[kSScaled]);
-                // ---- after the update: split S for the next chunk (and, at the
-                // end, write the final state)
+                mbar_arrive(&bars[kSReady]);
                 if (!waitw(&bars[kSUpdated], ph)) { ok = false; break; }
-                tc::fence_after_sync();
-                float *sfin = (j == NC - 1 && p.state) ? p.state + ((int64_t)b * p.H + h) * kD * kD + (int64_t)r * kD
-                                                      : nullptr;
-#pragma unroll
-                for (int c = 0; c < kD; c += 32) {
-                    float v[32];
-                    tc::tmem_ld32(tS + lane_off + c, v);
-                    tc::wait_ld();
-                    if (sfin) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4 *>(sfin + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                    }
-                    if (j + 1 < NC) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 hi, lo;
-                            uint32_t *hp = &hi.x, *lp = &lo.x;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float x0 = v[e + 2 * q], x1 = v[e + 2 * q + 1];
-                                hp[q] = tc::pack_bf16x2(x0, x1);
-                                lp[q] = tc::pack_bf16x2(x0 - __uint_as_float(hp[q] << 16),
-                                                        x1 - __uint_as_float(hp[q] & 0xffff0000u));
-                            }
-                            *reinterpret_cast<uint4 *>(sb + kShi + sw_off(r, c + e)) = hi;
-                            *reinterpret_cast<uint4 *>(sb + kSlo + sw_off(r, c + e)) = lo;
-                        }
-                    }
-                }
-                if (j + 1 < NC) {
-                    fence_proxy_async_smem();
-                    tc::fence_before_sync();
-                    mbar_arrive(&bars[kSplit]);
-                }
             }
         }
+        if (ok && state_role && p.state) {
+            // the final state
+            tc::fence_after_sync();
+            float *sfin = p.state + ((int64_t)b * p.H + h) * kD * kD + (int64_t)r * kD;
+#pragma unroll
+            for (int c = 0; c < kD; c += 32) {
+                float v[32];
+                tc::tmem_ld32(tS + lane_off + c, v);
+                tc::wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(sfin + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            }
+        }
+        if (store_thread) tc::bulk_wait_all();  // the output tiles are written before exit
         if (!ok) *abort_flag = 1;
         tc::wait_st();
     }
@@ -439,13 +514,13 @@ cudaError_t launch_gret_prefill_tc(const GretArgs &a, cudaStream_t st) {
     if (a.dtype != kBF16 || a.D != kD) return cudaErrorNotSupported;
     if (a.B == 0 || a.T == 0 || a.H == 0) return cudaSuccess;
     if ((int64_t)a.B * a.H > INT32_MAX || a.T > INT32_MAX) return cudaErrorNotSupported;
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H))
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mo, a.o, a.B, a.T, a.H))
         return cudaErrorNotSupported;
     GretTcParams p;
     p.g = a.g;
     p.state = a.state;
-    p.o = static_cast<__nv_bfloat16 *>(a.o);
     p.B = a.B; p.H = a.H; p.T = a.T;
     p.lg_scale = kLog2e / a.tau;
     p.scale = a.scale;
@@ -453,7 +528,7 @@ cudaError_t launch_gret_prefill_tc(const GretArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(gret_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAlloc);
     if (e != cudaSuccess) return e;
     note_launches(1);
-    gret_tc_kernel<<<a.B * a.H, kThreads, kAlloc, st>>>(mq, mk, mv, p);
+    gret_tc_kernel<<<a.B * a.H, kThreads, kAlloc, st>>>(mq, mk, mv, mo, p);
     return cudaGetLastError();
 }
 
