@@ -121,7 +121,7 @@ def reduce_max_over_ranks(values, device=None):
     return [float(v) for v in t.tolist()]
 
 
-def gret_flops(B, T, H, D, chunk=64):
+def gret_flops(B, T, H, D, chunk=128):
     """Tensor FLOPs of chunkwise gated retention at the kernel's chunk size: per
     chunk and head, Q K^T and P V over the chunk's causal pairs (counted in
     full, C x C) plus the cross term Q S and the state update K^T V (D x D
@@ -408,11 +408,14 @@ def gret_layer(W, reps):
 
     t_pre = timed(lambda: yoco.gret_prefill(q, k, v, g, tau, state=st, o=o))
     t_dec = timed(lambda: yoco.gret_decode(qd, kd, vd, gd, tau, sd, o=od))
+    pre_bytes = 4.0 * B * T * H * D * 2 + B * T * H * 4.0 + 2.0 * B * H * D * D * 4
     return {"prefill_ms": t_pre, "prefill_tflops": gret_flops(B, T, H, D) / (t_pre * 1e-3) / 1e12,
             "prefill_tokens_per_s": B * T / (t_pre * 1e-3),
+            "prefill_hbm_gbs": pre_bytes / (t_pre * 1e-3) / 1e9,
             "decode_ms": t_dec, "decode_gbs": Bd * H * D * D * 8.0 / (t_dec * 1e-3) / 1e9,
             "shape": f"prefill B={B} T={T} H={H} D={D}; decode batch {Bd}",
-            "flops": "chunkwise at chunk 64: QK^T and PV over C x C, Q S and K^T V over D x D, per chunk and head"}
+            "flops": "chunkwise at chunk 128: QK^T and PV over C x C, Q S and K^T V over D x D, per chunk and head",
+            "bytes": "q, k, v read and o written once (bf16), gate logits, state in and out (fp32)"}
 
 
 def e2e_prefill(W, steps, warmup):
