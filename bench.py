@@ -85,14 +85,14 @@ def load_peaks():
 # and the report carries null instead.
 _CSRC = "shared_kv_decoder_b200/csrc/"
 TRAFFIC = {
-    # attn_prefill_pair_kernel<128>, T=32768: 1.829333 GB read + 238.978304 MB written
-    "prefill": {"bytes": 1829333000 + 238978304,
+    # attn_prefill_pair_kernel<128>, T=32768: 1.814138 GB read + 239.481088 MB written
+    "prefill": {"bytes": 1814138000 + 239481088,
                 "sources": ["prefill_pair.cu", "schedule.h", "tc.cuh", "common.cuh"],
-                "sha256": "fbaf62f0cc8dcc000c7d83c2a46392dd5909ea2890086fc6737808270a7a158c"},
-    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416178 GB read + 25.136896 MB written
-    "decode": {"bytes": 6416178000 + 25136896,
+                "sha256": "e8e2369b9f4bb812ccec27be99b70749aad412c78e133211f37f9a70b6043836"},
+    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416142 GB read + 25.513984 MB written
+    "decode": {"bytes": 6416142000 + 25513984,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
-               "sha256": "0640a8bac4919705a237a4213a7148d9feaabe0de312872db81dc6ac67504119"},
+               "sha256": "e6b1985a87f4803a25388c0999f795684d1fb490cbdd04333d8a8d63e6e3014d"},
 }
 
 
@@ -416,6 +416,38 @@ def gret_layer(W, reps):
             "shape": f"prefill B={B} T={T} H={H} D={D}; decode batch {Bd}",
             "flops": "chunkwise at chunk 128: QK^T and PV over C x C, Q S and K^T V over D x D, per chunk and head",
             "bytes": "q, k, v read and o written once (bf16), gate logits, state in and out (fp32)"}
+
+
+def decode_i8_step(W, reps):
+    """The benchmark's decode step over the 8-bit copy of the same shared cache,
+    measured beside the step (it is not part of it): quantise the bf16 cache
+    once, then 16 cross layers of yoco_cross_decode_i8 for the 16 sequences.
+    Device ms per decode step (mean over reps, L2 rewritten before each)."""
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    Hkv, D = DEC["Hkv"], DEC["D"]
+    kq, vq = yoco.kv_quantize_i8(W["kc"], W["vc"])
+
+    def step():
+        for l in range(DEC["layers"]):
+            yoco.cross_decode_i8(W["qd"][l], kq, vq, Hkv, W["seq_start"], W["seq_len"], W["max_len"],
+                                 workspace=W["ws"], o=W["od"])
+
+    ts = []
+    for i in range(reps + 1):
+        W["flush"].zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(); step(); e1.record()
+        torch.cuda.synchronize()
+        if i > 0:
+            ts.append(e0.elapsed_time(e1))
+    ms = statistics.mean(ts)
+    layer_bytes = 2.0 * W["rows"] * yoco.kv_i8_row_bytes(Hkv, D)
+    del kq, vq
+    return {"ms_per_decode_step": ms, "tokens_per_s": DEC["B"] / (ms * 1e-3),
+            "hbm_gbs": layer_bytes * DEC["layers"] / (ms * 1e-3) / 1e9, "bytes_per_layer": layer_bytes,
+            "note": "same sequences and queries as the decode block; int8 codes with one fp32 scale per "
+                    "(token, KV head): half the cache bytes"}
 
 
 def e2e_prefill(W, steps, warmup):
@@ -747,6 +779,7 @@ def main():
     if not args.no_early_exit:
         out["early_exit"] = early_exit(W, 3)
         out["gret"] = gret_layer(W, 3)
+        out["decode_i8"] = decode_i8_step(W, 3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(W, args.cpu_seconds)
     if world > 1:
