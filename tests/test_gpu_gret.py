@@ -102,3 +102,26 @@ def test_gret_prefill_long_sequence(cuda_lib):
     o = cuda_lib.gret_prefill(q.cuda(), k.cuda(), v.cuda(), g.cuda(), tau, state=st)
     _check(o, ro, "o")
     _check(st, rs, "final state")
+
+
+def test_gret_prefill_mixed_decay_chunks(cuda_lib):
+    # Chunks of 128 tokens whose gates alternate between strong decay (a
+    # chunk's total decay far below 2^-60), weak decay (far above) and levels
+    # either side of 2^-60, with a carried state and a ragged last chunk: the
+    # kernel's two score paths and every switch between them in one launch.
+    B, H, D, tau, C = 2, 3, 128, 1.0, 128
+    levels = [8.0, -3.0, 8.0, 0.93, 0.98, -3.0, -3.0, 8.0, 0.5]   # gate logit per chunk
+    T = C * (len(levels) - 1) + 37
+    q, k, v, _ = _inputs(B, T, H, D, 1500, 0.0)
+    base = torch.tensor([levels[t // C] for t in range(T)], dtype=F32)
+    g = base[None, :, None] + 0.05 * wl.normal((B, T, H), 1505, F32)
+    s0 = wl.normal((B, H, D, D), 1510, F32) * 0.5
+    lg = oracle.gret_log_decay(g.numpy(), tau)
+    # the levels do straddle the threshold: some chunk totals above 2^-60, some below
+    totals = [lg[0, i * C:(i + 1) * C, 0].sum() / np.log(2) for i in range(len(levels) - 1)]
+    assert min(totals) < -60 < max(totals)
+    ro, rs = oracle.gret_recurrent(q, k, v, lg, state=s0)
+    st = s0.clone().cuda()
+    o = cuda_lib.gret_prefill(q.cuda(), k.cuda(), v.cuda(), g.cuda(), tau, state=st)
+    _check(o, ro, "o")
+    _check(st, rs, "final state")
