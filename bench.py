@@ -61,7 +61,8 @@ def parse_args():
     ap.add_argument("--no-early-exit", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer",
-                                       "gret", "gret_decode", "decode_i8_layer", "gret1", "decode_i8"],
+                                       "gret", "gret_decode", "decode_i8_layer", "gret1", "decode_i8",
+                                       "long_prefill", "long_decode"],
                     default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
@@ -590,6 +591,9 @@ def run_case(args):
       gret_decode  one gated-retention decode step, batch 16, 32 heads (state 34 MB, L2 flushed)
       decode_i8_layer  one decode layer over the 8-bit cache of the benchmark's decode shape
       gret1 / decode_i8  the same at batch 1 / at the decode case's shape (for profiling)
+      long_prefill / long_decode  the 1M-token context (K/V 4 GiB): the last 32K-query
+               chunk of the causal prefill over the whole prefix / one decode step of one
+               sequence over all 1,048,576 rows
     Prints one JSON line with the mean launch time and the work rate."""
     import torch
     import shared_kv_decoder_b200 as yoco
@@ -635,6 +639,20 @@ def run_case(args):
                          dtype=torch.uint8, device=dev)
         fn = lambda: yoco.cross_decode_i8(q, kq, vq, Hkv, ss, sl, int(lens.max()), workspace=ws, o=o)
         work, unit = rows * 2.0 * yoco.kv_i8_row_bytes(Hkv, D), "GB/s"
+    elif args.case in ("long_prefill", "long_decode"):
+        T, C = 1 << 20, 32768
+        k = wl.normal((1, T, Hkv, D), 5001, bf, dev); v = wl.normal((1, T, Hkv, D), 5002, bf, dev)
+        if args.case == "long_prefill":
+            q = wl.normal((1, C, Hq, D), 5003, bf, dev); o = torch.empty_like(q)
+            fn = lambda: yoco.cross_prefill(q, k, v, q_pos0=T - C, o=o)
+            work, unit = prefill_flops_per_layer(C, Hq, D, T - C), "TFLOP/s"
+        else:
+            q = wl.normal((1, Hq, D), 5004, bf, dev); o = torch.empty_like(q)
+            ss = torch.zeros(1, dtype=torch.int64, device=dev)
+            sl = torch.tensor([T], dtype=torch.int32, device=dev)
+            ws = torch.empty(yoco.cross_decode_workspace_size(1, T, Hq, Hkv, D, bf), dtype=torch.uint8, device=dev)
+            fn = lambda: yoco.cross_decode(q, k[0], v[0], ss, sl, T, workspace=ws, o=o)
+            work, unit = T * Hkv * D * 4.0, "GB/s"
     elif args.case in ("gret", "gret1"):
         B, T, H = (GRET["B"] if args.case == "gret" else 1), GRET["T"], GRET["H"]
         q = wl.normal((B, T, H, D), 14, bf, dev); k = wl.normal((B, T, H, D), 15, bf, dev)
