@@ -24,7 +24,9 @@
 //    epilogue of chunk i overlaps the MMAs of chunk i+1.  Four-stage
 //    A/B ring.  Output columns below split_col go to out0, the rest to out1;
 //    dst_rows scatters rows (appending to the shared cache).
-// All waits are bounded (status word + abort flag); see prefill_tc.cu.
+// All mbarrier waits are bounded (status word + abort flag); see prefill_tc.cu.
+// The epilogue warps' one named barrier is a vote that all four reach on
+// every chunk, so a wait that gives up in one of them releases all of them.
 #include <cuda.h>
 
 #include <algorithm>
@@ -83,7 +85,20 @@ YOCO_DEV bool wait1(uint64_t *bar, uint32_t parity) {
 YOCO_DEV bool waitw(uint64_t *bar, uint32_t parity) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, &g_status_project_tc));
 }
-YOCO_DEV void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier of the four epilogue warps with an OR vote: true for every
+// thread if any thread passed true.
+YOCO_DEV bool epi_bar_any(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
 
 }  // namespace
 
@@ -236,24 +251,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int w1 = p.m - p.split_col;
         const int64_t drow = real_row ? (p.dst_rows ? p.dst_rows[tok] : tok) : 0;
-        for (int ci = 0; ci < n_chunks && ok; ++ci) {
+        // every epilogue warp enters this loop and reaches the vote on each
+        // chunk (a failed statistics wait included); any failure ends all four
+        for (int ci = 0; ci < n_chunks; ++ci) {
             const int ab = ci & 1;
-            if (!waitw(&bars[kAccFull + ab], (ci >> 1) & 1)) { ok = false; break; }
-            tc::fence_after_sync();
+            const bool got = ok && waitw(&bars[kAccFull + ab], (ci >> 1) & 1);
             const uint32_t tacc = tmem + lane_off + ab * kBN;
             float *cs = colsum + ab * kBN;
-            if (warp == 3) {  // lane 31 of warp 3 holds row 127: colsum of W
+            if (got) {
+                tc::fence_after_sync();
+                if (warp == 3) {  // lane 31 of warp 3 holds row 127: colsum of W
 #pragma unroll 1
-                for (int cc = 0; cc < kBN; cc += 32) {
-                    float v[32];
-                    tc::tmem_ld32(tacc + cc, v);
-                    tc::wait_ld();
-                    if (lane == 31)
+                    for (int cc = 0; cc < kBN; cc += 32) {
+                        float v[32];
+                        tc::tmem_ld32(tacc + cc, v);
+                        tc::wait_ld();
+                        if (lane == 31)
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) cs[cc + e] = v[e];
+                            for (int e = 0; e < 32; ++e) cs[cc + e] = v[e];
+                    }
                 }
             }
-            epi_bar();
+            if (epi_bar_any(!got)) { ok = false; break; }
             const int col0 = (chunk0 + ci) * kBN;
 #pragma unroll 1
             for (int cc = 0; cc < kBN; cc += 32) {
