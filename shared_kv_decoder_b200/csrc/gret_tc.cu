@@ -24,10 +24,11 @@
 // Shared memory (224 KB): Q, K, V (two buffers), K_w, S_prev rounded to bf16
 // and laid out like a V tile for the cross term, and the bf16 output tile
 // that the TMA stores.  The cross term's rounding is of the same order as the
-// bf16 rounding of P in P V and of K_w in the update (an fp64 emulation of
-// the chunk loop: rel-L2 2.7e-3 against 2.3e-3 with a two-part bf16 split of
-// S, both dominated by those other roundings); the state itself stays fp32
-// in TMEM.  The running log-decay sums live in registers and are exchanged
+// bf16 rounding of P in P V and of K_w in the update: an fp64 emulation of
+// the chunk loop with every bf16 rounding of this kernel, scores from K_w
+// included, gives rel-L2 2.9e-3 against the exact recurrence (2.3e-3 with a
+// two-part bf16 split of S and exponentials for the scores); the state
+// itself stays fp32 in TMEM.  The running log-decay sums live in registers and are exchanged
 // by warp shuffles.
 // Warp roles (352 threads):
 //   warps 0-3  output: P, then o = O + 2^{c_r} X into the output tile (warp 0
