@@ -203,7 +203,11 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
  * yoco_cross_decode_i8: yoco_cross_decode over 8-bit caches (same q, o, lse,
  * sequence and workspace arguments; the workspace size is
  * yoco_cross_decode_workspace_size with the bf16 cfg).  Built for D = 128
- * and bf16 q / o; other shapes return YOCO_ERR_UNSUPPORTED. */
+ * and bf16 q / o; other shapes return YOCO_ERR_UNSUPPORTED.  The scores are
+ * integer products of the K codes with q held per query head as 15-bit
+ * fixed point (a step of 1/16256 of the head's largest |q|, well below bf16's
+ * own rounding of q); everything else is the attention over the dequantised
+ * values. */
 int64_t yoco_kv_i8_row_bytes(const yoco_attn_cfg *cfg);
 yoco_status yoco_kv_quantize_i8(const void *k, const void *v, int64_t n_tok, const int64_t *dst_rows, void *k_i8,
                                 void *v_i8, const yoco_attn_cfg *cfg, cudaStream_t stream);
