@@ -10,8 +10,9 @@
 //   S_t     = gamma_t S_{t-1} + scale * k_t^T v_t       (S: D x D, fp32)
 //   o_t     = q_t S_t
 //
-// gret_prefill_kernel (bf16): one CTA of eight warps per (batch, head) walks
-// the sequence in chunks of 64 tokens.  With c_r the running sum of log gamma
+// gret_prefill_kernel (bf16, head dim 64; head dim 128 runs on the tensor-core
+// kernel in gret_tc.cu): one CTA of eight warps per (batch, head) walks the
+// sequence in chunks of 64 tokens.  With c_r the running sum of log gamma
 // over the chunk's rows 0..r:
 //   o_r   = sum_{u<=r} e^{c_r - c_u} scale (q_r . k_u) v_u      (inner part)
 //         + e^{c_r} q_r S_prev                                   (cross part)
