@@ -4,10 +4,12 @@
 One step is one pass of the whole hot path over one batch of synthetic,
 seeded inputs (bf16, ~N(0,1); weights ~N(0,1/d)):
 
-  swa      self-decoder layer slice: K/V projection of B=4 x T=65536 tokens
-           (d=4096) with the YOCO++ blend fused, sliding-window prefill
-           (window 1024, 32q/8kv heads, head_dim 128) with ring fill, then one
-           decode step (projection of 4 new tokens + ring write + window read)
+  swa      self-decoder, 16 sliding-window layers over B=4 x T=65536 tokens
+           (d=4096, window 1024, 32q/8kv heads, head_dim 128): per layer the
+           K/V projection with the YOCO++ blend to the bottom layer's K/V
+           (w_l ~ U(0,1)) fused, then the SWA prefill with ring fill; then 256
+           decode steps x 16 layers (projection of the 4 new tokens with the
+           blend, ring write, window read), replayed from one CUDA graph
   gkv      global KV produced once: LN(x) W_kv^g for T=32768 tokens
   prefill  cross-decoder causal prefill, T=32768, 32q/8kv, head_dim 128,
            14 cross layers (each its own Q) over the one shared K/V   <- value
@@ -15,13 +17,19 @@ seeded inputs (bf16, ~N(0,1); weights ~N(0,1/d)):
            layers each read the whole shared cache, batch 16, ragged
            lengths uniform in [65536, 131072]                          <- decode
 
+Beside the step (timed once per run, after it): the 1M-token context (one
+sequence, K/V 4 GiB): all 32 chunks of one cross layer's causal prefill, then
+64 decode steps x 16 cross layers at full context with one global-KV row
+appended per step; plus the early-exit prefill and the extension rows.
+
 `value` is the cross-decoder prefill throughput in TFLOP/s of algorithmic
 work (causal pairs only: 4 * Hq * D * sum_i (i + 1) per layer); `decode`
 carries tokens/s and HBM GB/s.  Inputs are resident in HBM when the timed
 region starts; a 256 MB buffer is rewritten between steps to flush L2 (every
 part's inputs are also larger than L2).  Times are CUDA events on the
 launching stream; with several GPUs each rank runs an independent replica and
-the max over ranks is taken.
+the max over ranks is taken.  The library's device status word is read after
+every timed block: a kernel whose bounded wait gave up makes the run fail.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl yoco|reference]
 """
@@ -40,11 +48,14 @@ if ROOT not in sys.path:
 
 METRIC = "cross-decoder prefill TFLOP/s + decode tokens/s & HBM GB/s, 1 B200"
 WORKLOAD = ("cross-decoder causal prefill B=1 T=32768 32q/8kv D=128 x14 layers over one shared KV "
-            "+ decode step B=16 ragged 64K-128K x16 layers + SWA/blend layer slice B=4 T=65536 W=1024")
+            "+ decode step B=16 ragged 64K-128K x16 layers + self-decoder SWA prefill B=4 T=65536 W=1024 "
+            "x16 layers with YOCO++ blend and 256 decode steps")
 
 P = dict(T=32768, Hq=32, Hkv=8, D=128, layers=14, d=4096)          # cross prefill
 DEC = dict(B=16, lo=65536, hi=131072, Hq=32, Hkv=8, D=128, layers=16, d=4096, seed=2000)
-SWA = dict(B=4, T=65536, W=1024, Hq=32, Hkv=8, D=128, d=4096)
+SWA = dict(B=4, T=65536, W=1024, Hq=32, Hkv=8, D=128, d=4096, layers=16, steps=256)
+# 1M-token context: one cross layer's 32-chunk prefill, 64 decode steps x 16 layers
+LONG = dict(T=1 << 20, C=32768, Hq=32, Hkv=8, D=128, d=4096, layers=16, steps=64)
 SELF_LAYERS = 14    # self-decoder depth of the early-exit measurement (half of a 28-layer stack)
 # gated-retention self-decoder layer (the sliding-window slice's shape with retention heads)
 GRET = dict(B=4, T=65536, H=32, D=128, tau=16.0, B_dec=16)
@@ -59,10 +70,13 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-early-exit", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the 1M-token context block")
+    ap.add_argument("--chunk-parallel", action="store_true",
+                    help="chunk-parallel prefill of one long sequence across the ranks (NCCL)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer",
                                        "gret", "gret_decode", "decode_i8_layer", "gret1", "decode_i8",
-                                       "long_prefill", "long_decode"],
+                                       "long_prefill", "long_decode", "swa_decode_layer"],
                     default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
@@ -222,33 +236,99 @@ def make_workload(dev):
     W["max_len"] = int(lens.max())
     W["ws"] = torch.empty(yoco.cross_decode_workspace_size(DEC["B"], W["max_len"], Hq, Hkv, D, bf),
                           dtype=torch.uint8, device=dev)
-    # self-decoder slice
-    B4, T4, W4 = SWA["B"], SWA["T"], SWA["W"]
+    # self-decoder: 16 sliding-window layers, each with its own x_l, W_kv^l,
+    # Q_l and YOCO++ weight w_l (w_1 unused: the bottom layer is not blended)
+    B4, T4, W4, L4, S4 = SWA["B"], SWA["T"], SWA["W"], SWA["layers"], SWA["steps"]
     n4 = B4 * T4
-    W["x4"] = wl.normal((n4, d), 3001, bf, dev)
-    W["w4"] = wl.normal((2 * Hkv * D, d), 3002, bf, dev, std=d ** -0.5)
-    W["k1"] = wl.normal((n4, Hkv, D), 3003, bf, dev)
-    W["v1"] = wl.normal((n4, Hkv, D), 3004, bf, dev)
-    W["w_l"] = float(wl.uniform((1,), 3005)[0])
-    W["k4"] = torch.empty((B4, T4, Hkv, D), dtype=bf, device=dev)
-    W["v4"] = torch.empty((B4, T4, Hkv, D), dtype=bf, device=dev)
-    W["q4"] = wl.normal((B4, T4, Hq, D), 3006, bf, dev)
+    W["x4"] = [wl.normal((n4, d), 3100 + l, bf, dev) for l in range(L4)]
+    W["w4"] = [wl.normal((2 * Hkv * D, d), 3200 + l, bf, dev, std=d ** -0.5) for l in range(L4)]
+    W["q4"] = [wl.normal((B4, T4, Hq, D), 3300 + l, bf, dev) for l in range(L4)]
+    W["w_l"] = [float(v) for v in wl.uniform((L4,), 3005)]
+    W["k1"], W["v1"], W["k4"], W["v4"] = (torch.empty((B4, T4, Hkv, D), dtype=bf, device=dev)
+                                          for _ in range(4))
     W["o4"] = torch.empty((B4, T4, Hq, D), dtype=bf, device=dev)
-    W["ring"] = (torch.empty((B4, W4, Hkv, D), dtype=bf, device=dev),
-                 torch.empty((B4, W4, Hkv, D), dtype=bf, device=dev),
-                 torch.empty((B4, W4), dtype=torch.int32, device=dev))
-    W["x4t"] = wl.normal((B4, d), 3007, bf, dev)
-    W["k1t"] = wl.normal((B4, Hkv, D), 3008, bf, dev)
-    W["v1t"] = wl.normal((B4, Hkv, D), 3009, bf, dev)
-    W["q4t"] = wl.normal((B4, Hq, D), 3010, bf, dev)
-    W["k4t"] = torch.empty((B4, Hkv, D), dtype=bf, device=dev)
-    W["v4t"] = torch.empty((B4, Hkv, D), dtype=bf, device=dev)
+    W["rings"] = [(torch.empty((B4, W4, Hkv, D), dtype=bf, device=dev),
+                   torch.empty((B4, W4, Hkv, D), dtype=bf, device=dev),
+                   torch.empty((B4, W4), dtype=torch.int32, device=dev)) for _ in range(L4)]
+    # decode steps past the prompt: per step and layer the 4 new tokens' x and q
+    W["x4d"] = wl.normal((S4, L4, B4, d), 3400, bf, dev)
+    W["q4d"] = wl.normal((S4, L4, B4, Hq, D), 3401, bf, dev)
+    W["pos4"] = (T4 + torch.arange(S4, dtype=torch.int64, device=dev))[:, None].repeat(1, B4).contiguous()
+    W["k1t"], W["v1t"], W["k4t"], W["v4t"] = (torch.empty((B4, Hkv, D), dtype=bf, device=dev)
+                                              for _ in range(4))
     W["o4t"] = torch.empty((B4, Hq, D), dtype=bf, device=dev)
-    W["pos4"] = torch.full((B4,), T4, dtype=torch.int64, device=dev)
     W["ws4"] = torch.empty(yoco.swa_decode_workspace_size(B4, W4, Hq, Hkv, D, bf),
                            dtype=torch.uint8, device=dev)
     W["flush"] = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     return W
+
+
+def self_decoder_prefill(W, ev=None):
+    """The 16 sliding-window layers over the B=4 x T=65536 prompt: the bottom
+    layer's K/V projection, then for every other layer its projection with the
+    YOCO++ blend w_l * (K_1, V_1) fused; each followed by the SWA prefill,
+    which also fills that layer's ring."""
+    import shared_kv_decoder_b200 as yoco
+    Hkv, D, Wn = SWA["Hkv"], SWA["D"], SWA["W"]
+    flat = lambda t: t.view(-1, Hkv, D)
+    for l in range(SWA["layers"]):
+        if ev is not None:
+            ev["swa_proj"][2 * l].record()
+        if l == 0:
+            yoco.kv_project_blend(W["x4"][0], W["w4"][0], Hkv, D, k_out=flat(W["k1"]), v_out=flat(W["v1"]))
+            k, v = W["k1"], W["v1"]
+        else:
+            yoco.kv_project_blend(W["x4"][l], W["w4"][l], Hkv, D, flat(W["k1"]), flat(W["v1"]),
+                                  W["w_l"][l], W["w_l"][l], k_out=flat(W["k4"]), v_out=flat(W["v4"]))
+            k, v = W["k4"], W["v4"]
+        if ev is not None:
+            ev["swa_proj"][2 * l + 1].record()
+            ev["swa_att"][2 * l].record()
+        yoco.swa_prefill(W["q4"][l], k, v, Wn, ring=W["rings"][l], o=W["o4"])
+        if ev is not None:
+            ev["swa_att"][2 * l + 1].record()
+
+
+def self_decoder_decode(W):
+    """256 decode steps of the 16 sliding-window layers: per step and layer
+    the 4 new tokens' K/V projection (blended with the bottom layer's K/V of
+    the same tokens), their ring write and the window read.  Position T + s
+    of step s overwrites the ring slot of T + s - window, so replaying the
+    steps after a prefill is idempotent."""
+    import shared_kv_decoder_b200 as yoco
+    Hkv, D, Wn = SWA["Hkv"], SWA["D"], SWA["W"]
+    for s in range(SWA["steps"]):
+        for l in range(SWA["layers"]):
+            if l == 0:
+                yoco.kv_project_blend(W["x4d"][s, 0], W["w4"][0], Hkv, D, k_out=W["k1t"], v_out=W["v1t"])
+                kn, vn = W["k1t"], W["v1t"]
+            else:
+                yoco.kv_project_blend(W["x4d"][s, l], W["w4"][l], Hkv, D, W["k1t"], W["v1t"],
+                                      W["w_l"][l], W["w_l"][l], k_out=W["k4t"], v_out=W["v4t"])
+                kn, vn = W["k4t"], W["v4t"]
+            rk, rv, sp = W["rings"][l]
+            yoco.swa_decode(W["q4d"][s, l], kn, vn, W["pos4"][s], rk, rv, sp, Wn,
+                            workspace=W["ws4"], o=W["o4t"])
+
+
+def capture_self_decoder_decode(W):
+    """One CUDA graph of the 256 x 16 decode layer-steps (4 kernels each), so
+    the steps run back to back without host launch overhead.  The rings must
+    hold a prefill's contents (the graph is recorded after one eager run).
+    Returns the number of library kernels one replay launches."""
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    self_decoder_prefill(W)
+    self_decoder_decode(W)          # eager once: every kernel's attributes are set
+    torch.cuda.synchronize()
+    n0 = yoco.launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        self_decoder_decode(W)
+    torch.cuda.synchronize()
+    W["swa_graph"] = g
+    W["swa_graph_launches"] = yoco.launch_count() - n0
+    return W["swa_graph_launches"]
 
 
 def run_step(W, ev=None):
@@ -260,17 +340,14 @@ def run_step(W, ev=None):
         if ev is not None:
             ev[name][i].record()
 
-    # self-decoder slice (projection + blend, SWA prefill + ring, one decode step)
+    # self-decoder: 16-layer prefill (projection + blend, SWA + ring), then
+    # 256 decode steps of the 16 layers
     rec("swa", 0)
-    yoco.kv_project_blend(W["x4"], W["w4"], Hkv, D, W["k1"], W["v1"], W["w_l"], W["w_l"],
-                          k_out=W["k4"].view(-1, Hkv, D), v_out=W["v4"].view(-1, Hkv, D))
-    yoco.swa_prefill(W["q4"], W["k4"], W["v4"], SWA["W"], ring=W["ring"], o=W["o4"])
-    yoco.kv_project_blend(W["x4t"], W["w4"], Hkv, D, W["k1t"], W["v1t"], W["w_l"], W["w_l"],
-                          k_out=W["k4t"], v_out=W["v4t"])
-    rk, rv, sp = W["ring"]
-    yoco.swa_decode(W["q4t"], W["k4t"], W["v4t"], W["pos4"], rk, rv, sp, SWA["W"],
-                    workspace=W["ws4"], o=W["o4t"])
+    self_decoder_prefill(W, ev)
     rec("swa", 1)
+    rec("swa_dec", 0)
+    W["swa_graph"].replay()
+    rec("swa_dec", 1)
     # global KV, produced once
     rec("gkv", 0)
     yoco.kv_project_blend(W["x_mid"], W["w_g"], Hkv, D, k_out=W["kg"].view(-1, Hkv, D),
@@ -300,8 +377,21 @@ def run_step(W, ev=None):
 def new_events():
     import torch
     mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-    return {"swa": mk(2), "gkv": mk(2), "decode": mk(2), "prefill_l": mk(2 * P["layers"]),
-            "decode_l": mk(2 * DEC["layers"]), "step": mk(2)}
+    return {"swa": mk(2), "swa_dec": mk(2), "swa_proj": mk(2 * SWA["layers"]),
+            "swa_att": mk(2 * SWA["layers"]), "gkv": mk(2), "decode": mk(2),
+            "prefill_l": mk(2 * P["layers"]), "decode_l": mk(2 * DEC["layers"]), "step": mk(2)}
+
+
+def swa_tile_flops_per_layer(B, T, Hq, D, window):
+    """FLOPs the tensor cores execute for a sliding-window prefill layer: every
+    visited 128 x 128 (query, key) tile in full, 4 * D FLOP per pair, with the
+    visited KV tiles of a query tile being those that hold a visible pair."""
+    n = 0
+    for qt in range(-(-T // 128)):
+        p_first, p_last = qt * 128, min(qt * 128 + 128, T) - 1
+        lo = max(0, p_first - window + 1) // 128
+        n += p_last // 128 - lo + 1
+    return 4.0 * D * 128 * 128 * n * B * Hq
 
 
 def early_exit(W, reps):
@@ -451,6 +541,85 @@ def decode_i8_step(W, reps):
                     "(token, KV head): half the cache bytes"}
 
 
+def long_context(W, peaks):
+    """The 1M-token context, measured beside the step (once per run): one
+    sequence whose shared K/V holds 1,048,576 rows (4 GiB of K and V).
+
+    Prefill: all 32 chunks of 32768 queries of one cross layer, chunk c at
+    positions [c C, (c + 1) C) attending causally to keys [0, (c + 1) C) (each
+    chunk its own seeded Q; 9.007e15 FLOP of visible pairs).  The other 15
+    cross layers repeat the same work on their own Q; one layer is timed in
+    full.  Decode: 64 steps, each appending the new token's global-KV row
+    (LN(x) W_kv^g written at row T + s) and then 16 cross layers over all
+    T + s + 1 rows.  Device ms from CUDA events; the first chunk and two
+    decode steps run once untimed first (the decode rows they append are
+    appended again, with the same values, by the timed steps)."""
+    import torch
+    import shared_kv_decoder_b200 as yoco
+    import workloads as wl
+    bf, dev = torch.bfloat16, W["o"].device
+    T, C, Hq, Hkv, D, d, L, S = (LONG[k] for k in ("T", "C", "Hq", "Hkv", "D", "d", "layers", "steps"))
+    n_chunks = T // C
+    kc = wl.normal((T + S, Hkv, D), 5001, bf, dev)
+    vc = wl.normal((T + S, Hkv, D), 5002, bf, dev)
+    qs = [wl.normal((1, C, Hq, D), 5100 + c, bf, dev) for c in range(n_chunks)]
+    o = torch.empty((1, C, Hq, D), dtype=bf, device=dev)
+    xd = wl.normal((S, 1, d), 5003, bf, dev)
+    wg = wl.normal((2 * Hkv * D, d), 5004, bf, dev, std=d ** -0.5)
+    qd = wl.normal((S, L, 1, Hq, D), 5005, bf, dev)
+    od = torch.empty((1, Hq, D), dtype=bf, device=dev)
+    rows = [torch.tensor([T + s], dtype=torch.int64, device=dev) for s in range(S)]
+    ss = torch.zeros(1, dtype=torch.int64, device=dev)
+    sl = [torch.tensor([T + s + 1], dtype=torch.int32, device=dev) for s in range(S)]
+    max_len = T + S
+    ws = torch.empty(yoco.cross_decode_workspace_size(1, max_len, Hq, Hkv, D, bf), dtype=torch.uint8, device=dev)
+
+    def chunk(c):
+        n = (c + 1) * C
+        yoco.cross_prefill(qs[c], kc[:n].view(1, n, Hkv, D), vc[:n].view(1, n, Hkv, D), q_pos0=c * C, o=o)
+
+    def step(s):
+        yoco.kv_project_blend(xd[s], wg, Hkv, D, dst_rows=rows[s], k_out=kc, v_out=vc)
+        for l in range(L):
+            yoco.cross_decode(qd[s, l], kc, vc, ss, sl[s], max_len, workspace=ws, o=od)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    chunk(n_chunks - 1)
+    step(0); step(1)
+    torch.cuda.synchronize()
+    W["flush"].zero_()
+    ce = [(ev(), ev()) for _ in range(n_chunks)]
+    for c in range(n_chunks):
+        ce[c][0].record(); chunk(c); ce[c][1].record()
+    W["flush"].zero_()
+    d0, d1 = ev(), ev()
+    d0.record()
+    for s in range(S):
+        step(s)
+    d1.record()
+    torch.cuda.synchronize()
+    chunk_ms = [a.elapsed_time(b) for a, b in ce]
+    pre_ms = sum(chunk_ms)
+    pre_fl = sum(prefill_flops_per_layer(C, Hq, D, c * C) for c in range(n_chunks))
+    last_fl = prefill_flops_per_layer(C, Hq, D, T - C)
+    dec_ms = d0.elapsed_time(d1)
+    row_bytes = Hkv * D * 2 * 2
+    dec_bytes = L * sum((T + s + 1) * row_bytes for s in range(S))
+    pre_tf = pre_fl / (pre_ms * 1e-3) / 1e12
+    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+    del kc, vc, qs
+    return {"T": T, "chunk": C, "chunks": n_chunks, "prefill_layers_timed": 1,
+            "prefill_ms_per_layer": pre_ms, "prefill_flops_per_layer": pre_fl, "prefill_tflops": pre_tf,
+            "prefill_frac": pre_tf / peaks["bf16_sus"], "prefill_peak_src": f"{peaks['src']} bf16 sustained",
+            "last_chunk_ms": chunk_ms[-1], "last_chunk_tflops": last_fl / (chunk_ms[-1] * 1e-3) / 1e12,
+            "decode_steps": S, "decode_layers": L, "decode_ms_per_step": dec_ms / S,
+            "decode_tokens_per_s": S / (dec_ms * 1e-3), "decode_hbm_gbs": dec_gbs,
+            "decode_frac": dec_gbs / peaks["hbm"], "decode_peak_src": f"{peaks['src']} hbm",
+            "note": "one cross layer's 32-chunk prefill timed in full (the other 15 layers repeat it on "
+                    "their own Q); decode: per step the appended row's projection + 16 cross layers over "
+                    "the whole cache; bytes are the K/V rows each layer reads"}
+
+
 def e2e_prefill(W, steps, warmup):
     """Prefill through the public API with HOST buffers: every step copies the
     step's Q (14 layers) and the shared K/V from pinned host memory and reads
@@ -594,6 +763,8 @@ def run_case(args):
       long_prefill / long_decode  the 1M-token context (K/V 4 GiB): the last 32K-query
                chunk of the causal prefill over the whole prefix / one decode step of one
                sequence over all 1,048,576 rows
+      swa_decode_layer  one sliding-window decode call at the self-decoder's shape (batch 4,
+               window 1024: ring write + window attention + merge over 16.8 MB of ring)
     Prints one JSON line with the mean launch time and the work rate."""
     import torch
     import shared_kv_decoder_b200 as yoco
@@ -625,6 +796,18 @@ def run_case(args):
         v = wl.normal((1, T, Hkv, D), 9, bf, dev); o = torch.empty_like(q)
         fn = lambda: yoco.swa_prefill(q, k, v, Wn, o=o)
         work, unit = prefill_flops_per_layer(T, Hq, D, 0, Wn), "TFLOP/s"
+    elif args.case == "swa_decode_layer":
+        B, T, Wn = SWA["B"], 4096, SWA["W"]
+        k = wl.normal((B, T, Hkv, D), 8, bf, dev); v = wl.normal((B, T, Hkv, D), 9, bf, dev)
+        ring = (torch.empty((B, Wn, Hkv, D), dtype=bf, device=dev), torch.empty((B, Wn, Hkv, D), dtype=bf, device=dev),
+                torch.empty((B, Wn), dtype=torch.int32, device=dev))
+        yoco.swa_prefill(wl.normal((B, T, Hq, D), 7, bf, dev), k, v, Wn, ring=ring)
+        q = wl.normal((B, Hq, D), 10, bf, dev); o = torch.empty_like(q)
+        kn = wl.normal((B, Hkv, D), 11, bf, dev); vn = wl.normal((B, Hkv, D), 12, bf, dev)
+        pos = torch.full((B,), T, dtype=torch.int64, device=dev)
+        ws = torch.empty(yoco.swa_decode_workspace_size(B, Wn, Hq, Hkv, D, bf), dtype=torch.uint8, device=dev)
+        fn = lambda: yoco.swa_decode(q, kn, vn, pos, ring[0], ring[1], ring[2], Wn, workspace=ws, o=o)
+        work, unit = 2.0 * B * Wn * Hkv * D * 2, "GB/s"
     elif args.case in ("decode_i8_layer", "decode_i8"):
         lens = (wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], DEC["seed"]) if args.case == "decode_i8_layer"
                 else wl.ragged_lengths(16, 16384, 32768, 9))
@@ -690,10 +873,152 @@ def run_case(args):
                       "status": yoco.device_status()}), flush=True)
 
 
+# chunk-parallel prefill across ranks: per rank one chunk of one long sequence
+CP = dict(Tc=16384, Hq=32, Hkv=8, D=128, W=1024, self_layers=4, cross_layers=4)
+
+
+class _Clock:
+    """Device time on CUDA (events on the current stream), host time on CPU."""
+
+    def __init__(self, device):
+        self.cuda = device.type == "cuda"
+
+    def mark(self):
+        import torch
+        if self.cuda:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            return e
+        return time.perf_counter()
+
+    def ms(self, a, b):
+        return a.elapsed_time(b) if self.cuda else (b - a) * 1e3
+
+
+def chunk_parallel_measure(comm, ops, device, dtype, steps, warmup, Tc, Hq, Hkv, D, W, self_layers,
+                           cross_layers):
+    """Chunk-parallel prefill of one sequence of world * Tc tokens ("You Only
+    Cache Once", paperlayer summary, Appendix A): rank r holds positions
+    [r Tc, (r + 1) Tc).  A step runs, on every rank, `self_layers` sliding-
+    window layers (each exchanging a window - 1 row halo with the neighbour
+    rank), ONE all-gather of the global K/V, then `cross_layers` causal cross
+    layers of the rank's rows over the gathered prefix.  Inputs are seeded per
+    rank and layer and resident before timing.  Returns this rank's report
+    (times, FLOPs) and the last step's outputs (last self layer, last cross
+    layer)."""
+    import torch
+    import workloads as wl
+    from shared_kv_decoder_b200 import chunk_parallel as cp
+    r, world = comm.rank, comm.world
+    s0 = r * Tc
+    gen = lambda shape, seed: wl.normal(shape, seed, dtype, device)
+    qs = [gen((1, Tc, Hq, D), 6000 + 100 * l + r) for l in range(self_layers)]
+    ks = [gen((1, Tc, Hkv, D), 6010 + 100 * l + r) for l in range(self_layers)]
+    vs = [gen((1, Tc, Hkv, D), 6020 + 100 * l + r) for l in range(self_layers)]
+    kg = gen((1, Tc, Hkv, D), 6030 + r)
+    vg = gen((1, Tc, Hkv, D), 6040 + r)
+    qc = [gen((1, Tc, Hq, D), 6050 + 100 * l + r) for l in range(cross_layers)]
+    clk = _Clock(device)
+    t_self, t_gather, t_cross = [], [], []
+    out = None
+    for it in range(warmup + steps):
+        m0 = clk.mark()
+        for l in range(self_layers):
+            o_s = cp.swa_chunk(qs[l], ks[l], vs[l], W, comm, ops)
+        m1 = clk.mark()
+        k_all, v_all = cp.gather_global_kv(kg, vg, comm)
+        m2 = clk.mark()
+        for l in range(cross_layers):
+            o_c = cp.cross_chunk(qc[l], k_all, v_all, s0, ops)
+        m3 = clk.mark()
+        if device.type == "cuda":
+            torch.cuda.synchronize()
+        if it >= warmup:
+            t_self.append(clk.ms(m0, m1))
+            t_gather.append(clk.ms(m1, m2))
+            t_cross.append(clk.ms(m2, m3))
+        out = (o_s, o_c)
+    swa_fl = self_layers * 4.0 * Hq * D * sum(min(s0 + i + 1, W) for i in range(Tc))
+    cross_fl = cross_layers * 4.0 * Hq * D * (Tc * s0 + Tc * (Tc + 1) / 2.0)
+    rep = {"rank": r, "ms_self": sum(t_self) / steps, "ms_gather": sum(t_gather) / steps,
+           "ms_cross": sum(t_cross) / steps, "flops_self": swa_fl, "flops_cross": cross_fl,
+           "gather_bytes": 2.0 * world * Tc * Hkv * D * torch.tensor([], dtype=dtype).element_size()}
+    rep["ms_step"] = rep["ms_self"] + rep["ms_gather"] + rep["ms_cross"]
+    return rep, out
+
+
+def run_chunk_parallel(args):
+    """bench.py --chunk-parallel: the chunk-parallel prefill over NCCL, one
+    rank per GPU (torchrun); prints one JSON line from rank 0 with the job's
+    TFLOP/s (all ranks' FLOPs over the slowest rank's step time) and each
+    rank's times, the all-gather's share among them."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import shared_kv_decoder_b200 as yoco
+    from shared_kv_decoder_b200 import chunk_parallel as cp
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29511")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), world_size=world,
+                            rank=int(os.environ.get("RANK", "0")))
+    yoco.load()
+    rep, _ = chunk_parallel_measure(cp.DistComm(), cp.KernelOps, dev, torch.bfloat16, args.steps,
+                                    args.warmup, **CP)
+    st = yoco.device_status()
+    reps = [None] * world
+    dist.all_gather_object(reps, rep)
+    t = torch.tensor([float(st)], device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    worst = int(t.item())
+    dist.barrier()
+    dist.destroy_process_group()
+    if worst != yoco.OK:
+        sys.stderr.write(f"bench: device status {worst}; no number is reported\n")
+        sys.exit(3)
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    step = max(x["ms_step"] for x in reps)
+    flops = sum(x["flops_self"] + x["flops_cross"] for x in reps)
+    out = {"metric": "chunk-parallel prefill TFLOP/s (self-decoder halo + one global-KV all-gather)",
+           "value": flops / (step * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": step, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"one sequence of {world} x {CP['Tc']} tokens, one chunk per rank; "
+                                  f"{CP['self_layers']} SWA layers (window {CP['W']}) + {CP['cross_layers']} "
+                                  "cross layers, 32q/8kv D=128",
+                      "parallelism": f"chunk-parallel over {world} ranks"},
+           "gather_share": max(x["ms_gather"] for x in reps) / step,
+           "ranks": reps, "device_status": worst}
+    print(json.dumps(out), flush=True)
+
+
+class DeviceStatusError(RuntimeError):
+    pass
+
+
+def check_device_status(where, dev):
+    """Read (and clear) the library's device status word after a timed block;
+    any non-OK status on any rank fails the run (every rank takes the same
+    collective step here, on the error path too)."""
+    import shared_kv_decoder_b200 as yoco
+    st = yoco.device_status()
+    worst = int(reduce_max_over_ranks([st], dev)[0])
+    if worst != yoco.OK:
+        raise DeviceStatusError(f"{where}: device status {worst} ({'this rank' if st else 'another rank'})")
+    return st
+
+
 def main():
     args = parse_args()
     if args.case:
         run_case(args)
+        return
+    if args.chunk_parallel:
+        run_chunk_parallel(args)
         return
     if args.impl == "reference":
         run_reference(args)
@@ -710,14 +1035,34 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     import shared_kv_decoder_b200 as yoco
     yoco.load()
+    try:
+        out = measure(args, world, rank, local, dev)
+    except DeviceStatusError as e:
+        sys.stderr.write(f"bench: {e}; no number is reported\n")
+        if world > 1:
+            dist.destroy_process_group()
+        sys.exit(3)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def measure(args, world, rank, local, dev):
+    import torch
+    import torch.distributed as dist
+    import shared_kv_decoder_b200 as yoco
     peaks = load_peaks()
     W = make_workload(dev)
+    graph_launches = capture_self_decoder_decode(W)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
         W["flush"].zero_()
         run_step(W)
     torch.cuda.synchronize()
+    check_device_status("warm-up steps", dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -734,8 +1079,11 @@ def main():
         ev["step"][1].record()
         evs.append(ev)
     torch.cuda.synchronize()
-    launches = yoco.launch_count() - launches0
+    # kernels launched from the library's host calls, plus those each replay
+    # of the self-decoder's decode graph launched (counted once at capture)
+    launches = yoco.launch_count() - launches0 + args.steps * graph_launches
     clk = clocks.stop()
+    status = check_device_status("timed steps", dev)
     if world > 1:
         dist.barrier()
 
@@ -747,11 +1095,15 @@ def main():
     dec_l = [pair(e, "decode_l", 2 * l) for e in evs for l in range(DEC["layers"])]
     pre_ms = [sum(pair(e, "prefill_l", 2 * l) for l in range(P["layers"])) for e in evs]
     dec_ms = [pair(e, "decode") for e in evs]
-    swa_ms = [pair(e, "swa") for e in evs]
+    L4, S4 = SWA["layers"], SWA["steps"]
+    swa_pre_ms = [pair(e, "swa") for e in evs]
+    swa_proj_l = [pair(e, "swa_proj", 2 * l) for e in evs for l in range(L4)]
+    swa_att_l = [pair(e, "swa_att", 2 * l) for e in evs for l in range(L4)]
+    swa_dec_ms = [pair(e, "swa_dec") for e in evs]
     gkv_ms = [pair(e, "gkv") for e in evs]
 
-    mx = reduce_max_over_ranks([sum(step_ms), sum(pre_ms), sum(dec_ms)], dev)
-    tot = {"step": mx[0], "pre": mx[1], "dec": mx[2]}
+    mx = reduce_max_over_ranks([sum(step_ms), sum(pre_ms), sum(dec_ms), sum(swa_pre_ms), sum(swa_dec_ms)], dev)
+    tot = {"step": mx[0], "pre": mx[1], "dec": mx[2], "swa_pre": mx[3], "swa_dec": mx[4]}
 
     f_layer = prefill_flops_per_layer(P["T"], P["Hq"], P["D"])
     value = world * args.steps * P["layers"] * f_layer / (tot["pre"] * 1e-3) / 1e12
@@ -759,9 +1111,21 @@ def main():
     dec_tok_s = world * args.steps * DEC["B"] / (tot["dec"] * 1e-3)
     dec_gbs_layer = dec_bytes_layer / (statistics.mean(dec_l) * 1e-3) / 1e9
     pre_tflops_launch = f_layer / (statistics.mean(pre_l) * 1e-3) / 1e12
-    n4 = SWA["B"] * SWA["T"]
-    swa_proj_fl = 2.0 * n4 * P["d"] * 2 * SWA["Hkv"] * SWA["D"]
-    swa_att_fl = SWA["B"] * prefill_flops_per_layer(SWA["T"], SWA["Hq"], SWA["D"], 0, SWA["W"])
+    B4, T4, W4, Hkv4, D4, d4, Hq4 = (SWA[k] for k in ("B", "T", "W", "Hkv", "D", "d", "Hq"))
+    n4 = B4 * T4
+    swa_proj_fl = 2.0 * n4 * d4 * 2 * Hkv4 * D4
+    swa_att_fl = B4 * prefill_flops_per_layer(T4, Hq4, D4, 0, W4)
+    swa_tile_fl = swa_tile_flops_per_layer(B4, T4, Hq4, D4, W4)
+    swa_att_tf = swa_att_fl / (statistics.mean(swa_att_l) * 1e-3) / 1e12
+    # one decode layer-step reads the layer's ring (K and V, B x W rows) and
+    # its W_kv, reads the 4 new tokens' x, q and the bottom layer's new K/V,
+    # and writes the new K/V (into the ring) and o
+    ring_bytes = 2.0 * B4 * W4 * Hkv4 * D4 * 2
+    wkv_bytes = 2.0 * Hkv4 * D4 * d4 * 2
+    small_bytes = B4 * (d4 + Hq4 * D4 * 2 + 2 * Hkv4 * D4 * 3) * 2.0
+    layer_step_bytes = ring_bytes + wkv_bytes + small_bytes
+    layer_step_ms = tot["swa_dec"] / (args.steps * S4 * L4)
+    swa_dec_gbs = layer_step_bytes / (layer_step_ms * 1e-3) / 1e9
     gkv_fl = 2.0 * P["T"] * P["d"] * 2 * P["Hkv"] * P["D"]
 
     out = {
@@ -775,8 +1139,22 @@ def main():
         "decode": {"tokens_per_s": dec_tok_s, "hbm_gbs": dec_gbs_layer,
                    "frac_hbm": dec_gbs_layer / peaks["hbm"], "ms_per_decode_step": tot["dec"] / args.steps,
                    "bytes_per_layer": dec_bytes_layer},
-        "swa_slice": {"ms": statistics.mean(swa_ms),
-                      "flops": swa_proj_fl + swa_att_fl},
+        "swa": {"shape": f"B={B4} T={T4} window={W4} 32q/8kv D=128 d={d4}, {L4} layers, w_l ~ U(0,1)",
+                "prefill_ms": tot["swa_pre"] / args.steps,
+                "prefill_tokens_per_s": world * args.steps * n4 / (tot["swa_pre"] * 1e-3),
+                "attention_ms_per_layer": statistics.mean(swa_att_l),
+                "attention_tflops": swa_att_tf,
+                "attention_tflops_tile": swa_tile_fl / (statistics.mean(swa_att_l) * 1e-3) / 1e12,
+                "attention_flops_per_layer": swa_att_fl, "attention_tile_flops_per_layer": swa_tile_fl,
+                "projection_ms_per_layer": statistics.mean(swa_proj_l),
+                "projection_tflops": swa_proj_fl / (statistics.mean(swa_proj_l) * 1e-3) / 1e12,
+                "decode_steps": S4, "decode_ms": tot["swa_dec"] / args.steps,
+                "decode_tokens_per_s": world * args.steps * S4 * B4 / (tot["swa_dec"] * 1e-3),
+                "decode_ms_per_layer_step": layer_step_ms, "decode_hbm_gbs": swa_dec_gbs,
+                "decode_bytes_per_layer_step": layer_step_bytes,
+                "note": "attention times include the ring fill; decode = 256 steps x 16 layers from one "
+                        "CUDA graph, each layer-step = projection of the 4 new tokens with the blend, "
+                        "ring write, window attention, split merge"},
         "gkv": {"ms": statistics.mean(gkv_ms), "tflops": gkv_fl / (statistics.mean(gkv_ms) * 1e-3) / 1e12},
         "roofline": {"kernel": "cross prefill (yoco_cross_prefill)", "bound": "tensor",
                      "achieved": pre_tflops_launch, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
@@ -786,25 +1164,43 @@ def main():
                             "achieved": dec_gbs_layer, "peak": peaks["hbm"], "unit": "GB/s",
                             "frac": dec_gbs_layer / peaks["hbm"], "traffic": traffic("decode"),
                             "peak_src": f"{peaks['src']} hbm"},
+        "roofline_swa_prefill": {"kernel": "sliding-window prefill (yoco_swa_prefill)", "bound": "tensor",
+                                 "achieved": swa_att_tf, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                                 "frac": swa_att_tf / peaks["bf16_sus"], "traffic": None,
+                                 "peak_src": f"{peaks['src']} bf16 sustained"},
+        "roofline_swa_decode": {"kernel": "sliding-window decode layer-step (projection + yoco_swa_decode)",
+                                "bound": "hbm", "achieved": swa_dec_gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                                "frac": swa_dec_gbs / peaks["hbm"], "traffic": None,
+                                "peak_src": f"{peaks['src']} hbm"},
         "gpu_launches": launches,
         "clocks": clk,
+        "device_status": status,
     }
+    # the self-decoder's inputs are not needed by the blocks below
+    W["swa_graph"].reset()
+    for k_ in ("x4", "q4", "x4d", "q4d", "k1", "v1", "k4", "v4", "o4"):
+        W.pop(k_, None)
+    torch.cuda.empty_cache()
     if not args.no_e2e:
         times, h2d, d2h = e2e_prefill(W, args.steps, args.warmup)
+        check_device_status("e2e", dev)
         e2e_ms = reduce_max_over_ranks([sum(times)], dev)[0]
         out["e2e"] = {"value": world * len(times) * P["layers"] * f_layer / (e2e_ms * 1e-3) / 1e12,
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if not args.no_long:
+        out["long_context"] = long_context(W, peaks)
+        check_device_status("long context", dev)
+        torch.cuda.empty_cache()
     if not args.no_early_exit:
         out["early_exit"] = early_exit(W, 3)
+        check_device_status("early exit", dev)
         out["gret"] = gret_layer(W, 3)
+        check_device_status("gated retention", dev)
         out["decode_i8"] = decode_i8_step(W, 3)
+        check_device_status("8-bit decode", dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(W, args.cpu_seconds)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(out), flush=True)
+    return out
 
 
 if __name__ == "__main__":

@@ -132,15 +132,21 @@ yoco_status yoco_cross_prefill(const void *q, const void *k, const void *v, int3
 
 /* Cross-decoder decode step: one new query token per sequence reads the whole
  * shared cache (podcast cue 26), split across the GPU and merged.
- * q [B, Hq, D]; k_cache, v_cache packed [rows, Hkv, D]; sequence b owns rows
- * [seq_start[b], seq_start[b] + seq_len[b]) (device int64 / int32 arrays,
- * seq_len >= 1 and including the new token's row).  max_len >= every
- * seq_len (host value; sizes the split plan without a device read).
+ * q [B, Hq, D]; k_cache, v_cache packed [cache_rows, Hkv, D] (both buffers
+ * hold at least cache_rows rows, 1 <= cache_rows <= 2^31 - 1); sequence b
+ * owns rows [seq_start[b], seq_start[b] + seq_len[b]) (device int64 / int32
+ * arrays, seq_len including the new token's row).  max_len (host value) sizes
+ * the split plan without a device read.
  * o [B, Hq, D]; lse [B, Hq] or NULL.
- * workspace: device scratch of yoco_cross_decode_workspace_size() bytes. */
+ * workspace: device scratch of yoco_cross_decode_workspace_size() bytes.
+ * Device-side range check: a sequence with seq_len < 1, seq_len > max_len,
+ * seq_start < 0 or seq_start + seq_len > cache_rows reads nothing; its o is 0
+ * and its lse -inf, the other sequences are computed, and the next
+ * yoco_get_device_status returns YOCO_ERR_INVALID.  No read ever leaves the
+ * cache's cache_rows rows. */
 yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_cache,
-                              const int64_t *seq_start, const int32_t *seq_len, int32_t B,
-                              int64_t max_len, void *o, float *lse, void *workspace,
+                              int64_t cache_rows, const int64_t *seq_start, const int32_t *seq_len,
+                              int32_t B, int64_t max_len, void *o, float *lse, void *workspace,
                               size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream);
 
 /* yoco_cross_decode for callers that cannot allocate device memory: a C host
@@ -153,13 +159,16 @@ yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_
  * (see yoco_cross_decode_workspace_size) returns YOCO_ERR_WORKSPACE and
  * launches nothing.  The first call on a device looks up the array's address
  * on that device (which must be current); make it before any stream capture.
+ * The address is kept for the life of the process and does not survive a
+ * cudaDeviceReset (or another teardown of the device's primary context) in
+ * the same process: do not call this entry point after one.
  * All calls on a device share the array and leave their partials in it;
  * nothing needs clearing between calls, but calls whose kernels overlap on
  * the GPU race on it, so serialise them. */
 yoco_status yoco_cross_decode_static(const void *q, const void *k_cache, const void *v_cache,
-                                     const int64_t *seq_start, const int32_t *seq_len, int32_t B,
-                                     int64_t max_len, void *o, float *lse,
-                                     const yoco_attn_cfg *cfg, cudaStream_t stream);
+                                     int64_t cache_rows, const int64_t *seq_start,
+                                     const int32_t *seq_len, int32_t B, int64_t max_len, void *o,
+                                     float *lse, const yoco_attn_cfg *cfg, cudaStream_t stream);
 
 /* General attention prefill over a key range that may start before the query
  * rows: query row i sits at position q_pos0 + i of the key buffer and sees
@@ -201,7 +210,8 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
  * Decode-time appends pass the new rows' indices, like yoco_kv_project_blend.
  *
  * yoco_cross_decode_i8: yoco_cross_decode over 8-bit caches (same q, o, lse,
- * sequence and workspace arguments; the workspace size is
+ * cache_rows, sequence and workspace arguments and the same device-side range
+ * check; cache_rows counts 8-bit rows; the workspace size is
  * yoco_cross_decode_workspace_size with the bf16 cfg).  Built for D = 128
  * and bf16 q / o; other shapes return YOCO_ERR_UNSUPPORTED.  The scores are
  * integer products of the K codes with q held per query head as 15-bit
@@ -211,9 +221,10 @@ yoco_status yoco_linear(const void *x, int64_t n, int32_t d_in, const void *w, i
 int64_t yoco_kv_i8_row_bytes(const yoco_attn_cfg *cfg);
 yoco_status yoco_kv_quantize_i8(const void *k, const void *v, int64_t n_tok, const int64_t *dst_rows, void *k_i8,
                                 void *v_i8, const yoco_attn_cfg *cfg, cudaStream_t stream);
-yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_i8, const int64_t *seq_start,
-                                 const int32_t *seq_len, int32_t B, int64_t max_len, void *o, float *lse,
-                                 void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream);
+yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_i8, int64_t cache_rows,
+                                 const int64_t *seq_start, const int32_t *seq_len, int32_t B, int64_t max_len,
+                                 void *o, float *lse, void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg,
+                                 cudaStream_t stream);
 
 /* Gated retention, the alternative self-decoder ("You Only Cache Once",
  * paperlayer summary, section 3 "Gated Retention" and Appendix B; podcast
@@ -254,6 +265,8 @@ yoco_status yoco_gret_decode(const void *q, const void *k, const void *v, const 
  *
  * kind YOCO_SCHEDULE_DECODE -- the split-KV plan of yoco_cross_decode for
  * B sequences with HOST arrays seq_start [B] and seq_len [B], and max_len.
+ * A sequence out of range (seq_len < 1, seq_len > max_len or seq_start < 0;
+ * the cache size is not an argument here) has no units, as in the kernels.
  * One record per unit, CTA by CTA, in processing order:
  *   {cta, b, split index, first cache row, tokens, pipeline stages}
  *
@@ -274,7 +287,9 @@ double yoco_cache_bytes(int32_t L_self, int32_t window, int64_t N, const yoco_at
 
 /* Synchronises the stream, then returns and clears the device status word:
  * YOCO_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call,
- * YOCO_ERR_CUDA if the stream reports an error, else YOCO_OK. */
+ * else YOCO_ERR_INVALID if a decode call met a sequence out of range (see
+ * yoco_cross_decode), else YOCO_ERR_CUDA if the stream reports an error,
+ * else YOCO_OK. */
 yoco_status yoco_get_device_status(cudaStream_t stream);
 
 /* Test-only, with no counterpart on the pages: launches one kernel that waits,
@@ -284,6 +299,13 @@ yoco_status yoco_get_device_status(cudaStream_t stream);
  * YOCO_ERR_TIMEOUT; nothing faults and the context stays usable.  Until the
  * status is read, the library's kernels exit at once (their first check). */
 yoco_status yoco_debug_wait_timeout_probe(cudaStream_t stream);
+
+/* Test-only, with no counterpart on the pages: y[i] = the polynomial 2^x[i]
+ * that the bf16 prefill kernels evaluate on the FMA pipe for a quarter of
+ * their softmax exponentials (Cody-Waite reduction, degree-3 minimax fit on
+ * [-1/2, 1/2], relative error <= 7.5e-5; inputs below -125, -inf included,
+ * give 2^-125 in place of 0).  x, y: device fp32 [n].  Asynchronous. */
+yoco_status yoco_debug_exp2_poly(const float *x, float *y, int64_t n, cudaStream_t stream);
 
 /* Static description of a status code. */
 const char *yoco_status_string(yoco_status s);

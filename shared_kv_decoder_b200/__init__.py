@@ -24,7 +24,7 @@ __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_p
            "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg",
            "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE", "gret_prefill", "gret_decode",
            "kv_i8_row_bytes", "kv_quantize_i8", "cross_decode_i8",
-           "attention_prefill"]
+           "attention_prefill", "debug_exp2_poly"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -73,19 +73,21 @@ def load():
         "yoco_swa_decode": (st, [vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, sz, cfgp, vp]),
         "yoco_cross_prefill": (st, [vp, vp, vp, i32, i64, i64, i64, vp, vp, cfgp, vp]),
         "yoco_attention_prefill": (st, [vp, vp, vp, i32, i64, i64, i64, i32, vp, vp, cfgp, vp]),
-        "yoco_cross_decode": (st, [vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_cross_decode": (st, [vp, vp, vp, i64, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_cross_decode_static": (st, [vp, vp, vp, i64, vp, vp, i32, i64, vp, vp, cfgp, vp]),
         "yoco_cross_decode_workspace_size": (sz, [i32, i64, cfgp]),
         "yoco_swa_decode_workspace_size": (sz, [i32, i32, cfgp]),
         "yoco_cache_bytes": (ctypes.c_double, [i32, i32, i64, cfgp]),
         "yoco_gret_prefill": (st, [vp, vp, vp, vp, i32, i64, f32, vp, vp, cfgp, vp]),
         "yoco_kv_i8_row_bytes": (i64, [cfgp]),
         "yoco_kv_quantize_i8": (st, [vp, vp, i64, vp, vp, vp, cfgp, vp]),
-        "yoco_cross_decode_i8": (st, [vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_cross_decode_i8": (st, [vp, vp, vp, i64, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
         "yoco_gret_decode": (st, [vp, vp, vp, vp, i32, f32, vp, vp, cfgp, vp]),
         "yoco_debug_tile_schedule": (st, [i32, cfgp, i32, i64, i64, i64, i32, vp, vp, i64, i32, vp,
                                           i64, ctypes.POINTER(ctypes.c_int64)]),
         "yoco_get_device_status": (st, [vp]),
         "yoco_debug_wait_timeout_probe": (st, [vp]),
+        "yoco_debug_exp2_poly": (st, [vp, vp, i64, vp]),
         "yoco_status_string": (ctypes.c_char_p, [st]),
         "yoco_version": (ctypes.c_char_p, []),
         "yoco_launch_count": (ctypes.c_uint64, []),
@@ -229,6 +231,8 @@ def cross_decode(q, k_cache, v_cache, seq_start, seq_len, max_len, workspace=Non
     L = load()
     B, Hq, D = q.shape
     Hkv = k_cache.shape[1]
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape")
     if workspace is None:
         workspace = torch.empty(cross_decode_workspace_size(B, max_len, Hq, Hkv, D, q.dtype),
                                 dtype=torch.uint8, device=q.device)
@@ -237,7 +241,7 @@ def cross_decode(q, k_cache, v_cache, seq_start, seq_len, max_len, workspace=Non
     lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if want_lse else None
     _dev(q, k_cache, v_cache, seq_start, seq_len, o, lse, workspace)
     cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
-    _check(L.yoco_cross_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_start),
+    _check(L.yoco_cross_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(seq_start),
                                _ptr(seq_len), B, int(max_len), _ptr(o), _ptr(lse),
                                _ptr(workspace), workspace.numel() * workspace.element_size(),
                                ctypes.byref(cfg), _stream()), "yoco_cross_decode")
@@ -350,7 +354,9 @@ def cross_decode_i8(q, k_i8, v_i8, Hkv, seq_start, seq_len, max_len, workspace=N
         n = L.yoco_cross_decode_workspace_size(B, int(max_len), ctypes.byref(cfg))
         workspace = torch.empty(max(int(n), 16), dtype=torch.uint8, device=q.device)
     _dev(q, k_i8, v_i8, seq_start, seq_len, o, lse, workspace)
-    _check(L.yoco_cross_decode_i8(_ptr(q), _ptr(k_i8), _ptr(v_i8), _ptr(seq_start), _ptr(seq_len), B,
+    if v_i8.shape != k_i8.shape:
+        raise ValueError("k_i8 and v_i8 must have the same shape")
+    _check(L.yoco_cross_decode_i8(_ptr(q), _ptr(k_i8), _ptr(v_i8), k_i8.shape[0], _ptr(seq_start), _ptr(seq_len), B,
                                   int(max_len), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(),
                                   ctypes.byref(cfg), _stream()), "yoco_cross_decode_i8")
     return (o, lse) if want_lse else o
@@ -370,3 +376,16 @@ def attention_prefill(q, k, v, q_pos0=0, window=0, o=None, want_lse=False, scale
     _check(L.yoco_attention_prefill(_ptr(q), _ptr(k), _ptr(v), B, Tq, Tkv, int(q_pos0), int(window), _ptr(o),
                                     _ptr(lse), ctypes.byref(cfg), _stream()), "yoco_attention_prefill")
     return (o, lse) if want_lse else o
+
+
+def debug_exp2_poly(x, y=None):
+    """Test-only: the prefill softmax's polynomial 2^x (the FMA-pipe half of its
+    exponentials) applied elementwise to an fp32 CUDA tensor."""
+    L = load()
+    if y is None:
+        y = torch.empty_like(x)
+    _dev(x, y)
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or y.numel() != x.numel():
+        raise ValueError("debug_exp2_poly takes fp32 tensors of one size")
+    _check(L.yoco_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream()), "yoco_debug_exp2_poly")
+    return y

@@ -24,6 +24,8 @@ namespace {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
 bool ok_opt(const void *p) { return p == nullptr || aligned16(p); }
+// The decode kernels address cache rows with 32-bit TMA coordinates.
+bool ok_cache_rows(int64_t rows) { return rows >= 1 && rows <= INT32_MAX; }
 
 yoco_status check_cfg(const yoco_attn_cfg *cfg) {
     if (!cfg) return YOCO_ERR_INVALID;
@@ -200,12 +202,12 @@ size_t yoco_swa_decode_workspace_size(int32_t B, int32_t window, const yoco_attn
 }
 
 yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_cache,
-                              const int64_t *seq_start, const int32_t *seq_len, int32_t B,
-                              int64_t max_len, void *o, float *lse, void *workspace,
+                              int64_t cache_rows, const int64_t *seq_start, const int32_t *seq_len,
+                              int32_t B, int64_t max_len, void *o, float *lse, void *workspace,
                               size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream) {
     yoco_status st = check_cfg(cfg);
     if (st != YOCO_OK) return st;
-    if (B < 0 || max_len < 1) return YOCO_ERR_INVALID;
+    if (B < 0 || max_len < 1 || !ok_cache_rows(cache_rows)) return YOCO_ERR_INVALID;
     if (B == 0) return YOCO_OK;
     if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_start) ||
         !seq_len || !ok_ptr(o) || !ok_opt(lse))
@@ -217,6 +219,7 @@ yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_
     DecodeArgs a;
     a.q = q; a.k = k_cache; a.v = v_cache; a.seq_start = seq_start; a.seq_len = seq_len;
     a.slot_pos = nullptr; a.pos = nullptr; a.window = 0;
+    a.cache_rows = cache_rows; a.max_len = max_len;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = lse; a.ws = workspace;
     return from_cuda(launch_decode(a, pl, stream));
@@ -243,6 +246,7 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     DecodeArgs a;
     a.q = q; a.k = ring_k; a.v = ring_v; a.seq_start = nullptr; a.seq_len = nullptr;
     a.slot_pos = slot_pos; a.pos = pos; a.window = window;
+    a.cache_rows = (int64_t)B * window; a.max_len = window;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = nullptr; a.ws = workspace;
     return from_cuda(launch_decode(a, pl, stream));
@@ -263,12 +267,13 @@ yoco_status yoco_kv_quantize_i8(const void *k, const void *v, int64_t n_tok, con
     return from_cuda(launch_kv_quantize_i8(k, v, n_tok, cfg->Hkv, cfg->D, cfg->dtype, dst_rows, k_i8, v_i8, stream));
 }
 
-yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_i8, const int64_t *seq_start,
-                                 const int32_t *seq_len, int32_t B, int64_t max_len, void *o, float *lse,
-                                 void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream) {
+yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_i8, int64_t cache_rows,
+                                 const int64_t *seq_start, const int32_t *seq_len, int32_t B, int64_t max_len,
+                                 void *o, float *lse, void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg,
+                                 cudaStream_t stream) {
     yoco_status st = check_cfg(cfg);
     if (st != YOCO_OK) return st;
-    if (B < 0 || max_len < 1) return YOCO_ERR_INVALID;
+    if (B < 0 || max_len < 1 || !ok_cache_rows(cache_rows)) return YOCO_ERR_INVALID;
     if (B == 0) return YOCO_OK;
     if (!ok_ptr(q) || !ok_ptr(k_i8) || !ok_ptr(v_i8) || !ok_ptr(seq_start) || !seq_len || !ok_ptr(o) || !ok_opt(lse))
         return YOCO_ERR_INVALID;
@@ -279,6 +284,7 @@ yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_
     DecodeArgs a;
     a.q = q; a.k = k_i8; a.v = v_i8; a.seq_start = seq_start; a.seq_len = seq_len;
     a.slot_pos = nullptr; a.pos = nullptr; a.window = 0;
+    a.cache_rows = cache_rows; a.max_len = max_len;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = lse; a.ws = workspace;
     return from_cuda(launch_decode_i8(a, pl, stream));
@@ -347,6 +353,8 @@ yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int
         if (n_work > INT32_MAX / 2) return YOCO_ERR_UNSUPPORTED;
         s.n_qtiles = (int32_t)n_qtiles;
         const int grid = (int)(n_work < sms ? n_work : sms);
+        s.band = sched::prefill_band(grid, (cfg->Hq / cfg->Hkv) / heads,
+                                     (int64_t)B * Tkv * cfg->Hkv * cfg->D * dtype_bytes(cfg->dtype) * 2);
         for (int c = 0; c < grid; ++c)
             for (int r = 0;; ++r) {
                 const int w = sched::prefill_work_index(r, c, grid);
@@ -362,16 +370,22 @@ yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int
         if (!make_decode_plan(B, max_len, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl))
             return YOCO_ERR_UNSUPPORTED;
         // the compact unit list, sequence by sequence, as the kernel enumerates it
+        // (the cache's row count is not an argument here: a sequence is in
+        // range when 1 <= seq_len <= max_len and seq_start >= 0)
+        auto units = [&](int b) {
+            return sched::decode_seq_ok(seq_start[b], seq_len[b], max_len, INT64_MAX)
+                       ? sched::decode_units(seq_len[b], pl.split, pl.n_split)
+                       : 0;
+        };
         int64_t total = 0;
-        for (int b = 0; b < B; ++b) total += sched::decode_units(seq_len[b], pl.split, pl.n_split);
+        for (int b = 0; b < B; ++b) total += units(b);
         const int64_t slots = (int64_t)B * pl.n_split;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(slots, sms));
         for (int c = 0; c < grid; ++c) {
             int b = 0;
             int64_t before = 0;  // units of sequences < b
             for (int64_t u = c; u < total; u += grid) {
-                while (before + sched::decode_units(seq_len[b], pl.split, pl.n_split) <= u)
-                    before += sched::decode_units(seq_len[b++], pl.split, pl.n_split);
+                while (before + units(b) <= u) before += units(b++);
                 const int64_t sidx = u - before;
                 const int64_t t0 = sidx * pl.split;
                 const int64_t n_tok = std::min<int64_t>(pl.split, seq_len[b] - t0);
@@ -401,7 +415,8 @@ yoco_status yoco_get_device_status(cudaStream_t stream) {
     const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc() |
                            read_and_clear_status_prefill_pair() | read_and_clear_status_project_tc() |
                            read_and_clear_status_gret_tc();
-    if (s) return YOCO_ERR_TIMEOUT;
+    if (s & 1u) return YOCO_ERR_TIMEOUT;
+    if (s & 2u) return YOCO_ERR_INVALID;
     return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;
 }
 

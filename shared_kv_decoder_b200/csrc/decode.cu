@@ -36,7 +36,13 @@
 
 namespace yoco {
 
+// Status word of this translation unit: bit 0 (kStatusTimeout) records a
+// bounded wait that gave up, bit 1 (kStatusBadSequence) a decode sequence
+// whose seq_start / seq_len were out of range.  Only a timeout makes later
+// kernels exit at once; a bad sequence affects only itself.
 static __device__ unsigned int g_status_decode;
+constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusBadSequence = 2u;
 
 constexpr int kConsumerWarps = 8;
 constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);
@@ -55,6 +61,7 @@ struct DecodeKParams {
     const int64_t *pos;
     int32_t window;
     int32_t B, Hkv, Hq;
+    int64_t cache_rows, max_len;   // rows of the cache buffers; longest allowed sequence
     int64_t stage_tokens, split, n_split;
     int32_t sub, stages;
     float scale_log2;
@@ -71,11 +78,14 @@ static __device__ bool find_unit(const DecodeKParams &p, int64_t u, int *b_out, 
     int64_t base = 0;
     for (int b0 = 0; b0 < p.B; b0 += 32) {
         const int b = b0 + lane;
-        int64_t len = 0;
-        if (b < p.B) len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
-        // never more units than the workspace plan holds (lengths above max_len
-        // are a caller error; their tail is not read)
-        const int64_t cnt = sched::decode_units(len, p.split, p.n_split);
+        int64_t cnt = 0;
+        if (b < p.B) {
+            // a sequence whose length or rows are out of range has no units
+            // (the merge kernel reports it); ring slots are always in range
+            const int64_t len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
+            if (!p.seq_len || sched::decode_seq_ok(p.seq_start[b], len, p.max_len, p.cache_rows))
+                cnt = sched::decode_units(len, p.split, p.n_split);
+        }
         int64_t incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -115,7 +125,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
     constexpr int DPL = CPL * EPC;            // dims per lane
     static_assert(CPL >= 1 && CPR % kLanesPerTok == 0, "head dim too small for the lane layout");
 
-    if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
+    if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     extern __shared__ __align__(128) unsigned char smem[];
     const int64_t row_elems = (int64_t)p.Hkv * D;
     const size_t half_bytes = (size_t)kRowsPerStage * D * sizeof(T);
@@ -369,7 +379,7 @@ template <int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeKParams p) {
-    if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
+    if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     static_assert(G >= 1 && G <= 8, "query heads per KV head");
     constexpr int KB = D / 64;                       // 64-column blocks per head row
     constexpr uint32_t kBox = kRowsPerStage * 128;   // one box: 128 rows of 128 bytes
@@ -663,7 +673,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const DecodeI8Params pi) {
     static_assert(G >= 1 && G <= 8, "the query heads of a group are the 8 columns of an MMA");
-    if (*(volatile unsigned int *)&g_status_decode) return;  // an earlier CTA timed out
+    if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     constexpr int D = 128;
     constexpr uint32_t kBox = kRowsPerStage * 128;  // one code box: 128 rows of 128 bytes
     const DecodeKParams &p = pi.k;
@@ -1000,15 +1010,20 @@ constexpr int kMergeWarps = 8;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(
-    const float *ws_o, const float *ws_ml, const int32_t *seq_len, int32_t window, int32_t B, int32_t Hq,
-    int64_t split, int64_t n_split, int32_t sub, T *o, float *lse) {
+    const float *ws_o, const float *ws_ml, const int64_t *seq_start, const int32_t *seq_len, int32_t window,
+    int32_t B, int32_t Hq, int64_t max_len, int64_t cache_rows, int64_t split, int64_t n_split, int32_t sub,
+    T *o, float *lse) {
     constexpr int DPL = D / 32;
     __shared__ float s_m[kMergeWarps], s_l[kMergeWarps];
     __shared__ float s_acc[kMergeWarps][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = (int)(blockIdx.x / Hq), h = (int)(blockIdx.x % Hq);
     const int64_t len = seq_len ? (int64_t)seq_len[b] : (int64_t)window;
-    const int64_t n_s = sched::decode_units(len, split, n_split);
+    // the split kernel gave an out-of-range sequence no units; its output
+    // becomes 0 (lse -inf) and the status word records it once
+    const bool ok = !seq_len || sched::decode_seq_ok(seq_start[b], len, max_len, cache_rows);
+    if (!ok && h == 0 && threadIdx.x == 0) atomicOr(&g_status_decode, kStatusBadSequence);
+    const int64_t n_s = ok ? sched::decode_units(len, split, n_split) : 0;
     const int64_t n_e = n_s * sub;
     const int64_t e0 = (int64_t)b * n_split * sub;
 
@@ -1103,13 +1118,13 @@ int device_sm_count() {
 }
 
 // TMA view of a packed cache [rows, Hkv, D]: dimensions {D, token, head, 1},
-// box {64, stage_tokens, Hkv, 1}.  The token extent only has to cover every
-// row a full stage reads (the kernel never asks for a box past a sequence's
-// end); it is set to a 1 TiB span, beyond any device's memory.
-static bool make_cache_map(CUtensorMap *m, const void *cache, int Hkv, int D, int64_t stage_tokens) {
+// box {64, stage_tokens, Hkv, 1}.  The token extent is the caller's cache_rows,
+// so a box can never read past the allocation (the kernel only asks for
+// boxes inside a sequence whose rows it has checked against cache_rows).
+static bool make_cache_map(CUtensorMap *m, const void *cache, int64_t cache_rows, int Hkv, int D,
+                           int64_t stage_tokens) {
     const uint64_t row_bytes = (uint64_t)Hkv * D * 2;
-    const uint64_t rows = std::min<uint64_t>((uint64_t)INT32_MAX, (1ull << 40) / row_bytes);
-    const uint64_t dims[4] = {(uint64_t)D, rows, (uint64_t)Hkv, 1};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)cache_rows, (uint64_t)Hkv, 1};
     const uint64_t strides[3] = {row_bytes, (uint64_t)D * 2, row_bytes};
     const uint32_t box[4] = {64, (uint32_t)stage_tokens, (uint32_t)Hkv, 1};
     return encode_bf16_map_4d(m, cache, dims, strides, box);
@@ -1119,8 +1134,8 @@ template <int D, int G>
 static cudaError_t launch_decode_tma(const DecodeArgs &a, const DecodePlan &pl, const DecodeKParams &p,
                                      int grid, cudaStream_t st) {
     CUtensorMap mk, mv;
-    if (!make_cache_map(&mk, a.k, a.Hkv, D, p.stage_tokens) ||
-        !make_cache_map(&mv, a.v, a.Hkv, D, p.stage_tokens))
+    if (!make_cache_map(&mk, a.k, a.cache_rows, a.Hkv, D, p.stage_tokens) ||
+        !make_cache_map(&mv, a.v, a.cache_rows, a.Hkv, D, p.stage_tokens))
         return cudaErrorNotSupported;
     auto kern = decode_tma_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
@@ -1136,6 +1151,7 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
     p.seq_start = a.seq_start; p.seq_len = a.seq_len;
     p.slot_pos = a.slot_pos; p.pos = a.pos; p.window = a.window;
     p.B = a.B; p.Hkv = a.Hkv; p.Hq = a.Hq;
+    p.cache_rows = a.cache_rows; p.max_len = a.max_len;
     p.stage_tokens = pl.stage_tokens; p.split = pl.split; p.n_split = pl.n_split;
     p.sub = pl.sub; p.stages = pl.stages;
     p.scale_log2 = a.scale * kLog2e;
@@ -1157,9 +1173,9 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
     note_launches(2);
     if (e != cudaSuccess) return e;
     const int mgrid = (int)((int64_t)a.B * a.Hq);
-    decode_merge_kernel<T, D><<<mgrid, 32 * kMergeWarps, 0, st>>>(p.ws_o, p.ws_ml, a.seq_len, a.window, a.B,
-                                                     a.Hq, pl.split, pl.n_split, pl.sub,
-                                                     static_cast<T *>(a.o), a.lse);
+    decode_merge_kernel<T, D><<<mgrid, 32 * kMergeWarps, 0, st>>>(
+        p.ws_o, p.ws_ml, a.seq_start, a.seq_len, a.window, a.B, a.Hq, a.max_len, a.cache_rows, pl.split,
+        pl.n_split, pl.sub, static_cast<T *>(a.o), a.lse);
     return cudaGetLastError();
 }
 
@@ -1191,9 +1207,10 @@ cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &pl, cudaStream_
 // stride row_bytes, head stride 128), box {128, stage_tokens, Hkv, 1} with the
 // 128-byte swizzle; the scales as {scale_bytes, token, 1, 1} starting at the
 // row's scale offset, box {scale_bytes, stage_tokens, 1, 1}.
-static bool make_i8_maps(CUtensorMap *codes, CUtensorMap *scales, const void *cache, int Hkv, int64_t ST) {
+static bool make_i8_maps(CUtensorMap *codes, CUtensorMap *scales, const void *cache, int64_t cache_rows, int Hkv,
+                         int64_t ST) {
     const uint64_t rb = (uint64_t)i8_row_bytes(Hkv, 128);
-    const uint64_t rows = std::min<uint64_t>((uint64_t)INT32_MAX, (1ull << 40) / rb);
+    const uint64_t rows = (uint64_t)cache_rows;
     const uint64_t dims[4] = {128, rows, (uint64_t)Hkv, 1};
     const uint64_t strides[3] = {rb, 128, rb};
     const uint32_t box[4] = {128, (uint32_t)ST, (uint32_t)Hkv, 1};
@@ -1208,7 +1225,8 @@ static bool make_i8_maps(CUtensorMap *codes, CUtensorMap *scales, const void *ca
 template <int G>
 static cudaError_t launch_decode_i8_g(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t st) {
     CUtensorMap mk, mks, mv, mvs;
-    if (!make_i8_maps(&mk, &mks, a.k, a.Hkv, pl.stage_tokens) || !make_i8_maps(&mv, &mvs, a.v, a.Hkv, pl.stage_tokens))
+    if (!make_i8_maps(&mk, &mks, a.k, a.cache_rows, a.Hkv, pl.stage_tokens) ||
+        !make_i8_maps(&mv, &mvs, a.v, a.cache_rows, a.Hkv, pl.stage_tokens))
         return cudaErrorNotSupported;
     DecodeI8Params pi;
     DecodeKParams &p = pi.k;
@@ -1216,6 +1234,7 @@ static cudaError_t launch_decode_i8_g(const DecodeArgs &a, const DecodePlan &pl,
     p.seq_start = a.seq_start; p.seq_len = a.seq_len;
     p.slot_pos = a.slot_pos; p.pos = a.pos; p.window = a.window;
     p.B = a.B; p.Hkv = a.Hkv; p.Hq = a.Hq;
+    p.cache_rows = a.cache_rows; p.max_len = a.max_len;
     p.stage_tokens = pl.stage_tokens; p.split = pl.split; p.n_split = pl.n_split;
     p.sub = pl.sub; p.stages = kI8Stages;
     p.scale_log2 = a.scale * kLog2e;
@@ -1238,8 +1257,8 @@ static cudaError_t launch_decode_i8_g(const DecodeArgs &a, const DecodePlan &pl,
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_merge_kernel<__nv_bfloat16, 128><<<(int)((int64_t)a.B * a.Hq), 32 * kMergeWarps, 0, st>>>(
-        p.ws_o, p.ws_ml, a.seq_len, a.window, a.B, a.Hq, pl.split, pl.n_split, pl.sub,
-        static_cast<__nv_bfloat16 *>(a.o), a.lse);
+        p.ws_o, p.ws_ml, a.seq_start, a.seq_len, a.window, a.B, a.Hq, a.max_len, a.cache_rows, pl.split,
+        pl.n_split, pl.sub, static_cast<__nv_bfloat16 *>(a.o), a.lse);
     return cudaGetLastError();
 }
 

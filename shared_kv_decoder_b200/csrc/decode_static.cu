@@ -15,7 +15,10 @@
 //    nothing (yoco_cross_decode_workspace_size tells the need in advance).
 //  * Set-up: the first call on a device looks up the array's device address
 //    on that device (the device must be current, as for any launch on its
-//    streams).  Make that first call before any stream capture.
+//    streams).  Make that first call before any stream capture.  The address
+//    is kept for the life of the process: it does not survive a
+//    cudaDeviceReset (or any other teardown of the device's primary context)
+//    in the same process, after which this entry point must not be called.
 //  * Sharing: every call on a device uses the same array and leaves its
 //    contents behind.  Nothing in it needs to start at zero: each call writes
 //    every partial it later reads.  Calls whose kernels overlap on the GPU
@@ -55,17 +58,18 @@ cudaError_t scratch_on_current_device(void **out) {
 }  // namespace
 
 extern "C" yoco_status yoco_cross_decode_static(const void *q, const void *k_cache,
-                                                const void *v_cache, const int64_t *seq_start,
-                                                const int32_t *seq_len, int32_t B, int64_t max_len,
-                                                void *o, float *lse, const yoco_attn_cfg *cfg,
-                                                cudaStream_t stream) {
-    const size_t need = yoco_cross_decode_workspace_size(B, max_len, cfg);
-    if (need == 0)  // bad arguments: report them exactly as yoco_cross_decode does
-        return yoco_cross_decode(q, k_cache, v_cache, seq_start, seq_len, B, max_len, o, lse,
-                                 nullptr, 0, cfg, stream);
-    if (need > kStaticScratchBytes) return YOCO_ERR_WORKSPACE;
+                                                const void *v_cache, int64_t cache_rows,
+                                                const int64_t *seq_start, const int32_t *seq_len,
+                                                int32_t B, int64_t max_len, void *o, float *lse,
+                                                const yoco_attn_cfg *cfg, cudaStream_t stream) {
+    // every argument check of yoco_cross_decode first: without a workspace it
+    // launches nothing and answers YOCO_ERR_WORKSPACE only when all else is valid
+    const yoco_status st = yoco_cross_decode(q, k_cache, v_cache, cache_rows, seq_start, seq_len, B,
+                                             max_len, o, lse, nullptr, 0, cfg, stream);
+    if (st != YOCO_ERR_WORKSPACE) return st;
+    if (yoco_cross_decode_workspace_size(B, max_len, cfg) > kStaticScratchBytes) return YOCO_ERR_WORKSPACE;
     void *scratch = nullptr;
     if (scratch_on_current_device(&scratch) != cudaSuccess) return YOCO_ERR_CUDA;
-    return yoco_cross_decode(q, k_cache, v_cache, seq_start, seq_len, B, max_len, o, lse, scratch,
-                             kStaticScratchBytes, cfg, stream);
+    return yoco_cross_decode(q, k_cache, v_cache, cache_rows, seq_start, seq_len, B, max_len, o,
+                             lse, scratch, kStaticScratchBytes, cfg, stream);
 }

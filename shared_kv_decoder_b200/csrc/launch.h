@@ -41,6 +41,8 @@ struct DecodeArgs {
     const int32_t *slot_pos;   // ring only: [B, window]
     const int64_t *pos;        // ring only: [B]
     int32_t window;            // ring only
+    int64_t cache_rows;        // rows of the K and V cache buffers (ring: B * window)
+    int64_t max_len;           // longest allowed sequence (the plan's max_len; ring: window)
     int32_t B, Hq, Hkv, D, dtype;
     float scale;
     void *o;       // [B, Hq, D]
@@ -121,7 +123,9 @@ cudaError_t launch_gret_prefill_tc(const GretArgs &a, cudaStream_t s);
 // Test-only: a kernel whose bounded wait is never satisfied (see decode.cu).
 cudaError_t launch_wait_timeout_probe(cudaStream_t s);
 
-// Device status words of the translation units that hold bounded waits.
+// Device status words of the translation units that hold bounded waits:
+// bit 0 = a bounded wait gave up; bit 1 (decode only) = a decode sequence's
+// seq_start / seq_len were out of range.
 unsigned int read_and_clear_status_decode();
 unsigned int read_and_clear_status_prefill_tc();
 unsigned int read_and_clear_status_prefill_pair();

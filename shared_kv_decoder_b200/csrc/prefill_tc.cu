@@ -443,11 +443,12 @@ cudaError_t launch_tc_d(const PrefillArgs &a, cudaStream_t st) {
     if (n_work > INT32_MAX / 2) return cudaErrorNotSupported;
     p.s.n_qtiles = (int)n_qtiles;
     p.n_work = (int)n_work;
+    const int grid = (int)std::min<int64_t>(n_work, device_sm_count());
+    p.s.band = sched::prefill_band(grid, a.Hq / a.Hkv, (int64_t)a.B * a.Tkv * a.Hkv * D * 2 * 2);
     auto kern = attn_prefill_tc_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Smem<D>::ALLOC);
     if (e != cudaSuccess) return e;
-    const int grid = (int)std::min<int64_t>(n_work, device_sm_count());
     note_launches(1);
     kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, p);
     return cudaGetLastError();

@@ -22,8 +22,18 @@ constexpr int kPrefillBN = 128;  // keys per KV tile
 YOCO_HD int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 YOCO_HD int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
-// Prefill work tiles are numbered heaviest causal tile first: all (head,
-// batch) pairs of the last query tile, then of the one before, and so on.
+// Prefill work order.  A K/V "stream" is one batch entry's keys and values of
+// one KV head; the work tiles of a query tile and stream are its query heads
+// (or head pairs).  Work tiles are numbered in bands of `band` query tiles,
+// the band of the last (heaviest causal) query tiles first; inside a band,
+// stream by stream; inside a stream, query tile descending, then the heads.
+// The host sets band so that one stream's share of a band holds about as many
+// work tiles as the persistent grid has CTAs: each round of the grid then
+// reads ONE stream, and CTAs that drift a round apart read at most a few, so
+// the K/V tiles they stream stay in L2 instead of the whole K/V of every
+// stream being live at once.  Consecutive bands are each lighter than the
+// last, and within a band every stream repeats the same lengths, so the
+// snake dealing below still balances the CTAs' totals.
 struct PrefillWork {
     int qt, h, b, g;              // query tile, query head, batch, KV head
     int64_t i0;                   // first query row
@@ -36,7 +46,21 @@ struct PrefillShape {
     int64_t Tq, Tkv, q_pos0;
     int32_t window;               // 0: causal
     int32_t n_qtiles;
+    int32_t band;                 // query tiles per band of the work order (>= 1)
 };
+
+// K/V bytes (all streams) up to which the whole K/V stays in L2 anyway; then
+// the band is one query tile, which is the plain heaviest-first order (all
+// streams' work tiles of the last query tile, then of the one before, ...).
+constexpr int64_t kPrefillBandMinKVBytes = (int64_t)32 << 20;
+
+// Query tiles per band for a grid of `grid` CTAs, `per` work tiles per (query
+// tile, stream) and kv_bytes of K and V over all streams.
+YOCO_HD int32_t prefill_band(int grid, int per, int64_t kv_bytes) {
+    if (kv_bytes <= kPrefillBandMinKVBytes) return 1;
+    const int b = per > 0 ? grid / per : 1;
+    return b > 0 ? b : 1;
+}
 
 // The KV range of query tile qt of (batch b, query head h).
 YOCO_HD PrefillWork prefill_work_at(const PrefillShape &s, int qt, int h, int b) {
@@ -57,18 +81,32 @@ YOCO_HD PrefillWork prefill_work_at(const PrefillShape &s, int qt, int h, int b)
     return x;
 }
 
-// One query head per work tile (any group size).
+// Work tile w of the banded order when each (query tile, stream) has `per`
+// work tiles of `heads` consecutive query heads.
+YOCO_HD PrefillWork prefill_work_banded(const PrefillShape &s, int w, int per, int heads) {
+    const int streams = s.B * s.Hkv;
+    const int64_t band_works = (int64_t)s.band * streams * per;
+    const int j = (int)(w / band_works);
+    const int64_t off = w - (int64_t)j * band_works;
+    const int nb = (int)min64(s.band, (int64_t)s.n_qtiles - (int64_t)j * s.band);
+    const int64_t stream_works = (int64_t)nb * per;
+    const int stream = (int)(off / stream_works);
+    const int rem = (int)(off - (int64_t)stream * stream_works);
+    const int qt = s.n_qtiles - 1 - (j * s.band + rem / per);
+    const int b = stream / s.Hkv, g = stream - b * s.Hkv;
+    return prefill_work_at(s, qt, g * (s.Hq / s.Hkv) + (rem % per) * heads, b);
+}
+
+// One query head per work tile (any group size): n_work = n_qtiles * Hq * B.
 YOCO_HD PrefillWork prefill_work(const PrefillShape &s, int w) {
-    const int per = s.Hq * s.B;
-    return prefill_work_at(s, s.n_qtiles - 1 - w / per, (w % per) % s.Hq, (w % per) / s.Hq);
+    return prefill_work_banded(s, w, s.Hq / s.Hkv, 1);
 }
 
 // Two query heads per work tile, 2hp and 2hp + 1, which share their KV head
 // when the group size Hq / Hkv is even: n_work = n_qtiles * (Hq / 2) * B.
 // The returned h is the first head of the pair.
 YOCO_HD PrefillWork prefill_pair_work(const PrefillShape &s, int w) {
-    const int hp = s.Hq / 2, per = hp * s.B;
-    return prefill_work_at(s, s.n_qtiles - 1 - w / per, 2 * ((w % per) % hp), (w % per) / hp);
+    return prefill_work_banded(s, w, s.Hq / s.Hkv / 2, 2);
 }
 
 // The paired kernel serves bf16 shapes whose group size is even.
@@ -91,6 +129,15 @@ YOCO_HD bool prefill_tile_masked(const PrefillShape &s, const PrefillWork &x, in
 // ranges of split tokens, never more than the n_split the workspace holds.
 YOCO_HD int64_t decode_units(int64_t len, int64_t split, int64_t n_split) {
     return len > 0 ? min64((len + split - 1) / split, n_split) : 0;
+}
+
+// A decode sequence's arguments are in range when 1 <= len <= max_len (the
+// length the split plan was sized for) and its rows [start, start + len) lie
+// inside the cache's rows [0, cache_rows).  A sequence out of range gets no
+// units: it reads nothing, its output is 0 and its lse -inf, and the kernels
+// report it through the status word.
+YOCO_HD bool decode_seq_ok(int64_t start, int64_t len, int64_t max_len, int64_t cache_rows) {
+    return len >= 1 && len <= max_len && start >= 0 && start <= cache_rows - len;
 }
 
 }  // namespace sched

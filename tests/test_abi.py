@@ -73,10 +73,19 @@ def test_bad_arguments_rejected_before_launch():
     # window < 1, partial ring arguments
     assert L.yoco_swa_prefill(FAKE, FAKE, FAKE, 1, 64, 0, FAKE, None, None, None, None, b, None) == yoco.ERR_INVALID
     assert L.yoco_swa_prefill(FAKE, FAKE, FAKE, 1, 64, 8, FAKE, None, FAKE, None, None, b, None) == yoco.ERR_INVALID
-    # decode: max_len < 1, workspace missing / too small
-    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, FAKE, None, FAKE, 1 << 30, b, None) == yoco.ERR_INVALID
-    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 1000, FAKE, None, None, 0, b, None) == yoco.ERR_WORKSPACE
-    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 1000, FAKE, None, FAKE, 16, b, None) == yoco.ERR_WORKSPACE
+    # decode: max_len < 1, cache_rows out of [1, 2^31 - 1], workspace missing / too small
+    R = 4096
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, R, FAKE, FAKE, 2, 0, FAKE, None, FAKE, 1 << 30, b, None) == yoco.ERR_INVALID
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 2, 1000, FAKE, None, FAKE, 1 << 30, b, None) == yoco.ERR_INVALID
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, 1 << 31, FAKE, FAKE, 2, 1000, FAKE, None, FAKE, 1 << 30, b,
+                               None) == yoco.ERR_INVALID
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, R, FAKE, FAKE, 2, 1000, FAKE, None, None, 0, b, None) == yoco.ERR_WORKSPACE
+    assert L.yoco_cross_decode(FAKE, FAKE, FAKE, R, FAKE, FAKE, 2, 1000, FAKE, None, FAKE, 16, b, None) == yoco.ERR_WORKSPACE
+    assert L.yoco_cross_decode_static(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 2, 1000, FAKE, None, b, None) == yoco.ERR_INVALID
+    # test-only exp2 probe: negative size, null pointers
+    assert L.yoco_debug_exp2_poly(FAKE, FAKE, -1, None) == yoco.ERR_INVALID
+    assert L.yoco_debug_exp2_poly(None, FAKE, 8, None) == yoco.ERR_INVALID
+    assert L.yoco_debug_exp2_poly(FAKE, FAKE, 0, None) == yoco.OK
     # projection: bad eps
     assert L.yoco_kv_project_blend(FAKE, 4, 64, FAKE, 1, 0.0, None, None, 0.0, 0.0, None, FAKE, FAKE, b, None) == yoco.ERR_INVALID
     # empty inputs are a successful no-op (nothing launched)
@@ -112,10 +121,13 @@ def test_i8_cache_arguments_rejected_before_launch():
     assert L.yoco_kv_i8_row_bytes(b) == 8 * 128 + 32
     assert L.yoco_kv_i8_row_bytes(ctypes.byref(_cfg(Hq=8, Hkv=1))) == 128 + 16
     # the 8-bit decode is built for D = 128 and bf16
-    assert L.yoco_cross_decode_i8(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, FAKE, None, FAKE, 1 << 30,
+    R = 4096
+    assert L.yoco_cross_decode_i8(FAKE, FAKE, FAKE, R, FAKE, FAKE, 2, 100, FAKE, None, FAKE, 1 << 30,
                                   ctypes.byref(_cfg(D=64)), None) == yoco.ERR_UNSUPPORTED
-    assert L.yoco_cross_decode_i8(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, FAKE, None, None, 0, b, None) == yoco.ERR_WORKSPACE
-    assert L.yoco_cross_decode_i8(FAKE, MISALIGNED, FAKE, FAKE, FAKE, 2, 100, FAKE, None, FAKE, 1 << 30, b,
+    assert L.yoco_cross_decode_i8(FAKE, FAKE, FAKE, R, FAKE, FAKE, 2, 100, FAKE, None, None, 0, b, None) == yoco.ERR_WORKSPACE
+    assert L.yoco_cross_decode_i8(FAKE, MISALIGNED, FAKE, R, FAKE, FAKE, 2, 100, FAKE, None, FAKE, 1 << 30, b,
+                                  None) == yoco.ERR_INVALID
+    assert L.yoco_cross_decode_i8(FAKE, FAKE, FAKE, -1, FAKE, FAKE, 2, 100, FAKE, None, FAKE, 1 << 30, b,
                                   None) == yoco.ERR_INVALID
     assert L.yoco_kv_quantize_i8(FAKE, FAKE, -1, None, FAKE, FAKE, b, None) == yoco.ERR_INVALID
     assert L.yoco_kv_quantize_i8(FAKE, FAKE, 0, None, FAKE, FAKE, b, None) == yoco.OK

@@ -67,3 +67,57 @@ def test_hot_calls_capture_into_a_cuda_graph(cuda_lib):
     torch.cuda.synchronize()
     assert torch.equal(od, ref_d) and torch.equal(op, ref_p)
     g.reset()
+
+
+def test_out_of_range_sequences_read_nothing_and_are_reported(cuda_lib):
+    # A packed cache of R rows and five sequences: one in range, and four whose
+    # arguments are not (length above max_len, rows past the cache's end, a
+    # negative start, length 0).  The kernels' range check gives the four no
+    # work: each output is 0 with lse -inf, the in-range sequence is exact, and
+    # the status word reports the bad arguments once, without a fault.
+    Hq, Hkv, D, R, max_len = 8, 2, 128, 5000, 3000
+    kc = wl.normal((R, Hkv, D), 4300, BF, "cuda")
+    vc = wl.normal((R, Hkv, D), 4301, BF, "cuda")
+    starts = [100, 0, 4000, -8, 50]
+    lens = [2900, 3001, 1001, 64, 0]
+    B = len(lens)
+    q = wl.normal((B, Hq, D), 4302, BF, "cuda")
+    ss = torch.tensor(starts, dtype=torch.int64, device="cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    assert cuda_lib.device_status() == cuda_lib.OK
+    o, lse = cuda_lib.cross_decode(q, kc, vc, ss, sl, max_len, want_lse=True)
+    assert cuda_lib.device_status() == cuda_lib.ERR_INVALID
+    assert cuda_lib.device_status() == cuda_lib.OK               # cleared by the read
+    ro, rlse = oracle.cross_decode(q[:1].cpu(), kc.cpu(), vc.cpu(), starts[:1], lens[:1])
+    assert_close(o[:1], ro, BF, "in-range sequence")
+    assert_close(lse[:1], rlse, BF, "in-range lse", max_abs=1e-3, rel_l2=1e-4)
+    assert torch.all(o[1:] == 0)
+    assert torch.all(torch.isneginf(lse[1:]))
+    # the same plan over the 8-bit cache
+    kq, vq = cuda_lib.kv_quantize_i8(kc, vc)
+    o8 = cuda_lib.cross_decode_i8(q, kq, vq, Hkv, ss, sl, max_len)
+    assert cuda_lib.device_status() == cuda_lib.ERR_INVALID
+    assert torch.all(o8[1:] == 0)
+    # a call after the report runs normally
+    o2 = cuda_lib.cross_decode(q[:1].contiguous(), kc, vc, ss[:1].contiguous(), sl[:1].contiguous(), max_len)
+    assert cuda_lib.device_status() == cuda_lib.OK
+    assert_close(o2, ro, BF, "decode after the report")
+
+
+def test_polynomial_exp2_within_its_bound(cuda_lib):
+    # The prefill kernels take a quarter of their softmax exponentials from a
+    # degree-3 polynomial (Cody-Waite reduction + minimax fit).  Over its
+    # input range the relative error against 2^x stays within 7.5e-5; inputs
+    # below -125 (and -inf, a masked score) give 2^-125 instead of 0, which is
+    # ~1e-38 of the row's largest weight, below any fp32 sum's resolution.
+    x = np.concatenate([np.linspace(-125.0, 9.0, 2_000_001),
+                        np.array([0.0, -0.5, 0.5, -1.0, 1.0, 8.0, -124.5, -125.0])])
+    xt = torch.tensor(x, dtype=torch.float32, device="cuda")
+    y = cuda_lib.debug_exp2_poly(xt).cpu().double().numpy()
+    ref = np.exp2(xt.cpu().double().numpy())
+    rel = np.abs(y / ref - 1.0)
+    assert rel.max() <= 7.5e-5, f"max relative error {rel.max():.3e}"
+    low = torch.tensor([-125.5, -130.0, -1e4, -np.inf], dtype=torch.float32, device="cuda")
+    yl = cuda_lib.debug_exp2_poly(low).cpu().double().numpy()
+    assert np.all(yl > 0) and np.all(yl <= 2.0 ** -124)
+    assert cuda_lib.device_status() == cuda_lib.OK

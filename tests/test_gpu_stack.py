@@ -7,14 +7,20 @@ Prefill covers rows 0..255; each decode step t runs one token through every
 layer (ring write + window read, global-KV append, cross decode over the
 whole cache) and must reproduce row t of the oracle's 272-row run -- the
 decode == prefill-row invariant of the method (rows depend only on earlier
-rows), and the reason early exit is exact."""
+rows), and the reason early exit is exact.
+
+In bf16 the stack stores every intermediate in bf16; its outputs are checked
+stage by stage against a float64 model that rounds at the same points
+(tests/stack_model.py) at the bf16 bar, and end to end against the
+unrounded oracle within bounds derived from that model."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import workloads as wl
-from tests.util import assert_close
+from tests import stack_model as sm
+from tests.util import BF16_MAX_ABS, BF16_REL_L2, assert_close, errors, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -82,6 +88,36 @@ def gpu_stack(yoco, x, w, cfg):
     return out
 
 
+def _close_to_bf16_steps(got, ref, what):
+    """The bf16 bar for a stored bf16 tensor whose values reach past 4 (the
+    residual stream x, |x| up to ~6; K and V): where one bf16 step exceeds
+    2e-2 a value may sit one step (2^-7 |value| at most) from the
+    reference's, so max-abs allows 2e-2 plus one step; rel-L2 stays 5e-3."""
+    g, r = to_np(got), to_np(ref)
+    assert np.all(np.isfinite(g)), what
+    excess = float(np.max(np.abs(g - r) - 2.0 ** -7 * np.abs(r)))
+    _, rl = errors(g, r)
+    assert excess <= BF16_MAX_ABS and rl <= BF16_REL_L2, f"{what}: excess {excess:.3e}, rel_l2 {rl:.3e}"
+
+
+def _check_against_rounding_model(got, x, w, cfg):
+    """Stage by stage against the float64 model that rounds to bf16 where the
+    GPU stores bf16: only the kernels' own arithmetic differs, so every stored
+    tensor meets the bf16 bar (2e-2, 5e-3), its max-abs part widened by one
+    bf16 step where the values reach 4 and a step exceeds 2e-2 (K, V and x
+    have such values; a value next to a rounding boundary lands one step
+    apart)."""
+    T = cfg.T
+    m = sm.stack(x, w, cfg)
+    for key in ("self_k", "self_v", "self_o", "cross_o"):
+        for l in range(len(m[key])):
+            _close_to_bf16_steps(got[key][l], m[key][l][:T], f"{key}{l} vs rounding model")
+    _close_to_bf16_steps(got["k_g"], m["k_g"], "k_g vs rounding model")
+    _close_to_bf16_steps(got["v_g"], m["v_g"], "v_g vs rounding model")
+    _close_to_bf16_steps(got["x_prefill"], m["x"][:T], "x prefill vs rounding model")
+    _close_to_bf16_steps(got["x_decode"], m["x"][T:], "x decode vs rounding model")
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_tiny_stack_prefill_and_decode(cuda_lib, dtype):
     cfg = wl.TinyStack()
@@ -93,8 +129,10 @@ def test_tiny_stack_prefill_and_decode(cuda_lib, dtype):
     if dtype == torch.float32:
         tol = dict(max_abs=2e-3, rel_l2=2e-5)
     else:
-        # bf16 storage of every intermediate through 4 residual layers
-        tol = dict(max_abs=1e-1, rel_l2=1.5e-2)
+        # against the unrounded oracle: the bf16 storage of every intermediate
+        # costs up to half of these bounds by itself (tests/stack_model.py)
+        tol = dict(max_abs=sm.BF16_STACK_MAX_ABS, rel_l2=sm.BF16_STACK_REL_L2)
+        _check_against_rounding_model(got, x, w, cfg)
     for l in range(cfg.n_self):
         assert_close(got["self_k"][l], ref["self_k"][l][:T], dtype, f"self_k{l}", **tol)
         assert_close(got["self_v"][l], ref["self_v"][l][:T], dtype, f"self_v{l}", **tol)
@@ -150,7 +188,10 @@ def test_tiny_stack_early_exit(cuda_lib, dtype):
     full = gpu_stack(cuda_lib, x.cuda(), wc, cfg)["x_prefill"][T - 1]
     if dtype == torch.float32:
         tol = dict(max_abs=2e-3, rel_l2=2e-5)
+        assert_close(got, full.float().cpu().numpy(), dtype, "early exit vs full prefill", **tol)
     else:
-        tol = dict(max_abs=1e-1, rel_l2=1.5e-2)
+        tol = dict(max_abs=sm.BF16_STACK_MAX_ABS, rel_l2=sm.BF16_STACK_REL_L2)
+        # the residual stream at the bf16 bar, scaled to x's magnitude
+        _close_to_bf16_steps(got, sm.stack(x[:T], w, cfg, early_exit=True), "early exit vs rounding model")
+        _close_to_bf16_steps(got, full.float().cpu().numpy(), "early exit vs full prefill")
     assert_close(got, ref, dtype, "early exit vs oracle", **tol)
-    assert_close(got, full.float().cpu().numpy(), dtype, "early exit vs full prefill", **tol)

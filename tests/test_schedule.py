@@ -100,6 +100,7 @@ def test_prefill_plan_order_and_balance(B, Hq, Hkv, Tq, Tkv, q_pos0, W, n_cta):
     ([1, 2, 3, 130, 4097], 5000, 8, 1, 64, 148),
     ([65536, 70001, 131072, 100000], 131072, 32, 8, 128, 148),
     ([0, 5, 0, 300], 300, 4, 2, 64, 3),
+    ([100, 5000, 7, 1000], 1000, 32, 8, 128, 16),   # 5000 > max_len: out of range, no units
 ])
 def test_decode_plan_partitions_sequences(lens, max_len, Hq, Hkv, D, n_cta):
     starts = np.cumsum([0] + [l + 7 for l in lens[:-1]])
@@ -119,7 +120,8 @@ def test_decode_plan_partitions_sequences(lens, max_len, Hq, Hkv, D, n_cta):
         for k, (off, n, s) in enumerate(segs):
             assert off == pos and s == k         # consecutive, no gap or overlap
             pos += n
-        assert pos == L                          # the whole sequence, nothing past it
+        # the whole sequence, nothing past it; none of a sequence out of range
+        assert pos == (L if 1 <= L <= max_len else 0)
         if len(segs) > 1:                        # equal splits, a multiple of the stage
             split = segs[0][1]
             assert split % stage == 0 and all(n == split for _, n, _ in segs[:-1])
@@ -135,3 +137,42 @@ def test_schedule_rejects_bad_arguments():
         yoco.debug_tile_schedule(7, 4, 2, 64)
     with pytest.raises(yoco.YocoError):
         yoco.debug_tile_schedule(yoco.SCHEDULE_PREFILL, 3, 2, 64, Tq=1, Tkv=1)   # Hq % Hkv
+
+
+def test_prefill_banded_order_reads_one_stream_per_round():
+    # K/V beyond 32 MB (here 67 MB: T=16384, 8 KV heads, D=128, bf16): the work
+    # order goes in bands, so that each round of the 148-CTA grid streams the
+    # K/V of ONE KV head (two head pairs x 74 query tiles) and the tiles the
+    # CTAs read stay in L2.  Checked: every work tile once, on one CTA, over
+    # exactly KV tiles 0..qt (causal); each round's CTAs on one KV head; the
+    # bands heaviest first; per-CTA totals within one work tile.
+    B, Hq, Hkv, T, n_cta = 1, 32, 8, 16384, 148
+    rec = yoco.debug_tile_schedule(yoco.SCHEDULE_PREFILL, Hq, Hkv, 128, B=B, Tq=T, Tkv=T, n_cta=n_cta)
+    n_qt = T // BM
+    works = {}
+    order = []
+    for cta, b, h, qt, kt, masked in rec.tolist():
+        key = (b, h // 2, qt)
+        if key not in works:
+            works[key] = [cta, []]
+            order.append((cta, key))
+        assert works[key][0] == cta
+        works[key][1].append((h, kt, masked))
+    assert len(works) == n_qt * Hq // 2 * B
+    for (b, hp, qt), (cta, visits) in works.items():
+        assert [kt for h, kt, _ in visits if h == 2 * hp] == list(range(qt + 1))
+        assert all(m == (kt == qt) for _, kt, m in visits)     # only the diagonal tile is masked
+    # round r of CTA c is its r-th work tile; each round is one KV head
+    per_cta = {}
+    for cta, key in order:
+        per_cta.setdefault(cta, []).append(key)
+    G = Hq // Hkv
+    n_rounds = max(len(v) for v in per_cta.values())
+    for r in range(n_rounds):
+        heads = {(2 * k[1]) // G for v in per_cta.values() if r < len(v) for k in [v[r]]}
+        qts = [v[r][2] for v in per_cta.values() if r < len(v)]
+        assert len(heads) <= 3, (r, heads)    # the last, shorter band mixes streams
+        if r == 0:
+            assert len(heads) == 1 and min(qts) >= n_qt - 74      # the heaviest band first
+    tot = {c: sum(k[2] + 1 for k in v) for c, v in per_cta.items()}
+    assert max(tot.values()) - min(tot.values()) <= n_qt

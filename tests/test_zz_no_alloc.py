@@ -4,14 +4,16 @@ a process whose framework holds nearly all device memory), whose split-KV
 scratch is a fixed array inside the library.
 
 Checks, through the C ABI, that two calls in a row (the second finding the
-first call's partials still in the shared array) match the workspace entry
-point within the parity tolerance, and that a decode too large for the
-array is refused with YOCO_ERR_WORKSPACE.  This file is collected last."""
+first call's partials still in the shared array) match both the CPU oracle
+and the workspace entry point within the parity tolerance, and that a decode
+too large for the array is refused with YOCO_ERR_WORKSPACE.  This file is
+collected last."""
 import ctypes
 
 import pytest
 import torch
 
+import oracle
 import workloads as wl
 from tests.util import assert_close
 
@@ -23,7 +25,7 @@ def _static_entry(yoco):
     fn = yoco.load().yoco_cross_decode_static
     vp = ctypes.c_void_p
     fn.restype = ctypes.c_int
-    fn.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int32, ctypes.c_int64, vp, vp,
+    fn.argtypes = [vp, vp, vp, ctypes.c_int64, vp, vp, ctypes.c_int32, ctypes.c_int64, vp, vp,
                    ctypes.POINTER(yoco.AttnCfg), vp]
     return fn
 
@@ -52,10 +54,14 @@ def test_static_scratch_decode_matches_workspace_decode(cuda_lib):
         ref, ref_lse = cuda_lib.cross_decode(q, kc, vc, ss, sl, max(lens), want_lse=True)
         o = torch.empty_like(q)
         lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
-        st = fn(_ptr(q), _ptr(kc), _ptr(vc), _ptr(ss), _ptr(sl), B, max(lens), _ptr(o), _ptr(lse),
+        st = fn(_ptr(q), _ptr(kc), _ptr(vc), rows, _ptr(ss), _ptr(sl), B, max(lens), _ptr(o), _ptr(lse),
                 ctypes.byref(cfg), stream)
         assert st == cuda_lib.OK, f"status {st}"
         torch.cuda.synchronize()
+        ro, rlse = oracle.cross_decode(q.cpu(), kc.cpu(), vc.cpu(), starts.numpy(), lens)
+        for b in range(B):     # per sequence: the random-key outputs are far below unit scale
+            assert_close(o[b], ro[b], BF, f"o vs oracle, sequence {b}")
+        assert_close(lse, rlse, BF, "lse vs oracle", max_abs=1e-3, rel_l2=1e-4)
         assert_close(o, ref, BF, "o vs workspace entry point")
         assert_close(lse, ref_lse, BF, "lse vs workspace entry point", max_abs=1e-3, rel_l2=1e-4)
     assert cuda_lib.device_status() == cuda_lib.OK
@@ -69,5 +75,5 @@ def test_static_scratch_rejects_oversized_decode(cuda_lib):
     assert need > (32 << 20)
     dummy = torch.empty(16, dtype=torch.uint8, device="cuda")
     p = _ptr(dummy)
-    st = fn(p, p, p, p, p, B, max_len, p, None, ctypes.byref(cfg), None)
+    st = fn(p, p, p, 1 << 20, p, p, B, max_len, p, None, ctypes.byref(cfg), None)
     assert st == cuda_lib.ERR_WORKSPACE
