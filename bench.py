@@ -499,10 +499,17 @@ def gret_layer(W, reps):
 
     t_pre = timed(lambda: yoco.gret_prefill(q, k, v, g, tau, state=st, o=o))
     t_dec = timed(lambda: yoco.gret_decode(qd, kd, vd, gd, tau, sd, o=od))
+    # batch 1: 32 sequences for 148 SMs, so each runs as superchunks on
+    # separate CTAs (the workspace the library asks for)
+    q1, k1, v1, g1, o1 = q[:1], k[:1], v[:1], g[:1], o[:1]
+    st1 = torch.zeros((1, H, D, D), dtype=torch.float32, device=dev)
+    ws1 = torch.empty(max(16, yoco.gret_prefill_workspace_size(1, T, H, D)), dtype=torch.uint8, device=dev)
+    t_pre1 = timed(lambda: yoco.gret_prefill(q1, k1, v1, g1, tau, state=st1, o=o1, workspace=ws1))
     pre_bytes = 4.0 * B * T * H * D * 2 + B * T * H * 4.0 + 2.0 * B * H * D * D * 4
     return {"prefill_ms": t_pre, "prefill_tflops": gret_flops(B, T, H, D) / (t_pre * 1e-3) / 1e12,
             "prefill_tokens_per_s": B * T / (t_pre * 1e-3),
             "prefill_hbm_gbs": pre_bytes / (t_pre * 1e-3) / 1e9,
+            "prefill_b1_ms": t_pre1, "prefill_b1_tflops": gret_flops(1, T, H, D) / (t_pre1 * 1e-3) / 1e12,
             "decode_ms": t_dec, "decode_gbs": Bd * H * D * D * 8.0 / (t_dec * 1e-3) / 1e9,
             "shape": f"prefill B={B} T={T} H={H} D={D}; decode batch {Bd}",
             "flops": "chunkwise at chunk 128: QK^T and PV over C x C, Q S and K^T V over D x D, per chunk and head",

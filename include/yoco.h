@@ -238,10 +238,19 @@ yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_
  * fp32 returns YOCO_ERR_UNSUPPORTED); g [B, T, H] fp32 gate logits; tau > 0.
  * state [B, H, D, D] fp32, S[d][e] multiplying q_d into o_e: the initial state
  * on entry and the final state on return, or NULL to start from zero and
- * drop the final state.  Caller-owned device memory; asynchronous on stream. */
+ * drop the final state.  Caller-owned device memory; asynchronous on stream.
+ * workspace: NULL, or device scratch of yoco_gret_prefill_workspace_size()
+ * bytes (a smaller non-zero ws_bytes is YOCO_ERR_WORKSPACE).  With it, when
+ * B x H sequences leave SMs idle (D = 128), each sequence's chunks are cut
+ * into up to 8 superchunks on separate CTAs: a first pass forms every
+ * superchunk's state contribution from a zero start and its total decay, and
+ * each superchunk then starts from the decayed sum of those before it (the
+ * same recurrence, regrouped).  The size query returns 0 when no split
+ * applies. */
+size_t yoco_gret_prefill_workspace_size(int32_t B, int64_t T, const yoco_attn_cfg *cfg);
 yoco_status yoco_gret_prefill(const void *q, const void *k, const void *v, const float *g, int32_t B,
-                              int64_t T, float tau, float *state, void *o, const yoco_attn_cfg *cfg,
-                              cudaStream_t stream);
+                              int64_t T, float tau, float *state, void *o, void *workspace, size_t ws_bytes,
+                              const yoco_attn_cfg *cfg, cudaStream_t stream);
 
 /* yoco_gret_decode: one recurrent step.  q, k, v, o [B, H, D] (bf16 or fp32);
  * g [B, H] fp32; state [B, H, D, D] fp32, read and updated in place

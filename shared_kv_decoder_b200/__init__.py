@@ -24,7 +24,7 @@ __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_p
            "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg",
            "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE", "gret_prefill", "gret_decode",
            "kv_i8_row_bytes", "kv_quantize_i8", "cross_decode_i8",
-           "attention_prefill", "debug_exp2_poly"]
+           "attention_prefill", "debug_exp2_poly", "gret_prefill_workspace_size"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -78,7 +78,8 @@ def load():
         "yoco_cross_decode_workspace_size": (sz, [i32, i64, cfgp]),
         "yoco_swa_decode_workspace_size": (sz, [i32, i32, cfgp]),
         "yoco_cache_bytes": (ctypes.c_double, [i32, i32, i64, cfgp]),
-        "yoco_gret_prefill": (st, [vp, vp, vp, vp, i32, i64, f32, vp, vp, cfgp, vp]),
+        "yoco_gret_prefill": (st, [vp, vp, vp, vp, i32, i64, f32, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_gret_prefill_workspace_size": (sz, [i32, i64, cfgp]),
         "yoco_kv_i8_row_bytes": (i64, [cfgp]),
         "yoco_kv_quantize_i8": (st, [vp, vp, i64, vp, vp, vp, cfgp, vp]),
         "yoco_cross_decode_i8": (st, [vp, vp, vp, i64, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
@@ -289,18 +290,30 @@ def debug_tile_schedule(kind, Hq, Hkv, D, dtype=torch.bfloat16, B=1, Tq=0, Tkv=0
     return out
 
 
-def gret_prefill(q, k, v, g, tau, state=None, scale=0.0, o=None):
+def gret_prefill_workspace_size(B, T, H, D, dtype=torch.bfloat16):
+    cfg = _cfg(H, H, D, dtype)
+    return int(load().yoco_gret_prefill_workspace_size(B, int(T), ctypes.byref(cfg)))
+
+
+def gret_prefill(q, k, v, g, tau, state=None, scale=0.0, o=None, workspace="auto"):
     """Chunkwise gated retention over a prompt.  q, k, v [B, T, H, D] bf16;
     g [B, T, H] fp32 gate logits; state [B, H, D, D] fp32 initial state,
-    overwritten with the final state (None: start from zero).  Returns o."""
+    overwritten with the final state (None: start from zero).
+    workspace: a uint8 CUDA tensor for the split over superchunks, "auto" to
+    allocate one of the size the library asks for, or None (no split).
+    Returns o."""
     L = load()
     B, T, H, D = q.shape
     if o is None:
         o = torch.empty_like(q)
-    _dev(q, k, v, g, state, o)
+    if isinstance(workspace, str):
+        n = gret_prefill_workspace_size(B, T, H, D, q.dtype)
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device) if n > 0 else None
+    _dev(q, k, v, g, state, o, workspace)
     cfg = _cfg(H, H, D, q.dtype, scale)
+    ws_bytes = workspace.numel() if workspace is not None else 0
     _check(L.yoco_gret_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, T, float(tau), _ptr(state), _ptr(o),
-                               ctypes.byref(cfg), _stream()), "yoco_gret_prefill")
+                               _ptr(workspace), ws_bytes, ctypes.byref(cfg), _stream()), "yoco_gret_prefill")
     return o
 
 

@@ -290,20 +290,31 @@ yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_
     return from_cuda(launch_decode_i8(a, pl, stream));
 }
 
+size_t yoco_gret_prefill_workspace_size(int32_t B, int64_t T, const yoco_attn_cfg *cfg) {
+    if (check_cfg(cfg) != YOCO_OK || cfg->Hq != cfg->Hkv || cfg->dtype != YOCO_BF16) return 0;
+    return gret_workspace_bytes(B, cfg->Hq, T, cfg->D);
+}
+
 yoco_status yoco_gret_prefill(const void *q, const void *k, const void *v, const float *g, int32_t B,
-                              int64_t T, float tau, float *state, void *o, const yoco_attn_cfg *cfg,
-                              cudaStream_t stream) {
+                              int64_t T, float tau, float *state, void *o, void *workspace, size_t ws_bytes,
+                              const yoco_attn_cfg *cfg, cudaStream_t stream) {
     yoco_status st = check_cfg(cfg);
     if (st != YOCO_OK) return st;
     if (cfg->Hq != cfg->Hkv || B < 0 || T < 0 || !(tau > 0.f) || isinf(tau)) return YOCO_ERR_INVALID;
     if (B == 0 || T == 0) return YOCO_OK;
-    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_opt(state) || !ok_ptr(o))
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_opt(state) || !ok_ptr(o) ||
+        !ok_opt(workspace))
         return YOCO_ERR_INVALID;
     if (cfg->dtype != YOCO_BF16) return YOCO_ERR_UNSUPPORTED;
+    // a workspace enables the split over superchunks; one smaller than the
+    // size query's answer is an error, a NULL one (or a size of 0) means no split
+    const size_t need = gret_workspace_bytes(B, cfg->Hq, T, cfg->D);
+    if (workspace && ws_bytes < need) return YOCO_ERR_WORKSPACE;
     GretArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.state = state; a.o = o;
     a.B = B; a.H = cfg->Hq; a.D = cfg->D; a.dtype = cfg->dtype; a.T = T;
     a.tau = tau; a.scale = eff_scale(cfg);
+    a.ws = (workspace && need > 0) ? workspace : nullptr;
     return from_cuda(launch_gret_prefill(a, stream));
 }
 
@@ -318,7 +329,7 @@ yoco_status yoco_gret_decode(const void *q, const void *k, const void *v, const 
     GretArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.state = state; a.o = o;
     a.B = B; a.H = cfg->Hq; a.D = cfg->D; a.dtype = cfg->dtype; a.T = 1;
-    a.tau = tau; a.scale = eff_scale(cfg);
+    a.tau = tau; a.scale = eff_scale(cfg); a.ws = nullptr;
     return from_cuda(launch_gret_decode(a, stream));
 }
 

@@ -107,6 +107,19 @@ YOCO_DEV void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, uin
         : "memory");
 }
 
+// ------------------------------------------- programmatic dependent launch
+// The decode-step kernels (small projections, ring write, split decode,
+// merge) are launched with programmatic stream serialization (launch_pdl): the
+// next kernel on the stream is launched while this one runs and its CTAs wait
+// in pdl_wait() -- which returns once every earlier kernel on the stream has
+// finished and its writes are visible -- so the launch gap between the short
+// kernels of a decode step disappears.  Every such kernel calls pdl_wait()
+// before it reads any input (and before any early exit), which also keeps the
+// ordering transitive along the stream.  Without the launch attribute both
+// are no-ops.
+YOCO_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+YOCO_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------ warp helpers
 YOCO_DEV float warp_max(float v) {
 #pragma unroll

@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
     constexpr int DPL = CPL * EPC;            // dims per lane
     static_assert(CPL >= 1 && CPR % kLanesPerTok == 0, "head dim too small for the lane layout");
 
+    pdl_trigger();
+    pdl_wait();
     if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     extern __shared__ __align__(128) unsigned char smem[];
     const int64_t row_elems = (int64_t)p.Hkv * D;
@@ -379,6 +381,8 @@ template <int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeKParams p) {
+    pdl_trigger();
+    pdl_wait();
     if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     static_assert(G >= 1 && G <= 8, "query heads per KV head");
     constexpr int KB = D / 64;                       // 64-column blocks per head row
@@ -673,6 +677,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const DecodeI8Params pi) {
     static_assert(G >= 1 && G <= 8, "the query heads of a group are the 8 columns of an MMA");
+    pdl_trigger();
+    pdl_wait();
     if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     constexpr int D = 128;
     constexpr uint32_t kBox = kRowsPerStage * 128;  // one code box: 128 rows of 128 bytes
@@ -1018,6 +1024,8 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(
     __shared__ float s_acc[kMergeWarps][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = (int)(blockIdx.x / Hq), h = (int)(blockIdx.x % Hq);
+    pdl_trigger();
+    pdl_wait();
     const int64_t len = seq_len ? (int64_t)seq_len[b] : (int64_t)window;
     // the split kernel gave an out-of-range sequence no units; its output
     // becomes 0 (lse -inf) and the status word records it once
@@ -1091,7 +1099,10 @@ bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dt
     DecodePlan pl;
     pl.stage_tokens = kRowsPerStage / Hkv;
     pl.sub = kConsumerWarps / Hkv;
-    const int64_t min_split = 4 * pl.stage_tokens;
+    // at least two pipeline stages per unit; small decodes (a sliding-window
+    // ring of 4 x 1024 slots) then spread over ~128 CTAs, each with its whole
+    // unit in flight, instead of 64 CTAs streaming four stages each
+    const int64_t min_split = 2 * pl.stage_tokens;
     int64_t per = ((int64_t)std::max(B, 1) * max_len + kTargetUnits - 1) / kTargetUnits;
     per = ((per + pl.stage_tokens - 1) / pl.stage_tokens) * pl.stage_tokens;
     pl.split = std::max(per, min_split);
@@ -1140,8 +1151,7 @@ static cudaError_t launch_decode_tma(const DecodeArgs &a, const DecodePlan &pl, 
     auto kern = decode_tma_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kDecodeThreads, pl.smem_bytes, st>>>(mk, mv, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kDecodeThreads), pl.smem_bytes, st, mk, mv, p);
 }
 
 template <typename T, int D, int G>
@@ -1167,16 +1177,14 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
         auto kern = decode_split_kernel<T, D, G>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
         if (e != cudaSuccess) return e;
-        kern<<<grid, kDecodeThreads, pl.smem_bytes, st>>>(p);
-        e = cudaGetLastError();
+        e = launch_pdl(kern, dim3(grid), dim3(kDecodeThreads), pl.smem_bytes, st, p);
     }
     note_launches(2);
     if (e != cudaSuccess) return e;
     const int mgrid = (int)((int64_t)a.B * a.Hq);
-    decode_merge_kernel<T, D><<<mgrid, 32 * kMergeWarps, 0, st>>>(
-        p.ws_o, p.ws_ml, a.seq_start, a.seq_len, a.window, a.B, a.Hq, a.max_len, a.cache_rows, pl.split,
-        pl.n_split, pl.sub, static_cast<T *>(a.o), a.lse);
-    return cudaGetLastError();
+    return launch_pdl(decode_merge_kernel<T, D>, dim3(mgrid), dim3(32 * kMergeWarps), 0, st, p.ws_o, p.ws_ml,
+                      a.seq_start, a.seq_len, a.window, a.B, a.Hq, a.max_len, a.cache_rows, pl.split, pl.n_split,
+                      pl.sub, static_cast<T *>(a.o), a.lse);
 }
 
 template <typename T, int D>
@@ -1252,14 +1260,13 @@ static cudaError_t launch_decode_i8_g(const DecodeArgs &a, const DecodePlan &pl,
     if (e != cudaSuccess) return e;
     const int64_t units = (int64_t)a.B * pl.n_split;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, device_sm_count()));
-    kern<<<grid, kDecodeThreads, smem, st>>>(mk, mv, mks, mvs, pi);
     note_launches(2);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3(grid), dim3(kDecodeThreads), smem, st, mk, mv, mks, mvs, pi);
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<__nv_bfloat16, 128><<<(int)((int64_t)a.B * a.Hq), 32 * kMergeWarps, 0, st>>>(
-        p.ws_o, p.ws_ml, a.seq_start, a.seq_len, a.window, a.B, a.Hq, a.max_len, a.cache_rows, pl.split,
-        pl.n_split, pl.sub, static_cast<__nv_bfloat16 *>(a.o), a.lse);
-    return cudaGetLastError();
+    return launch_pdl(decode_merge_kernel<__nv_bfloat16, 128>, dim3((unsigned)((int64_t)a.B * a.Hq)),
+                      dim3(32 * kMergeWarps), 0, st, p.ws_o, p.ws_ml, a.seq_start, a.seq_len, a.window, a.B,
+                      a.Hq, a.max_len, a.cache_rows, pl.split, pl.n_split, pl.sub,
+                      static_cast<__nv_bfloat16 *>(a.o), a.lse);
 }
 
 cudaError_t launch_decode_i8(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t st) {
@@ -1326,6 +1333,8 @@ template <typename T>
 __global__ void ring_write_kernel(const T *k_new, const T *v_new, const int64_t *pos, int32_t window,
                                   int64_t row_elems, T *ring_k, T *ring_v, int32_t *slot_pos) {
     const int b = blockIdx.x;
+    pdl_trigger();
+    pdl_wait();
     const int64_t p = pos[b];
     const int64_t slot = ((p % window) + window) % window;
     T *dk = ring_k + ((int64_t)b * window + slot) * row_elems;
@@ -1344,16 +1353,13 @@ cudaError_t launch_ring_write(const void *k_new, const void *v_new, const int64_
     const int64_t re = (int64_t)Hkv * D;
     note_launches(1);
     if (dtype == kBF16)
-        ring_write_kernel<__nv_bfloat16><<<B, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new), pos,
-            window, re, static_cast<__nv_bfloat16 *>(ring_k), static_cast<__nv_bfloat16 *>(ring_v),
-            slot_pos);
-    else
-        ring_write_kernel<float><<<B, 256, 0, st>>>(static_cast<const float *>(k_new),
-                                                    static_cast<const float *>(v_new), pos, window, re,
-                                                    static_cast<float *>(ring_k),
-                                                    static_cast<float *>(ring_v), slot_pos);
-    return cudaGetLastError();
+        return launch_pdl(ring_write_kernel<__nv_bfloat16>, dim3(B), dim3(256), 0, st,
+                          static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new),
+                          pos, window, re, static_cast<__nv_bfloat16 *>(ring_k),
+                          static_cast<__nv_bfloat16 *>(ring_v), slot_pos);
+    return launch_pdl(ring_write_kernel<float>, dim3(B), dim3(256), 0, st, static_cast<const float *>(k_new),
+                      static_cast<const float *>(v_new), pos, window, re, static_cast<float *>(ring_k),
+                      static_cast<float *>(ring_v), slot_pos);
 }
 
 // Ring contents after a prefill of T tokens: slot s keeps the newest position

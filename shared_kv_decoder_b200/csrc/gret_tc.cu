@@ -69,6 +69,7 @@ constexpr int kThreads = 352;
 constexpr uint32_t kBlk = 128 * 128;      // one [128 rows x 128 bytes] swizzled block
 constexpr uint32_t kTile = 2 * kBlk;      // a [128, 128] bf16 tile (two 64-column blocks)
 constexpr float kFoldMinLog2 = -60.f;     // smallest chunk decay (log2) that folds into K_w
+constexpr int kMaxSuperchunks = 8;        // CTAs per sequence at most (see gret_superchunks)
 
 enum Smem : uint32_t {
     kQ = 0,
@@ -113,7 +114,19 @@ struct GretTcParams {
     int64_t T;
     float lg_scale;   // log2(e) / tau
     float scale;
-    int32_t n_chunks;
+    int32_t n_chunks;     // chunks of the whole sequence
+    // Superchunks (see launch_gret_prefill_tc): each sequence's chunks split
+    // into n_sc contiguous runs of sc_chunks, one CTA each.  n_sc = 1: one CTA
+    // walks the whole sequence.
+    int32_t n_sc, sc_chunks;
+    int32_t state_only;   // this launch forms superchunks 0 .. n_sc - 2's state contributions
+    // scratch of a split launch, per sequence: n_sc [D, D] fp32 slots --
+    // slot s < n_sc - 1: superchunk s's final state from a zero start; slot
+    // n_sc - 1: a copy of the initial state (zeros without one), so that no
+    // CTA of the output pass reads `state`, which the last superchunk
+    // overwrites -- then n_sc floats, log2 of each superchunk's total decay
+    float *sc_state;
+    float *sc_log2decay;
 };
 
 YOCO_DEV bool wait1(uint64_t *bar, uint32_t parity) { return mbar_wait(bar, parity, &g_status_gret_tc); }
@@ -149,14 +162,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sb + kMisc + 4);
     volatile int *fold_flag = reinterpret_cast<volatile int *>(sb + kMisc + 8);  // [2]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
-    const int NC = p.n_chunks;
+    // CTA -> (sequence, superchunk); the state-only launch covers superchunks
+    // 0 .. n_sc - 2 (the last one's contribution feeds nothing)
+    const bool so = p.state_only != 0;
+    const int per_seq = so ? p.n_sc - 1 : p.n_sc;
+    const int bh = blockIdx.x / per_seq, sc = blockIdx.x % per_seq;
+    const int b = bh / p.H, h = bh % p.H;
+    const int j0 = sc * p.sc_chunks;                         // first chunk of this CTA
+    const int NC = min(p.sc_chunks, p.n_chunks - j0);        // chunks of this CTA
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) {
             int cnt = 1;
             if (i == kPFull || i == kOFree || i == kOStaged || i == kSReady) cnt = 128;
-            if (i == kKEmpty || i == kVEmpty || i == kVEmpty + 1) cnt = 2;
+            // K and V buffers are released by the output side and the state
+            // side; a state-only launch has no output side
+            if (!so && (i == kKEmpty || i == kVEmpty || i == kVEmpty + 1)) cnt = 2;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -175,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 8) {
         // ------------------------------------------------------ TMA producer
         // lane 0: Q, lane 1: K, lane 2: V (two buffers)
-        if (lane < 3) {
+        if (lane < 3 && !(so && lane == 0)) {   // a state-only launch reads no Q
             const CUtensorMap *map = lane == 0 ? &tm_q : lane == 1 ? &tm_k : &tm_v;
             const int nb = lane == 2 ? 2 : 1;
             const uint32_t dst0 = base + (lane == 0 ? kQ : lane == 1 ? kK : kV0);
@@ -187,9 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (use > 0 && !wait1(&empty[bi], (use - 1) & 1)) { *abort_flag = 1; break; }
                 mbar_arrive_expect_tx(&full[bi], kC * kD * 2);
                 for (int kb = 0; kb < 2; ++kb)
-                    tc::tma_load_4d(dst0 + bi * kTile + kb * kBlk, map, kb * 64, h, j * kC, b, &full[bi]);
+                    tc::tma_load_4d(dst0 + bi * kTile + kb * kBlk, map, kb * 64, h, (j0 + j) * kC, b, &full[bi]);
                 if (j + nb < NC)
-                    for (int kb = 0; kb < 2; ++kb) tc::tma_prefetch_4d(map, kb * 64, h, (j + nb) * kC, b);
+                    for (int kb = 0; kb < 2; ++kb) tc::tma_prefetch_4d(map, kb * 64, h, (j0 + j + nb) * kC, b);
             }
             // the last copy into each buffer has landed before exit
             for (int jj = j - 1; jj >= 0 && jj >= j - nb; --jj) wait1(&full[jj % nb], (jj / nb) & 1);
@@ -200,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idQK = tc::idesc_bf16(128, 128, false, false);
             constexpr uint32_t idMNB = tc::idesc_bf16(128, 128, false, true);
             bool ok = true;
-            for (int j = 0; ok && j < NC; ++j) {
+            for (int j = 0; ok && !so && j < NC; ++j) {
                 const uint32_t ph = j & 1, bi = j & 1, ph2 = (j >> 1) & 1;
                 const uint32_t v_s = base + kV0 + bi * kTile;
                 // scores: Q K_w^T when the chunk folds, else Q K^T
@@ -273,15 +294,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float *gb = p.g + (int64_t)b * p.T * p.H + h;
         const bool store_thread = warp == 0 && lane == 0;   // issues the output tile's TMA store
         bool ok = true;
+        float sc_log2 = 0.f;   // running log2 of this CTA's total decay (state-only launch)
 
         if (state_role) {
-            // initial state into TMEM rows
+            // initial state into TMEM rows: zero for a state-only launch; for
+            // superchunk s > 0 of the output launch, the state after the
+            // superchunks before it,
+            //   S_s = 2^(G_0 + .. + G_{s-1}) S_init + sum_{s' < s} 2^(G_{s'+1} + .. + G_{s-1}) dS_{s'}
+            // (G: a superchunk's log2 total decay, dS: its state from zero)
             const float *s0 = p.state ? p.state + ((int64_t)b * p.H + h) * kD * kD + (int64_t)r * kD : nullptr;
+            float *dS = nullptr, *s_copy = nullptr;
+            const float *G = nullptr;
+            if (p.n_sc > 1) {
+                dS = p.sc_state + (int64_t)bh * p.n_sc * kD * kD + (int64_t)r * kD;
+                s_copy = dS + (int64_t)(p.n_sc - 1) * kD * kD;
+                G = p.sc_log2decay + (int64_t)bh * p.n_sc;
+                if (!so) s0 = s_copy;   // the state-only pass copied the initial state
+            }
 #pragma unroll
             for (int c = 0; c < kD; c += 32) {
                 float v[32];
+                if (so) {
+                    if (sc == 0) {   // the initial state's copy for the output pass
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[c + e] : 0.f;
+                        for (int e = 0; e < 32; ++e) s_copy[c + e] = s0 ? s0[c + e] : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                } else if (p.n_sc == 1) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[c + e] : 0.f;
+                } else {
+                    float tail = 0.f;   // G_{s'+1} + .. + G_{sc-1}, built from s' = sc - 1 down
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                    for (int s2 = sc - 1; s2 >= 0; --s2) {
+                        const float wgt = tc::ex2(tail);
+                        const float *row = dS + (int64_t)s2 * kD * kD + c;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = fmaf(wgt, row[e], v[e]);
+                        tail += G[s2];
+                    }
+                    const float wgt = tc::ex2(tail);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = fmaf(wgt, s0[c + e], v[e]);
+                }
                 tc::tmem_st32(tS + lane_off + c, v);
             }
             tc::wait_st();
@@ -291,13 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         float gn[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int64_t t = 4 * lane + i;
+            const int64_t t = (int64_t)j0 * kC + 4 * lane + i;
             gn[i] = t < p.T ? gb[t * p.H] : 0.f;
         }
 
         for (int j = 0; ok && j < NC; ++j) {
             const uint32_t ph = j & 1;
-            const int64_t t0 = (int64_t)j * kC;
+            const int64_t t0 = (int64_t)(j0 + j) * kC;
             // running base-2 log-decay sums of the chunk in registers: lane l
             // holds c_u for u = 4l..4l+3 (padded rows decay by 1)
             float x[4];
@@ -336,7 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float c_last = __shfl_sync(0xffffffffu, x[3], 31);
             const bool fold = c_last >= kFoldMinLog2;   // the same in every warp
+            sc_log2 += c_last;
 
+            if (so && !state_role) break;   // a state-only launch: the output warps have nothing to do
             if (!state_role) {
                 // ---- P: 2^{c_r - c_last} (Q K_w^T) or scale 2^{c_r - c_u} (Q K^T),
                 // for u <= r, else 0
@@ -420,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- K_w = K * scale * 2^{c_last - c_u} (row u = r of the K tile);
                 // the previous update and the previous scores have read K_w
                 if (!waitw(&bars[kKFull], ph)) { ok = false; break; }
-                if (j > 0 && !waitw(&bars[kAFull], (j - 1) & 1)) { ok = false; break; }
+                if (!so && j > 0 && !waitw(&bars[kAFull], (j - 1) & 1)) { ok = false; break; }
                 {
                     const float w = p.scale * tc::ex2(c_last - c_r);
 #pragma unroll
@@ -440,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- one pass over S_prev: its bf16 copy for this chunk's cross
                 // term (once the previous cross term has read the last copy),
                 // and S *= 2^{c_last} in TMEM
-                if (j > 0 && !waitw(&bars[kQEmpty], (j - 1) & 1)) { ok = false; break; }
+                if (!so && j > 0 && !waitw(&bars[kQEmpty], (j - 1) & 1)) { ok = false; break; }
                 {
                     const float f = tc::ex2(c_last);
                     tc::fence_after_sync();
@@ -449,14 +508,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float v[32];
                         tc::tmem_ld32(tS + lane_off + c, v);
                         tc::wait_ld();
+                        if (!so) {   // the cross term's bf16 copy (no cross term without outputs)
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 hv;
-                            hv.x = tc::pack_bf16x2(v[e], v[e + 1]);
-                            hv.y = tc::pack_bf16x2(v[e + 2], v[e + 3]);
-                            hv.z = tc::pack_bf16x2(v[e + 4], v[e + 5]);
-                            hv.w = tc::pack_bf16x2(v[e + 6], v[e + 7]);
-                            *reinterpret_cast<uint4 *>(sb + kSb + sw_off(r, c + e)) = hv;
+                            for (int e = 0; e < 32; e += 8) {
+                                uint4 hv;
+                                hv.x = tc::pack_bf16x2(v[e], v[e + 1]);
+                                hv.y = tc::pack_bf16x2(v[e + 2], v[e + 3]);
+                                hv.z = tc::pack_bf16x2(v[e + 4], v[e + 5]);
+                                hv.w = tc::pack_bf16x2(v[e + 6], v[e + 7]);
+                                *reinterpret_cast<uint4 *>(sb + kSb + sw_off(r, c + e)) = hv;
+                            }
                         }
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] *= f;
@@ -471,10 +532,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!waitw(&bars[kSUpdated], ph)) { ok = false; break; }
             }
         }
-        if (ok && state_role && p.state) {
-            // the final state
+        // the final state: a state-only CTA's into the scratch (with its log2
+        // total decay); in the output launch only the last superchunk's
+        float *sfin = nullptr;
+        if (so)
+            sfin = p.sc_state + ((int64_t)bh * p.n_sc + sc) * kD * kD + (int64_t)r * kD;
+        else if (p.state && sc == p.n_sc - 1)
+            sfin = p.state + ((int64_t)b * p.H + h) * kD * kD + (int64_t)r * kD;
+        if (so && ok && warp == 4 && lane == 0) p.sc_log2decay[(int64_t)bh * p.n_sc + sc] = sc_log2;
+        if (ok && state_role && sfin) {
             tc::fence_after_sync();
-            float *sfin = p.state + ((int64_t)b * p.H + h) * kD * kD + (int64_t)r * kD;
 #pragma unroll
             for (int c = 0; c < kD; c += 32) {
                 float v[32];
@@ -526,11 +593,44 @@ cudaError_t launch_gret_prefill_tc(const GretArgs &a, cudaStream_t st) {
     p.lg_scale = kLog2e / a.tau;
     p.scale = a.scale;
     p.n_chunks = (int)((a.T + kC - 1) / kC);
+    p.n_sc = a.ws ? gret_superchunks(a.B, a.H, a.T, device_sm_count()) : 1;
+    p.sc_chunks = (p.n_chunks + p.n_sc - 1) / p.n_sc;
+    p.n_sc = (p.n_chunks + p.sc_chunks - 1) / p.sc_chunks;   // no empty superchunk
+    p.sc_state = static_cast<float *>(a.ws);
+    p.sc_log2decay = p.sc_state ? p.sc_state + (size_t)a.B * a.H * p.n_sc * kD * kD : nullptr;
     cudaError_t e = cudaFuncSetAttribute(gret_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAlloc);
     if (e != cudaSuccess) return e;
+    const int bh = a.B * a.H;
+    if (p.n_sc > 1) {
+        // pass 1: every superchunk but the last forms its state from zero
+        p.state_only = 1;
+        note_launches(1);
+        gret_tc_kernel<<<bh * (p.n_sc - 1), kThreads, kAlloc, st>>>(mq, mk, mv, mo, p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // pass 2 (or the only pass): outputs, each superchunk from its own start state
+    p.state_only = 0;
     note_launches(1);
-    gret_tc_kernel<<<a.B * a.H, kThreads, kAlloc, st>>>(mq, mk, mv, mo, p);
+    gret_tc_kernel<<<bh * p.n_sc, kThreads, kAlloc, st>>>(mq, mk, mv, mo, p);
     return cudaGetLastError();
+}
+
+int gret_superchunks(int32_t B, int32_t H, int64_t T, int sms) {
+    // as many superchunks as leave one per SM, at most kMaxSuperchunks, and
+    // at least 8 chunks each; 1 when the sequences alone fill the GPU
+    const int64_t bh = (int64_t)B * H;
+    const int64_t n_chunks = (T + kC - 1) / kC;
+    int64_t n = bh > 0 ? sms / bh : 1;
+    n = std::min<int64_t>(n, kMaxSuperchunks);
+    n = std::min<int64_t>(n, n_chunks / 8);
+    return (int)std::max<int64_t>(n, 1);
+}
+
+size_t gret_workspace_bytes(int32_t B, int32_t H, int64_t T, int D) {
+    if (D != kD || B < 1 || H < 1 || T < 1) return 0;
+    if ((int64_t)B * H >= 148) return 0;   // the sequences alone fill the GPU: no split
+    return (size_t)B * H * kMaxSuperchunks * (kD * kD + 1) * sizeof(float);
 }
 
 unsigned int read_and_clear_status_gret_tc() {

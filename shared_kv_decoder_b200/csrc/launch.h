@@ -112,6 +112,7 @@ struct GretArgs {
     int32_t B, H, D, dtype;
     int64_t T;              // prefill only
     float tau, scale;
+    void *ws;               // prefill: scratch for the split over superchunks, or NULL (no split)
 };
 // Chunkwise prefill (bf16; cudaErrorNotSupported for other dtypes).
 cudaError_t launch_gret_prefill(const GretArgs &a, cudaStream_t s);
@@ -119,6 +120,10 @@ cudaError_t launch_gret_prefill(const GretArgs &a, cudaStream_t s);
 cudaError_t launch_gret_decode(const GretArgs &a, cudaStream_t s);
 // Chunkwise prefill on the tensor cores (bf16, D = 128; cudaErrorNotSupported otherwise).
 cudaError_t launch_gret_prefill_tc(const GretArgs &a, cudaStream_t s);
+// Superchunks per sequence of that kernel for B x H sequences of T tokens on
+// `sms` SMs, and the scratch bytes a split needs (0: the kernel never splits).
+int gret_superchunks(int32_t B, int32_t H, int64_t T, int sms);
+size_t gret_workspace_bytes(int32_t B, int32_t H, int64_t T, int D);
 
 // Test-only: a kernel whose bounded wait is never satisfied (see decode.cu).
 cudaError_t launch_wait_timeout_probe(cudaStream_t s);
@@ -156,5 +161,24 @@ cudaError_t launch_decode_i8(const DecodeArgs &a, const DecodePlan &pl, cudaStre
 
 // Host-side count of kernel launches (reported by yoco_launch_count()).
 void note_launches(int n);
+
+// Launch with programmatic stream serialization (see pdl_wait in common.cuh):
+// the kernel may start before the previous kernel on the stream has finished,
+// and must call pdl_wait() before reading anything.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 }  // namespace yoco

@@ -114,68 +114,94 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const LinearArgs a) {
     }
 }
 
-// A few rows (decode-step projections): the weight is read once, from HBM,
-// by warps that each own four output columns and every row; x (a few KB per
-// row) comes from L2.  LayerNorm statistics per row first, then each x value
-// is normalised as it is loaded.
-constexpr int kSmallRows = 16, kSmallCols = 4, kSmallWarps = 8;
+// A few rows (decode-step projections, n <= 16): the weight is read once,
+// from HBM, and all of it is in flight at once.  One output column per warp
+// (256 CTAs for a 2048-wide [K | V]); each lane first issues every 16-byte
+// load of its slice of the column's weight row (up to 16 in flight per lane),
+// then the CTA stages its x rows in shared memory, takes each row's
+// LayerNorm statistics from there, and the warp forms the n dot products
+// against the registers, normalising x as it reads it.  An earlier version
+// with four columns per warp and 64 CTAs kept too few loads in flight: the
+// 16.8 MB weight of a d=4096 K/V projection took ~16 us to stream.
+constexpr int kSmallRows = 16, kSmallWarps = 8, kSmallChunks = 16;
+constexpr size_t kSmallMaxSmem = 200 * 1024;
 
 template <typename T>
-__global__ void __launch_bounds__(32 * kSmallWarps, 1) linear_small_kernel(const LinearArgs a) {
-    constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
+__global__ void __launch_bounds__(32 * kSmallWarps, 2) linear_small_kernel(const LinearArgs a) {
+    constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte chunk
+    extern __shared__ uint4 xs4[];       // the n x rows, [n][d_in]
     __shared__ float mu[kSmallRows], rs[kSmallRows];
     const T *x = static_cast<const T *>(a.x);
     const T *w = static_cast<const T *>(a.w);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = (int)a.n;
+    const int row_chunks = a.d_in / VEC;          // 16-byte chunks per row
+    const int c = blockIdx.x * kSmallWarps + warp;  // this warp's output column
+    const uint4 *wrow = reinterpret_cast<const uint4 *>(w + (int64_t)min(c, a.d_out - 1) * a.d_in);
+    // while the previous kernel finishes: ask L2 for this warp's weight row
+    // (a prefetch only warms the cache; nothing is read before pdl_wait)
+    pdl_trigger();
+    for (int ch = lane * 8; ch < row_chunks; ch += 256)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + ch));
+    pdl_wait();
+    // this lane's chunks of the weight row: lane, lane + 32, ... (blocks of 16)
+    uint4 wr[kSmallChunks];
+#pragma unroll
+    for (int k = 0; k < kSmallChunks; ++k)
+        if (lane + 32 * k < row_chunks) wr[k] = wrow[lane + 32 * k];
+    // stage x (every thread), then the statistics of each row
+    const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
+    for (int i = threadIdx.x; i < n * row_chunks; i += blockDim.x) xs4[i] = x4[i];
+    __syncthreads();
+    const T *xs = reinterpret_cast<const T *>(xs4);
     for (int r = warp; r < n; r += kSmallWarps) {
         float mean = 0.f, rstd = 1.f;
         if (a.apply_ln) {
-            const T *xr = x + (int64_t)r * a.d_in;
+            const T *xr = xs + (int64_t)r * a.d_in;
             float s1 = 0.f;
-            for (int c = lane; c < a.d_in; c += 32) s1 += to_f32(xr[c]);
+            for (int cc = lane; cc < a.d_in; cc += 32) s1 += to_f32(xr[cc]);
             mean = warp_sum(s1) / (float)a.d_in;
             float q = 0.f;
-            for (int c = lane; c < a.d_in; c += 32) {
-                const float t = to_f32(xr[c]) - mean;
+            for (int cc = lane; cc < a.d_in; cc += 32) {
+                const float t = to_f32(xr[cc]) - mean;
                 q = fmaf(t, t, q);
             }
             rstd = rsqrtf(warp_sum(q) / (float)a.d_in + a.eps);
         }
         if (lane == 0) {
-            mu[r] = a.apply_ln ? mean : 0.f;
-            rs[r] = a.apply_ln ? rstd : 1.f;
+            mu[r] = mean;
+            rs[r] = rstd;
         }
     }
     __syncthreads();
-    const int c0 = (blockIdx.x * kSmallWarps + warp) * kSmallCols;
-    if (c0 >= a.d_out) return;
-    float acc[kSmallRows][kSmallCols];
+    if (c >= a.d_out) return;
+    float acc[kSmallRows];
 #pragma unroll
-    for (int r = 0; r < kSmallRows; ++r)
+    for (int r = 0; r < kSmallRows; ++r) acc[r] = 0.f;
+    for (int k0 = 0; k0 * 32 < row_chunks; k0 += kSmallChunks) {
+        if (k0 > 0) {  // rows longer than 16 chunks per lane: the next block of loads
 #pragma unroll
-        for (int j = 0; j < kSmallCols; ++j) acc[r][j] = 0.f;
-    for (int d0 = lane * VEC; d0 < a.d_in; d0 += 32 * VEC) {
-        float wv[kSmallCols][VEC];
-#pragma unroll
-        for (int j = 0; j < kSmallCols; ++j) {
-            const int c = min(c0 + j, a.d_out - 1);
-            const uint4 raw = *reinterpret_cast<const uint4 *>(w + (int64_t)c * a.d_in + d0);
-            const T *e = reinterpret_cast<const T *>(&raw);
-#pragma unroll
-            for (int u = 0; u < VEC; ++u) wv[j][u] = to_f32(e[u]);
+            for (int k = 0; k < kSmallChunks; ++k)
+                if (lane + 32 * (k0 + k) < row_chunks) wr[k] = wrow[lane + 32 * (k0 + k)];
         }
 #pragma unroll
-        for (int r = 0; r < kSmallRows; ++r) {
-            if (r >= n) break;
-            const uint4 raw = *reinterpret_cast<const uint4 *>(x + (int64_t)r * a.d_in + d0);
-            const T *e = reinterpret_cast<const T *>(&raw);
-            const float m = mu[r], sc = rs[r];
+        for (int k = 0; k < kSmallChunks; ++k) {
+            const int ch = lane + 32 * (k0 + k);
+            if (ch >= row_chunks) break;
+            const T *we = reinterpret_cast<const T *>(&wr[k]);
+            float wv[VEC];
 #pragma unroll
-            for (int u = 0; u < VEC; ++u) {
-                const float xv = (to_f32(e[u]) - m) * sc;
+            for (int u = 0; u < VEC; ++u) wv[u] = to_f32(we[u]);
 #pragma unroll
-                for (int j = 0; j < kSmallCols; ++j) acc[r][j] = fmaf(xv, wv[j][u], acc[r][j]);
+            for (int r = 0; r < kSmallRows; ++r) {
+                if (r >= n) break;
+                const uint4 raw = xs4[(int64_t)r * row_chunks + ch];
+                const T *e = reinterpret_cast<const T *>(&raw);
+                const float m = mu[r], sc = rs[r];
+                float d = 0.f;
+#pragma unroll
+                for (int u = 0; u < VEC; ++u) d = fmaf((to_f32(e[u]) - m) * sc, wv[u], d);
+                acc[r] += d;
             }
         }
     }
@@ -183,21 +209,17 @@ __global__ void __launch_bounds__(32 * kSmallWarps, 1) linear_small_kernel(const
 #pragma unroll
     for (int r = 0; r < kSmallRows; ++r) {
         if (r >= n) break;
-#pragma unroll
-        for (int j = 0; j < kSmallCols; ++j) {
-            const float tot = warp_sum(acc[r][j]);
-            const int c = c0 + j;
-            if (lane != ((r * kSmallCols + j) & 31) || c >= a.d_out) continue;
-            const int64_t dr = a.dst_rows ? a.dst_rows[r] : r;
-            float val = tot;
-            if (c < a.split_col) {
-                if (a.base0) val = fmaf(a.w0, to_f32(static_cast<const T *>(a.base0)[(int64_t)r * a.split_col + c]), val);
-                static_cast<T *>(a.out0)[dr * a.split_col + c] = from_f32<T>(val);
-            } else {
-                const int cc = c - a.split_col;
-                if (a.base1) val = fmaf(a.w1, to_f32(static_cast<const T *>(a.base1)[(int64_t)r * w1 + cc]), val);
-                static_cast<T *>(a.out1)[dr * w1 + cc] = from_f32<T>(val);
-            }
+        const float tot = warp_sum(acc[r]);
+        if (lane != (r & 31)) continue;
+        const int64_t dr = a.dst_rows ? a.dst_rows[r] : r;
+        float val = tot;
+        if (c < a.split_col) {
+            if (a.base0) val = fmaf(a.w0, to_f32(static_cast<const T *>(a.base0)[(int64_t)r * a.split_col + c]), val);
+            static_cast<T *>(a.out0)[dr * a.split_col + c] = from_f32<T>(val);
+        } else {
+            const int cc = c - a.split_col;
+            if (a.base1) val = fmaf(a.w1, to_f32(static_cast<const T *>(a.base1)[(int64_t)r * w1 + cc]), val);
+            static_cast<T *>(a.out1)[dr * w1 + cc] = from_f32<T>(val);
         }
     }
 }
@@ -205,15 +227,24 @@ __global__ void __launch_bounds__(32 * kSmallWarps, 1) linear_small_kernel(const
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t st) {
     if (a.n == 0 || a.d_out == 0) return cudaSuccess;
     const int vec = a.dtype == kBF16 ? 8 : 4;
-    if (a.n <= kSmallRows && a.d_in % vec == 0) {
-        const int cols_per_cta = kSmallWarps * kSmallCols;
-        note_launches(1);
-        const int grid = (a.d_out + cols_per_cta - 1) / cols_per_cta;
-        if (a.dtype == kBF16)
-            linear_small_kernel<__nv_bfloat16><<<grid, 32 * kSmallWarps, 0, st>>>(a);
-        else
-            linear_small_kernel<float><<<grid, 32 * kSmallWarps, 0, st>>>(a);
-        return cudaGetLastError();
+    const size_t xs_bytes = (size_t)a.n * a.d_in * dtype_bytes(a.dtype);
+    if (a.n <= kSmallRows && a.d_in % vec == 0 && xs_bytes <= kSmallMaxSmem) {
+        const int grid = (a.d_out + kSmallWarps - 1) / kSmallWarps;
+        cudaError_t e;
+        if (a.dtype == kBF16) {
+            auto kern = linear_small_kernel<__nv_bfloat16>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallMaxSmem);
+            if (e != cudaSuccess) return e;
+            note_launches(1);
+            e = launch_pdl(kern, dim3(grid), dim3(32 * kSmallWarps), xs_bytes, st, a);
+        } else {
+            auto kern = linear_small_kernel<float>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallMaxSmem);
+            if (e != cudaSuccess) return e;
+            note_launches(1);
+            e = launch_pdl(kern, dim3(grid), dim3(32 * kSmallWarps), xs_bytes, st, a);
+        }
+        return e;
     }
     dim3 grid((unsigned)((a.d_out + kLinBN - 1) / kLinBN), (unsigned)((a.n + kLinBM - 1) / kLinBM));
     note_launches(1);

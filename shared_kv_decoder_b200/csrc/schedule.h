@@ -54,11 +54,19 @@ struct PrefillShape {
 // streams' work tiles of the last query tile, then of the one before, ...).
 constexpr int64_t kPrefillBandMinKVBytes = (int64_t)32 << 20;
 
+// Streams one round of the grid covers (a build-time tuning constant): one
+// keeps the fewest K/V bytes live, more spread the CTAs that read the same
+// tile at the same moment over more of L2.
+#ifndef YOCO_BAND_STREAMS
+#define YOCO_BAND_STREAMS 1
+#endif
+constexpr int kPrefillBandStreams = YOCO_BAND_STREAMS;
+
 // Query tiles per band for a grid of `grid` CTAs, `per` work tiles per (query
 // tile, stream) and kv_bytes of K and V over all streams.
 YOCO_HD int32_t prefill_band(int grid, int per, int64_t kv_bytes) {
     if (kv_bytes <= kPrefillBandMinKVBytes) return 1;
-    const int b = per > 0 ? grid / per : 1;
+    const int b = per > 0 ? grid / (per * kPrefillBandStreams) : 1;
     return b > 0 ? b : 1;
 }
 

@@ -100,17 +100,27 @@ def test_gret_arguments_rejected_before_launch():
     grouped = ctypes.byref(_cfg(Hq=8, Hkv=2))
     fp32 = ctypes.byref(_cfg(Hq=8, Hkv=8, dtype=1))
     # heads must match, tau > 0, pointers valid
-    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, None, FAKE, grouped, None) == yoco.ERR_INVALID
-    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 0.0, None, FAKE, same, None) == yoco.ERR_INVALID
-    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, None, 1, 64, 4.0, None, FAKE, same, None) == yoco.ERR_INVALID
-    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, MISALIGNED, FAKE, same, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, None, FAKE, None, 0, grouped, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 0.0, None, FAKE, None, 0, same, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, None, 1, 64, 4.0, None, FAKE, None, 0, same, None) == yoco.ERR_INVALID
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, MISALIGNED, FAKE, None, 0, same,
+                               None) == yoco.ERR_INVALID
     # the chunkwise prefill is built for bf16 only
-    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, None, FAKE, fp32, None) == yoco.ERR_UNSUPPORTED
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 64, 4.0, None, FAKE, None, 0, fp32, None) == yoco.ERR_UNSUPPORTED
+    # the split's workspace: too small is refused before launch; none is needed
+    # once B x H sequences fill the GPU, nor for D = 64
+    d128 = ctypes.byref(_cfg(Hq=32, Hkv=32))
+    need = L.yoco_gret_prefill_workspace_size(1, 65536, d128)
+    assert need == 32 * 8 * (128 * 128 + 1) * 4
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 1, 65536, 4.0, None, FAKE, FAKE, need - 16, d128,
+                               None) == yoco.ERR_WORKSPACE
+    assert L.yoco_gret_prefill_workspace_size(8, 65536, d128) == 0
+    assert L.yoco_gret_prefill_workspace_size(1, 65536, ctypes.byref(_cfg(Hq=8, Hkv=8, D=64))) == 0
     # decode needs its state
     assert L.yoco_gret_decode(FAKE, FAKE, FAKE, FAKE, 1, 4.0, None, FAKE, same, None) == yoco.ERR_INVALID
     assert L.yoco_gret_decode(FAKE, FAKE, FAKE, FAKE, 1, -1.0, FAKE, FAKE, same, None) == yoco.ERR_INVALID
     # empty inputs: successful no-op
-    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 0, 64, 4.0, None, FAKE, same, None) == yoco.OK
+    assert L.yoco_gret_prefill(FAKE, FAKE, FAKE, FAKE, 0, 64, 4.0, None, FAKE, None, 0, same, None) == yoco.OK
     assert L.yoco_gret_decode(FAKE, FAKE, FAKE, FAKE, 0, 4.0, FAKE, FAKE, same, None) == yoco.OK
 
 

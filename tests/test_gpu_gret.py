@@ -125,3 +125,32 @@ def test_gret_prefill_mixed_decay_chunks(cuda_lib):
     o = cuda_lib.gret_prefill(q.cuda(), k.cuda(), v.cuda(), g.cuda(), tau, state=st)
     _check(o, ro, "o")
     _check(st, rs, "final state")
+
+
+@pytest.mark.parametrize("B,T,H,gate_mean,tau,with_state", [
+    (1, 8192 + 37, 4, 4.0, 16.0, True),    # 65 chunks -> 8 superchunks of 9, ragged last chunk
+    (1, 4096, 2, 0.5, 2.0, False),         # strong decay: early superchunks' states fade out
+    (2, 3000, 3, 2.0, 8.0, True),          # 24 chunks -> 3 superchunks of 8
+])
+def test_gret_prefill_split_over_superchunks(cuda_lib, B, T, H, gate_mean, tau, with_state):
+    # With a workspace and few sequences, each sequence runs as superchunks on
+    # separate CTAs: outputs and the final state must still follow the
+    # recurrence, and agree with the one-CTA-per-sequence launch.
+    D = 128
+    assert cuda_lib.gret_prefill_workspace_size(B, T, H, D) > 0
+    q, k, v, g = _inputs(B, T, H, D, 1600 + T, gate_mean)
+    s0 = wl.normal((B, H, D, D), 1690, F32) * 0.5 if with_state else None
+    lg = oracle.gret_log_decay(g.numpy(), tau)
+    ro, rs = oracle.gret_recurrent(q, k, v, lg, state=s0)
+    qd, kd, vd, gd = q.cuda(), k.cuda(), v.cuda(), g.cuda()
+    st = s0.clone().cuda() if with_state else None
+    o = cuda_lib.gret_prefill(qd, kd, vd, gd, tau, state=st)                  # split (workspace "auto")
+    _check(o, ro, "o, split")
+    if with_state:
+        _check(st, rs, "final state, split")
+    st1 = s0.clone().cuda() if with_state else None
+    o1 = cuda_lib.gret_prefill(qd, kd, vd, gd, tau, state=st1, workspace=None)  # one CTA per sequence
+    _check(o, o1.float().cpu().numpy(), "split vs one CTA per sequence")
+    if with_state:
+        _check(st, st1.cpu().numpy(), "final state, split vs one CTA")
+    assert cuda_lib.device_status() == cuda_lib.OK

@@ -88,14 +88,16 @@ def gpu_stack(yoco, x, w, cfg):
     return out
 
 
-def _close_to_bf16_steps(got, ref, what):
+def _close_to_bf16_steps(got, ref, what, steps=1):
     """The bf16 bar for a stored bf16 tensor whose values reach past 4 (the
     residual stream x, |x| up to ~6; K and V): where one bf16 step exceeds
     2e-2 a value may sit one step (2^-7 |value| at most) from the
-    reference's, so max-abs allows 2e-2 plus one step; rel-L2 stays 5e-3."""
+    reference's for each bf16 rounding on its path that can land on the other
+    side of a boundary, so max-abs allows 2e-2 plus `steps` steps; rel-L2
+    stays 5e-3."""
     g, r = to_np(got), to_np(ref)
     assert np.all(np.isfinite(g)), what
-    excess = float(np.max(np.abs(g - r) - 2.0 ** -7 * np.abs(r)))
+    excess = float(np.max(np.abs(g - r) - steps * 2.0 ** -7 * np.abs(r)))
     _, rl = errors(g, r)
     assert excess <= BF16_MAX_ABS and rl <= BF16_REL_L2, f"{what}: excess {excess:.3e}, rel_l2 {rl:.3e}"
 
@@ -114,8 +116,10 @@ def _check_against_rounding_model(got, x, w, cfg):
             _close_to_bf16_steps(got[key][l], m[key][l][:T], f"{key}{l} vs rounding model")
     _close_to_bf16_steps(got["k_g"], m["k_g"], "k_g vs rounding model")
     _close_to_bf16_steps(got["v_g"], m["v_g"], "v_g vs rounding model")
-    _close_to_bf16_steps(got["x_prefill"], m["x"][:T], "x prefill vs rounding model")
-    _close_to_bf16_steps(got["x_decode"], m["x"][T:], "x decode vs rounding model")
+    # x after the stack went through one bf16 rounding per residual addition
+    n_add = cfg.n_self + cfg.n_cross
+    _close_to_bf16_steps(got["x_prefill"], m["x"][:T], "x prefill vs rounding model", n_add)
+    _close_to_bf16_steps(got["x_decode"], m["x"][T:], "x decode vs rounding model", n_add)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -192,6 +196,7 @@ def test_tiny_stack_early_exit(cuda_lib, dtype):
     else:
         tol = dict(max_abs=sm.BF16_STACK_MAX_ABS, rel_l2=sm.BF16_STACK_REL_L2)
         # the residual stream at the bf16 bar, scaled to x's magnitude
-        _close_to_bf16_steps(got, sm.stack(x[:T], w, cfg, early_exit=True), "early exit vs rounding model")
-        _close_to_bf16_steps(got, full.float().cpu().numpy(), "early exit vs full prefill")
+        n_add = cfg.n_self + cfg.n_cross
+        _close_to_bf16_steps(got, sm.stack(x[:T], w, cfg, early_exit=True), "early exit vs rounding model", n_add)
+        _close_to_bf16_steps(got, full.float().cpu().numpy(), "early exit vs full prefill", n_add)
     assert_close(got, ref, dtype, "early exit vs oracle", **tol)
