@@ -111,9 +111,10 @@ yoco_status yoco_swa_prefill(const void *q, const void *k, const void *v, int32_
 
 /* Self-decoder sliding-window decode step over the ring.
  * q [B, Hq, D]; k_new, v_new [B, Hkv, D] (already blended); pos device int64
- * [B]: absolute position of the new token of each sequence.  The new K/V is
- * written to slot pos mod window (slot_pos updated), then the query attends
- * to every slot whose stored position lies in (pos - window, pos].
+ * [B]: absolute position of the new token of each sequence.  The query
+ * attends to the new token and to every other slot whose stored position lies
+ * in (pos - window, pos] -- the window after the new K/V replaces slot
+ * pos mod window -- and the new K/V is written there (slot_pos updated).
  * o [B, Hq, D].  workspace: yoco_swa_decode_workspace_size() bytes. */
 yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
                             const int64_t *pos, int32_t B, int32_t window, void *ring_k,

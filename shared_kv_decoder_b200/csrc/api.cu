@@ -218,7 +218,7 @@ yoco_status yoco_cross_decode(const void *q, const void *k_cache, const void *v_
     if (!workspace || !aligned16(workspace) || ws_bytes < pl.ws_bytes) return YOCO_ERR_WORKSPACE;
     DecodeArgs a;
     a.q = q; a.k = k_cache; a.v = v_cache; a.seq_start = seq_start; a.seq_len = seq_len;
-    a.slot_pos = nullptr; a.pos = nullptr; a.window = 0;
+    a.slot_pos = nullptr; a.pos = nullptr; a.window = 0; a.k_new = a.v_new = nullptr;
     a.cache_rows = cache_rows; a.max_len = max_len;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = lse; a.ws = workspace;
@@ -240,12 +240,12 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     if (!make_decode_plan(B, window, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl))
         return YOCO_ERR_UNSUPPORTED;
     if (!workspace || !aligned16(workspace) || ws_bytes < pl.ws_bytes) return YOCO_ERR_WORKSPACE;
-    st = from_cuda(launch_ring_write(k_new, v_new, pos, B, window, cfg->Hkv, cfg->D, cfg->dtype,
-                                     ring_k, ring_v, slot_pos, stream));
-    if (st != YOCO_OK) return st;
+    // the window read skips the new token's slot and the merge adds the new
+    // token and writes it into the ring (no separate ring-write kernel)
     DecodeArgs a;
     a.q = q; a.k = ring_k; a.v = ring_v; a.seq_start = nullptr; a.seq_len = nullptr;
     a.slot_pos = slot_pos; a.pos = pos; a.window = window;
+    a.k_new = k_new; a.v_new = v_new;
     a.cache_rows = (int64_t)B * window; a.max_len = window;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = nullptr; a.ws = workspace;
@@ -283,7 +283,7 @@ yoco_status yoco_cross_decode_i8(const void *q, const void *k_i8, const void *v_
     if (!workspace || !aligned16(workspace) || ws_bytes < pl.ws_bytes) return YOCO_ERR_WORKSPACE;
     DecodeArgs a;
     a.q = q; a.k = k_i8; a.v = v_i8; a.seq_start = seq_start; a.seq_len = seq_len;
-    a.slot_pos = nullptr; a.pos = nullptr; a.window = 0;
+    a.slot_pos = nullptr; a.pos = nullptr; a.window = 0; a.k_new = a.v_new = nullptr;
     a.cache_rows = cache_rows; a.max_len = max_len;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = lse; a.ws = workspace;
@@ -365,7 +365,7 @@ yoco_status yoco_debug_tile_schedule(int32_t kind, const yoco_attn_cfg *cfg, int
         s.n_qtiles = (int32_t)n_qtiles;
         const int grid = (int)(n_work < sms ? n_work : sms);
         s.band = sched::prefill_band(grid, (cfg->Hq / cfg->Hkv) / heads,
-                                     (int64_t)B * Tkv * cfg->Hkv * cfg->D * dtype_bytes(cfg->dtype) * 2);
+                                     (int64_t)B * Tkv * cfg->Hkv * cfg->D * dtype_bytes(cfg->dtype) * 2, window);
         for (int c = 0; c < grid; ++c)
             for (int r = 0;; ++r) {
                 const int w = sched::prefill_work_index(r, c, grid);

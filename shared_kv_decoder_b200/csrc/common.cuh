@@ -107,6 +107,12 @@ YOCO_DEV void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, uin
         : "memory");
 }
 
+// Ask L2 for a contiguous range (address and size multiples of 16 bytes); a
+// prefetch only warms the cache, so it may precede pdl_wait().
+YOCO_DEV void bulk_prefetch_l2(const void *src_gmem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------- programmatic dependent launch
 // The decode-step kernels (small projections, ring write, split decode,
 // merge) are launched with programmatic stream serialization (launch_pdl): the

@@ -51,7 +51,8 @@ constexpr int kTokPerWarp = 16;     // stage tokens handled by one consumer warp
 constexpr int kLanesPerTok = 8;
 constexpr int kTokPerPass = 32 / kLanesPerTok;
 constexpr int kPasses = kTokPerWarp / kTokPerPass;
-constexpr int64_t kTargetUnits = 148 * 12;
+constexpr int64_t kMinUnits = 148, kMaxUnits = 148 * 12;   // decode units per call (see make_decode_plan)
+constexpr int64_t kUnitBytes = (int64_t)2 << 20;
 
 struct DecodeKParams {
     const void *q, *k, *v;
@@ -186,6 +187,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
             const int r = lane % kLanesPerTok;
             const int64_t pos_b = p.pos ? p.pos[b] : 0;
             const int32_t *sp = p.slot_pos ? p.slot_pos + (int64_t)b * p.window + t0 : nullptr;
+            // ring mode: the slot the new token goes to is left out here (whatever it
+            // holds is replaced); the merge adds the new token from k_new / v_new
+            const int64_t new_slot = p.window > 0 ? ((pos_b % p.window) + p.window) % p.window : -1;
 
             float qf[G][DPL];
             {
@@ -227,7 +231,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_split_kernel(const D
                     bool vld = tok < n_tok;
                     if (vld && sp) {
                         const int32_t sp_t = sp[tok];
-                        vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window;
+                        vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window &&
+                              t0 + tok != new_slot;
                     }
                     valid[ps] = vld;
                     const uint4 *kr = reinterpret_cast<const uint4 *>(sk + ((int64_t)lt * p.Hkv + g) * D);
@@ -382,6 +387,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeKParams p) {
     pdl_trigger();
+    if (!p.seq_len && threadIdx.x == 32 * kConsumerWarps) {
+        // ring mode: every sequence has the same units and finding this CTA's
+        // first one reads no memory, so its K and V rows can be pulled into L2
+        // while the previous kernel (the ring write) finishes
+        const int64_t nu = sched::decode_units(p.window, p.split, p.n_split);
+        if ((int64_t)blockIdx.x < nu * p.B) {
+            const int64_t b = blockIdx.x / nu, t0 = (blockIdx.x % nu) * p.split;
+            const int64_t n_tok = min(p.split, (int64_t)p.window - t0);
+            const size_t off = ((size_t)b * p.window + t0) * p.Hkv * D * 2;
+            const uint32_t bytes = (uint32_t)(n_tok * p.Hkv * D * 2);
+            bulk_prefetch_l2(static_cast<const unsigned char *>(p.k) + off, bytes);
+            bulk_prefetch_l2(static_cast<const unsigned char *>(p.v) + off, bytes);
+        }
+    }
     pdl_wait();
     if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     static_assert(G >= 1 && G <= 8, "query heads per KV head");
@@ -455,6 +474,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const int t = lane & 3;
             const int64_t pos_b = p.pos ? p.pos[b] : 0;
             const int32_t *sp = p.slot_pos ? p.slot_pos + (int64_t)b * p.window + t0 : nullptr;
+            // ring mode: the slot the new token goes to is left out here (whatever it
+            // holds is replaced); the merge adds the new token from k_new / v_new
+            const int64_t new_slot = p.window > 0 ? ((pos_b % p.window) + p.window) % p.window : -1;
 
             uint32_t qa[D / 16][2];
             if (gq < G) {
@@ -538,7 +560,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                         bool vld = tok < n_tok;
                         if (vld && sp) {
                             const int32_t sp_t = sp[tok];
-                            vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window;
+                            vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window &&
+                                  t0 + tok != new_slot;
                         }
                         const float v = vld ? sc[n][e] * p.scale_log2 : -INFINITY;
                         pv[n][e] = v;
@@ -781,6 +804,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                     }
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                // the split below (x = rint(q * 16256 / amax), hi = rint(x / 128),
+                // lo = x - 128 hi) is restated in float32 by tests/test_i8_q_split.py,
+                // which checks the int8 ranges, the exact reconstruction and the
+                // half-step bound; keep the two in step
                 const float inv = amax > 0.f ? 16256.f / amax : 0.f;
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb)
@@ -1006,19 +1033,35 @@ __global__ void kv_quantize_i8_kernel(const T *k, const T *v, int64_t n, int Hkv
 }
 
 // Split merge: one CTA of kMergeWarps warps per (sequence, query head).  Warp
-// w takes the chunks of 32 partial entries w, w + kMergeWarps, ...; it forms
-// its own max, its lanes weight 32 entries at once and its weighted sum keeps
-// several partial rows in flight per lane; the warps' (max, sum, row) are then
-// combined through shared memory.  With one warp per (sequence, head), a
-// single long sequence left the merge with a few dozen warps to read
-// hundreds of partial rows each.
+// w takes the partial entries w, w + kMergeWarps, ... (each a 512-byte row
+// read by the whole warp), four at a time in flight, and keeps its own
+// running max, sum and weighted row (online rescaling); the warps' (max, sum,
+// row) are then combined through shared memory.  An earlier split of the
+// entries in runs of 32 per warp left all but one warp idle at the barrier
+// when a sequence had 32 partials (a 4 x 1024 sliding-window ring: 21 us per
+// merge under the profiler); with one warp per (sequence, head), a single
+// long sequence left the merge with a few dozen warps to read hundreds of
+// partial rows each.
 constexpr int kMergeWarps = 8;
+
+// The sliding-window decode's new token: its K/V (already blended) and query,
+// merged as one more partial, then written into the ring (NULL k_new: cross
+// decode, nothing to add).
+template <typename T>
+struct MergeNewToken {
+    const T *q, *k_new, *v_new;
+    const int64_t *pos;
+    T *ring_k, *ring_v;
+    int32_t *slot_pos;
+    int32_t Hkv;
+    float scale_log2;
+};
 
 template <typename T, int D>
 __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(
     const float *ws_o, const float *ws_ml, const int64_t *seq_start, const int32_t *seq_len, int32_t window,
     int32_t B, int32_t Hq, int64_t max_len, int64_t cache_rows, int64_t split, int64_t n_split, int32_t sub,
-    T *o, float *lse) {
+    T *o, float *lse, const MergeNewToken<T> nt) {
     constexpr int DPL = D / 32;
     __shared__ float s_m[kMergeWarps], s_l[kMergeWarps];
     __shared__ float s_acc[kMergeWarps][D];
@@ -1035,34 +1078,40 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(
     const int64_t n_e = n_s * sub;
     const int64_t e0 = (int64_t)b * n_split * sub;
 
-    float M = -INFINITY;
-    for (int64_t c = (int64_t)warp * 32; c < n_e; c += 32 * kMergeWarps) {
-        const int64_t e = c + lane;
-        if (e < n_e) M = fmaxf(M, ws_ml[((e0 + e) * Hq + h) * 2]);
-    }
-    M = warp_max(M);
-    float Lp = 0.f;
+    // warp w merges partials w, w + 8, ... with an online max (lane l holds
+    // dims l, l + 32, ...), four partials' loads in flight at a time
+    float M = -INFINITY, Lp = 0.f;
     float acc[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-    for (int64_t c = (int64_t)warp * 32; c < n_e; c += 32 * kMergeWarps) {
-        const int64_t e = c + lane;
-        float w = 0.f;
-        if (e < n_e) {
-            const float me = ws_ml[((e0 + e) * Hq + h) * 2];
-            w = (me == -INFINITY) ? 0.f : exp2f(me - M);
-            Lp = fmaf(ws_ml[((e0 + e) * Hq + h) * 2 + 1], w, Lp);
-        }
-        const int cnt = (int)min((int64_t)32, n_e - c);
-        const float *src = ws_o + ((e0 + c) * Hq + h) * D + lane;
-#pragma unroll 8
-        for (int k = 0; k < cnt; ++k) {
-            const float wk = __shfl_sync(0xffffffffu, w, k);
+    for (int64_t c = warp; c < n_e; c += 4 * kMergeWarps) {
+        float me[4], le[4], ov[4][DPL];
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wk, src[(int64_t)k * Hq * D + 32 * i], acc[i]);
+        for (int u = 0; u < 4; ++u) {
+            const int64_t e = c + (int64_t)u * kMergeWarps;
+            me[u] = -INFINITY;
+            le[u] = 0.f;
+            if (e < n_e) {
+                const float *ml = ws_ml + ((e0 + e) * Hq + h) * 2;
+                me[u] = ml[0];
+                le[u] = ml[1];
+                const float *src = ws_o + ((e0 + e) * Hq + h) * D + lane;
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) ov[u][i] = src[32 * i];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (me[u] == -INFINITY) continue;   // an empty partial (or none)
+            const float mn = fmaxf(M, me[u]);
+            const float fo = (M == -INFINITY) ? 0.f : exp2f(M - mn), fe = exp2f(me[u] - mn);
+            Lp = fmaf(Lp, fo, le[u] * fe);
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) acc[i] = fmaf(acc[i], fo, ov[u][i] * fe);
+            M = mn;
         }
     }
-    const float L = warp_sum(Lp);
+    const float L = Lp;   // the same in every lane of the warp
     if (lane == 0) {
         s_m[warp] = M;
         s_l[warp] = L;
@@ -1070,10 +1119,40 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(
 #pragma unroll
     for (int i = 0; i < DPL; ++i) s_acc[warp][lane + 32 * i] = acc[i];
     __syncthreads();
+    if (nt.k_new && h == 0 && warp >= 1) {
+        // the new token into the ring (the split kernel has read the ring;
+        // nothing else in this launch reads it): slot pos mod window
+        const int64_t p = nt.pos[b];
+        const int64_t slot = ((p % window) + window) % window;
+        const int64_t re = (int64_t)nt.Hkv * D;
+        T *dk = nt.ring_k + ((int64_t)b * window + slot) * re;
+        T *dv = nt.ring_v + ((int64_t)b * window + slot) * re;
+        for (int64_t e = threadIdx.x - 32; e < re; e += 32 * (kMergeWarps - 1)) {
+            dk[e] = nt.k_new[(int64_t)b * re + e];
+            dv[e] = nt.v_new[(int64_t)b * re + e];
+        }
+        if (threadIdx.x == 32) nt.slot_pos[(int64_t)b * window + slot] = (int32_t)p;
+    }
     if (warp != 0) return;
     float Mg = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kMergeWarps; ++w) Mg = fmaxf(Mg, s_m[w]);
+    // the new token's score (log2 domain) and value row, as one more partial
+    float m_new = -INFINITY, v_row[DPL];
+    if (nt.k_new) {
+        const int g = h / (Hq / nt.Hkv);
+        const T *qh = nt.q + ((int64_t)b * Hq + h) * D;
+        const T *kn = nt.k_new + ((int64_t)b * nt.Hkv + g) * D;
+        const T *vn = nt.v_new + ((int64_t)b * nt.Hkv + g) * D;
+        float dot = 0.f;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) {
+            dot = fmaf(to_f32(qh[lane + 32 * i]), to_f32(kn[lane + 32 * i]), dot);
+            v_row[i] = to_f32(vn[lane + 32 * i]);
+        }
+        m_new = warp_sum(dot) * nt.scale_log2;
+        Mg = fmaxf(Mg, m_new);
+    }
     float Lg = 0.f, out[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) out[i] = 0.f;
@@ -1083,6 +1162,12 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(
         Lg = fmaf(s_l[w], f, Lg);
 #pragma unroll
         for (int i = 0; i < DPL; ++i) out[i] = fmaf(s_acc[w][lane + 32 * i], f, out[i]);
+    }
+    if (nt.k_new) {
+        const float f = exp2f(m_new - Mg);
+        Lg += f;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) out[i] = fmaf(v_row[i], f, out[i]);
     }
     const float inv = Lg > 0.f ? 1.f / Lg : 0.f;
     T *dst = o + ((int64_t)b * Hq + h) * D;
@@ -1099,19 +1184,28 @@ bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dt
     DecodePlan pl;
     pl.stage_tokens = kRowsPerStage / Hkv;
     pl.sub = kConsumerWarps / Hkv;
-    // at least two pipeline stages per unit; small decodes (a sliding-window
-    // ring of 4 x 1024 slots) then spread over ~128 CTAs, each with its whole
-    // unit in flight, instead of 64 CTAs streaming four stages each
+    // Units: about kUnitBytes of K and V each, between one per SM and twelve
+    // per SM (many units balance ragged batches; few keep a short decode from
+    // paying per-unit overhead and a long merge), and at least two pipeline
+    // stages each.  A 16 x 64K-128K batch or a 1M-token sequence gets the
+    // maximum; a 4 x 1024 sliding-window ring ~128 units of two stages, each
+    // CTA with its whole unit in flight; one 32K-token sequence ~150 units.
+    const int64_t total = (int64_t)std::max(B, 1) * max_len;
+    const int64_t tok_bytes = 2 * (int64_t)Hkv * D * (int64_t)dtype_bytes(dtype);
+    const int64_t target = std::min<int64_t>(kMaxUnits, std::max<int64_t>(kMinUnits, total * tok_bytes / kUnitBytes));
     const int64_t min_split = 2 * pl.stage_tokens;
-    int64_t per = ((int64_t)std::max(B, 1) * max_len + kTargetUnits - 1) / kTargetUnits;
+    int64_t per = (total + target - 1) / target;
     per = ((per + pl.stage_tokens - 1) / pl.stage_tokens) * pl.stage_tokens;
     pl.split = std::max(per, min_split);
     pl.n_split = (max_len + pl.split - 1) / pl.split;
     // a stage holds 128 token-head rows of K and of V; the bf16 kernel adds
     // 1 KB so that its swizzled stages can start on a 1024-byte boundary
     const size_t stage_bytes = 2 * (size_t)kRowsPerStage * D * dtype_bytes(dtype);
-    pl.stages = (int)std::max<size_t>(1, std::min<size_t>(dtype == kBF16 ? 6 : 4,
-                                                          (200 * 1024) / stage_bytes));
+    // no deeper than a unit: a short unit's CTA then takes less shared memory
+    // and fits on an SM beside the kernel before it (programmatic launch)
+    pl.stages = (int)std::max<size_t>(1, std::min<size_t>(std::min<size_t>(dtype == kBF16 ? 6 : 4,
+                                                                           (200 * 1024) / stage_bytes),
+                                                          (size_t)(pl.split / pl.stage_tokens)));
     pl.smem_bytes = pl.stages * stage_bytes + 2 * pl.stages * sizeof(uint64_t) +
                     (dtype == kBF16 ? 1024 : 0);
     const size_t entries = (size_t)B * pl.n_split * pl.sub * Hq;
@@ -1182,9 +1276,21 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
     note_launches(2);
     if (e != cudaSuccess) return e;
     const int mgrid = (int)((int64_t)a.B * a.Hq);
+    MergeNewToken<T> nt = {};
+    if (a.k_new) {
+        nt.q = static_cast<const T *>(a.q);
+        nt.k_new = static_cast<const T *>(a.k_new);
+        nt.v_new = static_cast<const T *>(a.v_new);
+        nt.pos = a.pos;
+        nt.ring_k = static_cast<T *>(const_cast<void *>(a.k));
+        nt.ring_v = static_cast<T *>(const_cast<void *>(a.v));
+        nt.slot_pos = const_cast<int32_t *>(a.slot_pos);
+        nt.Hkv = a.Hkv;
+        nt.scale_log2 = a.scale * kLog2e;
+    }
     return launch_pdl(decode_merge_kernel<T, D>, dim3(mgrid), dim3(32 * kMergeWarps), 0, st, p.ws_o, p.ws_ml,
                       a.seq_start, a.seq_len, a.window, a.B, a.Hq, a.max_len, a.cache_rows, pl.split, pl.n_split,
-                      pl.sub, static_cast<T *>(a.o), a.lse);
+                      pl.sub, static_cast<T *>(a.o), a.lse, nt);
 }
 
 template <typename T, int D>
@@ -1266,7 +1372,7 @@ static cudaError_t launch_decode_i8_g(const DecodeArgs &a, const DecodePlan &pl,
     return launch_pdl(decode_merge_kernel<__nv_bfloat16, 128>, dim3((unsigned)((int64_t)a.B * a.Hq)),
                       dim3(32 * kMergeWarps), 0, st, p.ws_o, p.ws_ml, a.seq_start, a.seq_len, a.window, a.B,
                       a.Hq, a.max_len, a.cache_rows, pl.split, pl.n_split, pl.sub,
-                      static_cast<__nv_bfloat16 *>(a.o), a.lse);
+                      static_cast<__nv_bfloat16 *>(a.o), a.lse, MergeNewToken<__nv_bfloat16>{});
 }
 
 cudaError_t launch_decode_i8(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t st) {
@@ -1329,39 +1435,6 @@ cudaError_t launch_wait_timeout_probe(cudaStream_t st) {
 }
 
 // ------------------------------------------------------------------ ring
-template <typename T>
-__global__ void ring_write_kernel(const T *k_new, const T *v_new, const int64_t *pos, int32_t window,
-                                  int64_t row_elems, T *ring_k, T *ring_v, int32_t *slot_pos) {
-    const int b = blockIdx.x;
-    pdl_trigger();
-    pdl_wait();
-    const int64_t p = pos[b];
-    const int64_t slot = ((p % window) + window) % window;
-    T *dk = ring_k + ((int64_t)b * window + slot) * row_elems;
-    T *dv = ring_v + ((int64_t)b * window + slot) * row_elems;
-    for (int64_t i = threadIdx.x; i < row_elems; i += blockDim.x) {
-        dk[i] = k_new[(int64_t)b * row_elems + i];
-        dv[i] = v_new[(int64_t)b * row_elems + i];
-    }
-    if (threadIdx.x == 0) slot_pos[(int64_t)b * window + slot] = (int32_t)p;
-}
-
-cudaError_t launch_ring_write(const void *k_new, const void *v_new, const int64_t *pos, int32_t B,
-                              int32_t window, int Hkv, int D, int dtype, void *ring_k,
-                              void *ring_v, int32_t *slot_pos, cudaStream_t st) {
-    if (B == 0) return cudaSuccess;
-    const int64_t re = (int64_t)Hkv * D;
-    note_launches(1);
-    if (dtype == kBF16)
-        return launch_pdl(ring_write_kernel<__nv_bfloat16>, dim3(B), dim3(256), 0, st,
-                          static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new),
-                          pos, window, re, static_cast<__nv_bfloat16 *>(ring_k),
-                          static_cast<__nv_bfloat16 *>(ring_v), slot_pos);
-    return launch_pdl(ring_write_kernel<float>, dim3(B), dim3(256), 0, st, static_cast<const float *>(k_new),
-                      static_cast<const float *>(v_new), pos, window, re, static_cast<float *>(ring_k),
-                      static_cast<float *>(ring_v), slot_pos);
-}
-
 // Ring contents after a prefill of T tokens: slot s keeps the newest position
 // p < T with p mod window == s (slot_pos = p), or -1 and zeros.
 template <typename T>

@@ -40,6 +40,7 @@ struct DecodeArgs {
     const int32_t *seq_len;    // [B] (cross) or NULL (ring: window slots)
     const int32_t *slot_pos;   // ring only: [B, window]
     const int64_t *pos;        // ring only: [B]
+    const void *k_new, *v_new; // ring only: the new token's K / V [B, Hkv, D], merged and written by the merge
     int32_t window;            // ring only
     int64_t cache_rows;        // rows of the K and V cache buffers (ring: B * window)
     int64_t max_len;           // longest allowed sequence (the plan's max_len; ring: window)
@@ -50,11 +51,6 @@ struct DecodeArgs {
     void *ws;      // workspace
 };
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s);
-
-// SWA ring write of one new token per sequence.
-cudaError_t launch_ring_write(const void *k_new, const void *v_new, const int64_t *pos,
-                              int32_t B, int32_t window, int Hkv, int D, int dtype,
-                              void *ring_k, void *ring_v, int32_t *slot_pos, cudaStream_t s);
 
 // Ring fill after a prefill of T tokens.
 cudaError_t launch_ring_fill(const void *k, const void *v, int32_t B, int64_t T, int32_t window,

@@ -60,24 +60,16 @@ constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kBlk = 128 * 128;  // one [128 rows x 128 bytes] swizzled block
 
-// kStage: the sliding-window instantiation.  Its work tiles are short (nine
-// KV tiles at window 1024), so the output store is a large share of the time;
-// O goes through shared memory and a TMA store instead of one 16-byte global
-// store per thread and row (32 rows per warp instruction).  The 32 KB of
-// staging (one 64-column block per head) come from a third K stage, which a
-// window's K tiles -- shared by neighbouring query tiles, so found in L2 --
-// do not need.
-template <int D, bool kStage>
+template <int D>
 struct Smem {
     static constexpr int KB = D / 64;                  // 64-element column blocks
     static constexpr uint32_t TILE = (uint32_t)KB * kBlk;
-    static constexpr int KSTAGES = kStage ? 2 : 3;
+    static constexpr int KSTAGES = 3;
     static constexpr int VSTAGES = 2;
     static constexpr uint32_t Q = 0;                   // head A tile, then head B tile
     static constexpr uint32_t K = Q + 2 * TILE;
     static constexpr uint32_t V = K + KSTAGES * TILE;
-    static constexpr uint32_t OST = V + VSTAGES * TILE;   // O staging: one 64-column block per head
-    static constexpr uint32_t BAR = OST + (kStage ? 2 * kBlk : 0);
+    static constexpr uint32_t BAR = V + VSTAGES * TILE;
     static constexpr uint32_t BYTES = BAR + 256;
     static constexpr uint32_t ALLOC = BYTES + 1024;    // alignment slack
 };
@@ -112,35 +104,16 @@ YOCO_DEV bool waitw(uint64_t *bar, uint32_t parity) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, &g_status_prefill_pair));
 }
 
-// Named barrier 1 + hh over the 128 softmax threads of head hh, as a vote:
-// true when pred holds on every thread.  Every warp of the head reaches it
-// once per work tile, also after a bounded wait gave up, so no warp is left
-// waiting on one that has quit.
-YOCO_DEV bool head_vote_all(bool pred, int hh) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, 128, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(1 + hh)
-        : "memory");
-    return r != 0;
-}
-YOCO_DEV void head_sync(int hh) { asm volatile("bar.sync %0, 128;" ::"r"(1 + hh) : "memory"); }
-
 }  // namespace
 
-template <int D, bool kStage>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v,
-                             const __grid_constant__ CUtensorMap tm_o, const PairParams p) {
+                             const __grid_constant__ CUtensorMap tm_v, const PairParams p) {
     // once any CTA has recorded a timeout, the rest of the grid exits at once
     if (*(volatile unsigned int *)&g_status_prefill_pair) return;
-    using L = Smem<D, kStage>;
+    using L = Smem<D>;
     constexpr int KB = L::KB;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -395,6 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             e0 = tc::ex2(x0);
                             e1 = tc::ex2(x1);
                         } else {
+                            // a masked score (-inf) gives 2^-125 here, not 0: ~1e-38 of the
+                            // row's largest weight (>= 1 after the max), below any fp32 sum's
+                            // resolution; bound and -inf checked by the exp2 probe test
                             tc::exp2_pair_poly(x0, x1, e0, e1);
                         }
                         if (c & 2)
@@ -428,51 +404,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_before_sync();
                 mbar_arrive(&bars[kPFull + hh]);
             }
-            if constexpr (kStage) {
-                // the head's four warps go on together or quit together
-                if (ok) ok = waitw(&bars[kODone + hh], (g - 1) & 1);
-                if (!head_vote_all(ok, hh)) { ok = false; break; }
-                tc::fence_after_sync();
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                // per 64-column block: TMEM -> registers -> the head's staging
-                // block in the TMA's 128-byte swizzle (row r's 16-byte chunk j at
-                // j ^ (r & 7): eight distinct bank groups per eight rows) -> one
-                // TMA store; rows past Tq are clipped by the store
-                uint8_t *ost = sbase + L::OST + hh * kBlk;
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (r == 0) tc::bulk_wait_read_all();   // the previous store has read the block
-                    head_sync(hh);
-#pragma unroll
-                    for (int c = 0; c < 64; c += 32) {
-                        float o[32];
-                        tc::tmem_ld32(tO + kb * 64 + c, o);
-                        tc::wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            uint4 wv;
-                            wv.x = tc::pack_bf16x2(o[8 * e] * inv, o[8 * e + 1] * inv);
-                            wv.y = tc::pack_bf16x2(o[8 * e + 2] * inv, o[8 * e + 3] * inv);
-                            wv.z = tc::pack_bf16x2(o[8 * e + 4] * inv, o[8 * e + 5] * inv);
-                            wv.w = tc::pack_bf16x2(o[8 * e + 6] * inv, o[8 * e + 7] * inv);
-                            const int j = c / 8 + e;
-                            *reinterpret_cast<uint4 *>(ost + r * 128 + ((j ^ (r & 7)) << 4)) = wv;
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    head_sync(hh);
-                    if (r == 0) {
-                        tc::tma_store_4d(&tm_o, base + L::OST + hh * kBlk, kb * 64, h, (int)x.i0, x.b);
-                        tc::bulk_commit_group();
-                    }
-                }
-                if (p.lse && i < p.s.Tq)
-                    p.lse[((int64_t)x.b * p.s.Hq + h) * p.s.Tq + i] =
-                        l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
-                tc::fence_before_sync();
-                mbar_arrive(&bars[kOFree + hh]);
-                continue;
-            }
             if (!ok) break;
             // epilogue: the last P.V of this work tile, then O / l -> global
             if (!waitw(&bars[kODone + hh], (g - 1) & 1)) { ok = false; break; }
@@ -504,9 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) *abort_flag = 1;
         tc::wait_st();  // no TMEM store may be in flight when TMEM is freed
-        if constexpr (kStage) {
-            if (r == 0) tc::bulk_wait_all();  // the output stores are done before the CTA exits
-        }
     }
 
     tc::fence_before_sync();
@@ -528,11 +456,11 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t B, int64_t T, int64_t H, 
     return encode_bf16_map_4d(m, ptr, dims, strides, box);
 }
 
-template <int D, bool kStage>
+template <int D>
 cudaError_t launch_pair_d(const PrefillArgs &a, cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv;
     if (!make_map(&mq, a.q, a.B, a.Tq, a.Hq, D) || !make_map(&mk, a.k, a.B, a.Tkv, a.Hkv, D) ||
-        !make_map(&mv, a.v, a.B, a.Tkv, a.Hkv, D) || !make_map(&mo, a.o, a.B, a.Tq, a.Hq, D))
+        !make_map(&mv, a.v, a.B, a.Tkv, a.Hkv, D))
         return cudaErrorNotSupported;
     PairParams p;
     p.s.B = a.B; p.s.Hq = a.Hq; p.s.Hkv = a.Hkv;
@@ -545,13 +473,13 @@ cudaError_t launch_pair_d(const PrefillArgs &a, cudaStream_t st) {
     p.s.n_qtiles = (int)n_qtiles;
     p.n_work = (int)n_work;
     const int grid = (int)std::min<int64_t>(n_work, device_sm_count());
-    p.s.band = sched::prefill_band(grid, (a.Hq / a.Hkv) / 2, (int64_t)a.B * a.Tkv * a.Hkv * D * 2 * 2);
-    auto kern = attn_prefill_pair_kernel<D, kStage>;
+    p.s.band = sched::prefill_band(grid, (a.Hq / a.Hkv) / 2, (int64_t)a.B * a.Tkv * a.Hkv * D * 2 * 2, a.window);
+    auto kern = attn_prefill_pair_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Smem<D, kStage>::ALLOC);
+                                         (int)Smem<D>::ALLOC);
     if (e != cudaSuccess) return e;
     note_launches(1);
-    kern<<<grid, kThreads, Smem<D, kStage>::ALLOC, st>>>(mq, mk, mv, mo, p);
+    kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
@@ -560,9 +488,8 @@ cudaError_t launch_pair_d(const PrefillArgs &a, cudaStream_t st) {
 cudaError_t launch_prefill_pair(const PrefillArgs &a, cudaStream_t st) {
     if (a.dtype != kBF16 || !sched::prefill_pairs_heads(a.Hq, a.Hkv)) return cudaErrorNotSupported;
     if (a.B == 0 || a.Tq == 0) return cudaSuccess;
-    const bool window = a.window > 0;
-    if (a.D == 128) return window ? launch_pair_d<128, true>(a, st) : launch_pair_d<128, false>(a, st);
-    if (a.D == 64) return window ? launch_pair_d<64, true>(a, st) : launch_pair_d<64, false>(a, st);
+    if (a.D == 128) return launch_pair_d<128>(a, st);
+    if (a.D == 64) return launch_pair_d<64>(a, st);
     return cudaErrorNotSupported;
 }
 

@@ -341,6 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         e0 = tc::ex2(x0);
                         e1 = tc::ex2(x1);
                     } else {
+                        // a masked score (-inf) gives 2^-125 here, not 0: ~1e-38 of the
+                        // row's largest weight (>= 1 after the max), below any fp32 sum's
+                        // resolution; bound and -inf checked by the exp2 probe test
                         tc::exp2_pair_poly(x0, x1, e0, e1);
                     }
                     if (c & 2)
@@ -444,7 +447,7 @@ cudaError_t launch_tc_d(const PrefillArgs &a, cudaStream_t st) {
     p.s.n_qtiles = (int)n_qtiles;
     p.n_work = (int)n_work;
     const int grid = (int)std::min<int64_t>(n_work, device_sm_count());
-    p.s.band = sched::prefill_band(grid, a.Hq / a.Hkv, (int64_t)a.B * a.Tkv * a.Hkv * D * 2 * 2);
+    p.s.band = sched::prefill_band(grid, a.Hq / a.Hkv, (int64_t)a.B * a.Tkv * a.Hkv * D * 2 * 2, a.window);
     auto kern = attn_prefill_tc_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Smem<D>::ALLOC);

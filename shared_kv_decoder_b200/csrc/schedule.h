@@ -63,9 +63,13 @@ constexpr int64_t kPrefillBandMinKVBytes = (int64_t)32 << 20;
 constexpr int kPrefillBandStreams = YOCO_BAND_STREAMS;
 
 // Query tiles per band for a grid of `grid` CTAs, `per` work tiles per (query
-// tile, stream) and kv_bytes of K and V over all streams.
-YOCO_HD int32_t prefill_band(int grid, int per, int64_t kv_bytes) {
-    if (kv_bytes <= kPrefillBandMinKVBytes) return 1;
+// tile, stream), kv_bytes of K and V over all streams and the attention
+// window.  A sliding window needs no bands: its work tiles read only the
+// window's few KV tiles, which neighbouring query tiles share, so each tile
+// comes from DRAM about once in any order, and one stream per round would
+// only crowd all CTAs onto the same few tiles.
+YOCO_HD int32_t prefill_band(int grid, int per, int64_t kv_bytes, int32_t window) {
+    if (window > 0 || kv_bytes <= kPrefillBandMinKVBytes) return 1;
     const int b = per > 0 ? grid / (per * kPrefillBandStreams) : 1;
     return b > 0 ? b : 1;
 }
