@@ -425,7 +425,7 @@ yoco_status yoco_get_device_status(cudaStream_t stream) {
     const cudaError_t e = cudaStreamSynchronize(stream);
     const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc() |
                            read_and_clear_status_prefill_pair() | read_and_clear_status_project_tc() |
-                           read_and_clear_status_gret_tc();
+                           read_and_clear_status_gret_tc() | read_and_clear_status_linear();
     if (s & 1u) return YOCO_ERR_TIMEOUT;
     if (s & 2u) return YOCO_ERR_INVALID;
     return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;

@@ -132,6 +132,7 @@ unsigned int read_and_clear_status_prefill_tc();
 unsigned int read_and_clear_status_prefill_pair();
 unsigned int read_and_clear_status_gret_tc();
 unsigned int read_and_clear_status_project_tc();
+unsigned int read_and_clear_status_linear();
 
 int device_sm_count();
 

@@ -15,6 +15,8 @@
 // staged into shared memory.  Output columns below split_col go to out0, the
 // rest to out1 (K and V of one fused [K | V] weight); dst_rows, when given,
 // scatters output rows (appending to the shared cache).
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -115,20 +117,26 @@ __global__ void __launch_bounds__(256) linear_simt_kernel(const LinearArgs a) {
 }
 
 // A few rows (decode-step projections, n <= 16): the weight is read once,
-// from HBM, and all of it is in flight at once.  One output column per warp
-// (256 CTAs for a 2048-wide [K | V]); each lane first asks L2 for its slice of
-// the column's weight row, waits for the previous kernel (pdl_wait), then
-// issues every 16-byte load of that slice before using any.  The CTA stages
-// its x rows in shared memory and takes each row's LayerNorm statistics in
-// one pass shifted by the row's first value (mean and variance of x - x_0).
-// LayerNorm is folded out of the dot products:
+// from HBM, and all of a CTA's share is in flight at once.  A CTA owns eight
+// output columns (one per warp; 256 CTAs for a 2048-wide [K | V]).  One thread
+// issues bulk copies of the CTA's eight weight rows and of the n x rows into
+// shared memory, all completing on one mbarrier, so the bytes in flight cost
+// no registers; before that, while the previous kernel finishes, every warp
+// asks L2 for its weight row.  Each row's LayerNorm statistics come from one
+// pass over its staged copy, shifted by the row's first value, and LayerNorm
+// is folded out of the dot products,
 //   N(x) . w = rstd (x . w - mean * sum(w)),
 // so the inner loop is one packed f32x2 FMA per two weights and row.  NR
-// bounds the row count at compile time (4, 8 or 16): a loop unrolled for 16
-// rows when 4 are used ran ~4000 instructions per warp, bound by instruction
-// fetch, for 17 us where the weight streams in a few.
-constexpr int kSmallRows = 16, kSmallWarps = 8, kSmallChunks = 16;
+// bounds the row count at compile time (4, 8 or 16).
+// Earlier versions, measured on a 4 x 4096 -> 2048 projection: four columns
+// per warp and 64 CTAs, ~16 us (too few loads in flight); one column per warp
+// with the weight in registers and the loop unrolled for 16 rows, 17 us
+// (instruction-fetch bound); the same unrolled for 4 rows, 10 us (latency of
+// each warp's own dependent loads, 0.4 eligible warps per cycle).
+constexpr int kSmallRows = 16, kSmallWarps = 8;
 constexpr size_t kSmallMaxSmem = 200 * 1024;
+
+static __device__ unsigned int g_status_linear;
 
 // 8 bf16 (one 16-byte chunk) as four packed fp32 pairs; 4 fp32 as two
 template <typename T> YOCO_DEV void chunk_pairs(const uint4 &c, uint64_t *p);
@@ -169,135 +177,103 @@ YOCO_DEV float hsum2(uint64_t a) {
     return lo + hi;
 }
 
-// x staged in shared memory: fp32 for up to four rows (converted once, so the
-// inner loop reads ready pairs), else in its own type
-template <typename T, int NR> struct SmallStage { using type = T; };
-template <> struct SmallStage<__nv_bfloat16, 4> { using type = float; };
+// shared memory of the few-row projection: the CTA's weight rows, then the x
+// rows (both [rows][d_in] of T), then the mbarrier
+static inline size_t small_smem_bytes(int n, int d_in, int elem) {
+    return ((size_t)(kSmallWarps + n) * d_in * elem + 15) / 16 * 16 + 16;
+}
 
 template <typename T, int NR>
 __global__ void __launch_bounds__(32 * kSmallWarps, 2) linear_small_kernel(const LinearArgs a) {
-    using XS = typename SmallStage<T, NR>::type;
-    constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte chunk of T
+    constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte chunk
     constexpr int NP = VEC / 2;          // packed pairs per chunk
-    constexpr int XC = sizeof(XS) / sizeof(T);  // 16-byte staged chunks per chunk of T
-    extern __shared__ uint4 xs4[];       // the n x rows, [n][d_in] of XS
+    extern __shared__ __align__(16) uint4 sm4[];
     __shared__ float mu[NR], rs[NR];
     const T *w = static_cast<const T *>(a.w);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = (int)a.n;
     const int row_chunks = a.d_in / VEC;            // 16-byte chunks per row
-    const int c = blockIdx.x * kSmallWarps + warp;  // this warp's output column
-    const uint4 *wrow = reinterpret_cast<const uint4 *>(w + (int64_t)min(c, a.d_out - 1) * a.d_in);
+    const int c0 = blockIdx.x * kSmallWarps;        // the CTA's first output column
+    const int n_cols = min(kSmallWarps, a.d_out - c0);
+    const int c = c0 + warp;                        // this warp's output column
+    uint4 *ws4 = sm4;                               // [n_cols][row_chunks]
+    uint4 *xs4 = sm4 + (size_t)kSmallWarps * row_chunks;   // [n][row_chunks]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(xs4 + (size_t)n * row_chunks);
+    const uint32_t row_bytes = (uint32_t)row_chunks * 16u;
+
     // while the previous kernel finishes: ask L2 for this warp's weight row
     // (a prefetch only warms the cache; nothing is read before pdl_wait)
     pdl_trigger();
-    for (int ch = lane * 8; ch < row_chunks; ch += 256) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + ch));
+    if (warp < n_cols) {
+        const uint4 *wrow = reinterpret_cast<const uint4 *>(w + (int64_t)c * a.d_in);
+        for (int ch = lane * 8; ch < row_chunks; ch += 256) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + ch));
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
     pdl_wait();
-    uint4 wr[kSmallChunks];
-#pragma unroll
-    for (int k = 0; k < kSmallChunks; ++k)
-        if (lane + 32 * k < row_chunks) wr[k] = wrow[lane + 32 * k];
-    // stage x (every thread, eight 16-byte loads in flight each), then the
-    // statistics of each row
-    const uint4 *x4 = static_cast<const uint4 *>(a.x);
-    const int total = n * row_chunks;
-    for (int i0 = 0; i0 < total; i0 += 8 * (int)blockDim.x) {
-        uint4 t[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
-            if (i < total) t[u] = x4[i];
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
-            if (i < total) {
-                if constexpr (XC == 1) {
-                    xs4[i] = t[u];
-                } else {   // bf16 -> fp32: one chunk of T becomes two staged chunks
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(n_cols + n) * row_bytes);
+        for (int j = 0; j < n_cols; ++j)
+            bulk_g2s(ws4 + (size_t)j * row_chunks, w + (int64_t)(c0 + j) * a.d_in, row_bytes, bar);
+        for (int r = 0; r < n; ++r)
+            bulk_g2s(xs4 + (size_t)r * row_chunks, static_cast<const T *>(a.x) + (int64_t)r * a.d_in, row_bytes, bar);
+    }
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0, &g_status_linear));
+    // the row statistics (warp r: row r)
+    if (ok) {
+        for (int r = warp; r < n; r += kSmallWarps) {
+            float mean = 0.f, rstd = 1.f;
+            if (a.apply_ln) {
+                const float x0 = to_f32(reinterpret_cast<const T *>(xs4 + (size_t)r * row_chunks)[0]);
+                const uint64_t sh = pack2(-x0, -x0);
+                uint64_t s1 = 0, s2 = 0;
+                for (int ch = lane; ch < row_chunks; ch += 32) {
                     uint64_t p[NP];
-                    chunk_pairs<T>(t[u], p);
-                    uint4 lo, hi;
-                    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo.x), "=r"(lo.y) : "l"(p[0]));
-                    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo.z), "=r"(lo.w) : "l"(p[1]));
-                    asm("mov.b64 {%0, %1}, %2;" : "=r"(hi.x), "=r"(hi.y) : "l"(p[2]));
-                    asm("mov.b64 {%0, %1}, %2;" : "=r"(hi.z), "=r"(hi.w) : "l"(p[3]));
-                    xs4[2 * i] = lo;
-                    xs4[2 * i + 1] = hi;
-                }
-            }
-        }
-    }
-    __syncthreads();
-    // the NP pairs of chunk ch of staged row r
-    auto x_pairs = [&](int r, int ch, uint64_t *p) {
-        if constexpr (XC == 1) {
-            chunk_pairs<T>(xs4[(int64_t)r * row_chunks + ch], p);
-        } else {
-            const uint4 lo = xs4[2 * ((int64_t)r * row_chunks + ch)], hi = xs4[2 * ((int64_t)r * row_chunks + ch) + 1];
-            asm("mov.b64 %0, {%1, %2};" : "=l"(p[0]) : "r"(lo.x), "r"(lo.y));
-            asm("mov.b64 %0, {%1, %2};" : "=l"(p[1]) : "r"(lo.z), "r"(lo.w));
-            asm("mov.b64 %0, {%1, %2};" : "=l"(p[2]) : "r"(hi.x), "r"(hi.y));
-            asm("mov.b64 %0, {%1, %2};" : "=l"(p[3]) : "r"(hi.z), "r"(hi.w));
-        }
-    };
-    for (int r = warp; r < n; r += kSmallWarps) {
-        float mean = 0.f, rstd = 1.f;
-        if (a.apply_ln) {
-            const float x0 = to_f32(static_cast<const T *>(a.x)[(int64_t)r * a.d_in]);
-            const uint64_t sh = pack2(-x0, -x0);
-            uint64_t s1 = 0, s2 = 0;
-            for (int ch = lane; ch < row_chunks; ch += 32) {
-                uint64_t p[NP];
-                x_pairs(r, ch, p);
+                    chunk_pairs<T>(xs4[(size_t)r * row_chunks + ch], p);
 #pragma unroll
-                for (int i = 0; i < NP; ++i) {
-                    const uint64_t d = add2(p[i], sh);
-                    s1 = add2(s1, d);
-                    s2 = fma2(d, d, s2);
+                    for (int i = 0; i < NP; ++i) {
+                        const uint64_t d = add2(p[i], sh);
+                        s1 = add2(s1, d);
+                        s2 = fma2(d, d, s2);
+                    }
                 }
+                const float m1 = warp_sum(hsum2(s1)) / (float)a.d_in;   // mean of x - x0
+                const float var = fmaxf(warp_sum(hsum2(s2)) / (float)a.d_in - m1 * m1, 0.f);
+                mean = x0 + m1;
+                rstd = rsqrtf(var + a.eps);
             }
-            const float m1 = warp_sum(hsum2(s1)) / (float)a.d_in;          // mean of x - x0
-            const float var = fmaxf(warp_sum(hsum2(s2)) / (float)a.d_in - m1 * m1, 0.f);
-            mean = x0 + m1;
-            rstd = rsqrtf(var + a.eps);
-        }
-        if (lane == 0) {
-            mu[r] = mean;
-            rs[r] = rstd;
+            if (lane == 0) {
+                mu[r] = mean;
+                rs[r] = rstd;
+            }
         }
     }
     __syncthreads();
-    if (c >= a.d_out) return;
+    if (!ok || warp >= n_cols) return;
     uint64_t acc[NR], wsum = 0;
 #pragma unroll
     for (int r = 0; r < NR; ++r) acc[r] = 0;
-    for (int k0 = 0; k0 * 32 < row_chunks; k0 += kSmallChunks) {
-        if (k0 > 0) {  // rows longer than 16 chunks per lane: the next block of loads
+    const uint4 *wr = ws4 + (size_t)warp * row_chunks;
+#pragma unroll 4
+    for (int ch = lane; ch < row_chunks; ch += 32) {
+        uint64_t wp[NP];
+        chunk_pairs<T>(wr[ch], wp);
 #pragma unroll
-            for (int k = 0; k < kSmallChunks; ++k)
-                if (lane + 32 * (k0 + k) < row_chunks) wr[k] = wrow[lane + 32 * (k0 + k)];
-        }
+        for (int i = 0; i < NP; ++i) wsum = add2(wsum, wp[i]);
 #pragma unroll
-        for (int k = 0; k < kSmallChunks; ++k) {
-            const int ch = lane + 32 * (k0 + k);
-            if (ch >= row_chunks) break;
-            uint64_t wp[NP];
-            chunk_pairs<T>(wr[k], wp);
+        for (int r = 0; r < NR; ++r) {
+            if (r < n) {
+                uint64_t xp[NP];
+                chunk_pairs<T>(xs4[(size_t)r * row_chunks + ch], xp);
 #pragma unroll
-            for (int i = 0; i < NP; ++i) wsum = add2(wsum, wp[i]);
-#pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                if (r < n) {
-                    uint64_t xp[NP];
-                    x_pairs(r, ch, xp);
-#pragma unroll
-                    for (int i = 0; i < NP; ++i) acc[r] = fma2(xp[i], wp[i], acc[r]);
-                }
+                for (int i = 0; i < NP; ++i) acc[r] = fma2(xp[i], wp[i], acc[r]);
             }
         }
     }
-    const float ws = warp_sum(hsum2(wsum));
+    const float wsm = warp_sum(hsum2(wsum));
     const int w1 = a.d_out - a.split_col;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
@@ -305,7 +281,7 @@ __global__ void __launch_bounds__(32 * kSmallWarps, 2) linear_small_kernel(const
         const float tot = warp_sum(hsum2(acc[r]));
         if (lane != r) continue;
         const int64_t dr = a.dst_rows ? a.dst_rows[r] : r;
-        float val = a.apply_ln ? rs[r] * (tot - mu[r] * ws) : tot;
+        float val = a.apply_ln ? rs[r] * (tot - mu[r] * wsm) : tot;
         if (c < a.split_col) {
             if (a.base0) val = fmaf(a.w0, to_f32(static_cast<const T *>(a.base0)[(int64_t)r * a.split_col + c]), val);
             static_cast<T *>(a.out0)[dr * a.split_col + c] = from_f32<T>(val);
@@ -318,30 +294,28 @@ __global__ void __launch_bounds__(32 * kSmallWarps, 2) linear_small_kernel(const
 }
 
 template <typename T, int NR>
-static cudaError_t launch_small(const LinearArgs &a, size_t xs_bytes, cudaStream_t st) {
+static cudaError_t launch_small(const LinearArgs &a, size_t smem, cudaStream_t st) {
     auto kern = linear_small_kernel<T, NR>;
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallMaxSmem);
     if (e != cudaSuccess) return e;
     note_launches(1);
     const int grid = (a.d_out + kSmallWarps - 1) / kSmallWarps;
-    return launch_pdl(kern, dim3(grid), dim3(32 * kSmallWarps), xs_bytes, st, a);
+    return launch_pdl(kern, dim3(grid), dim3(32 * kSmallWarps), smem, st, a);
 }
 
 template <typename T>
-static cudaError_t launch_small_t(const LinearArgs &a, size_t xs_bytes, cudaStream_t st) {
-    // up to four rows are staged in fp32: twice the bytes of bf16
-    if (a.n <= 4) return launch_small<T, 4>(a, xs_bytes * sizeof(typename SmallStage<T, 4>::type) / sizeof(T), st);
-    if (a.n <= 8) return launch_small<T, 8>(a, xs_bytes, st);
-    return launch_small<T, 16>(a, xs_bytes, st);
+static cudaError_t launch_small_t(const LinearArgs &a, size_t smem, cudaStream_t st) {
+    if (a.n <= 4) return launch_small<T, 4>(a, smem, st);
+    if (a.n <= 8) return launch_small<T, 8>(a, smem, st);
+    return launch_small<T, 16>(a, smem, st);
 }
 
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t st) {
     if (a.n == 0 || a.d_out == 0) return cudaSuccess;
     const int vec = a.dtype == kBF16 ? 8 : 4;
-    const size_t xs_bytes = (size_t)a.n * a.d_in * dtype_bytes(a.dtype);
-    const size_t staged = (a.n <= 4 && a.dtype == kBF16) ? 2 * xs_bytes : xs_bytes;   // fp32 staging
-    if (a.n <= kSmallRows && a.d_in % vec == 0 && staged <= kSmallMaxSmem)
-        return a.dtype == kBF16 ? launch_small_t<__nv_bfloat16>(a, xs_bytes, st) : launch_small_t<float>(a, xs_bytes, st);
+    const size_t smem = small_smem_bytes((int)std::min<int64_t>(a.n, kSmallRows), a.d_in, (int)dtype_bytes(a.dtype));
+    if (a.n <= kSmallRows && a.d_in % vec == 0 && smem <= kSmallMaxSmem)
+        return a.dtype == kBF16 ? launch_small_t<__nv_bfloat16>(a, smem, st) : launch_small_t<float>(a, smem, st);
     dim3 grid((unsigned)((a.d_out + kLinBN - 1) / kLinBN), (unsigned)((a.n + kLinBM - 1) / kLinBM));
     note_launches(1);
     if (a.dtype == kBF16)
@@ -349,6 +323,13 @@ cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t st) {
     else
         linear_simt_kernel<float><<<grid, 256, 0, st>>>(a);
     return cudaGetLastError();
+}
+
+unsigned int read_and_clear_status_linear() {
+    unsigned int h = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&h, g_status_linear, sizeof(h)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_status_linear, &z, sizeof(z));
+    return h;
 }
 
 }  // namespace yoco

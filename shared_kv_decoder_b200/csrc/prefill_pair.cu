@@ -173,18 +173,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         (int)x.i0, x.b, &bars[kQFull + hh]);
                 }
                 if (!ok) { *abort_flag = 1; ++k; break; }
-                // pull the next work tile's Q tiles into L2 now: their loads,
-                // issued once this work tile's last S MMAs finish, then come
-                // from L2 instead of HBM while the tensor core has only the
-                // last P.V MMAs left to run (short work tiles -- the sliding
-                // window's nine KV tiles -- otherwise wait on that latency)
-                const int wn = sched::prefill_work_index(r + 1, blockIdx.x, gridDim.x);
-                if (wn < p.n_work) {
-                    const sched::PrefillWork xn = sched::prefill_pair_work(p.s, wn);
-                    for (int hh = 0; hh < 2; ++hh)
-                        for (int kb = 0; kb < KB; ++kb)
-                            tc::tma_prefetch_4d(&tm_q, kb * 64, xn.h + hh, (int)xn.i0, xn.b);
-                }
             }
             // drain: the last copies issued must land before this CTA may exit
             if (k > 0)
