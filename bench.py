@@ -76,7 +76,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer",
                                        "gret", "gret_decode", "decode_i8_layer", "gret1", "decode_i8",
-                                       "long_prefill", "long_decode", "swa_decode_layer"],
+                                       "long_prefill", "long_decode", "swa_decode_layer", "proj_small"],
                     default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
@@ -100,14 +100,14 @@ def load_peaks():
 # and the report carries null instead.
 _CSRC = "shared_kv_decoder_b200/csrc/"
 TRAFFIC = {
-    # attn_prefill_pair_kernel<128>, T=32768: 1.814138 GB read + 239.481088 MB written
-    "prefill": {"bytes": 1814138000 + 239481088,
+    # attn_prefill_pair_kernel<128>, T=32768: 568.586 MB read + 232.266 MB written
+    "prefill": {"bytes": 568585984 + 232265984,
                 "sources": ["prefill_pair.cu", "schedule.h", "tc.cuh", "common.cuh"],
-                "sha256": "e8e2369b9f4bb812ccec27be99b70749aad412c78e133211f37f9a70b6043836"},
-    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416142 GB read + 25.513984 MB written
-    "decode": {"bytes": 6416142000 + 25513984,
+                "sha256": "992d6629df8f74de25fecff8eeeccf505c37e589717e1947e48a9fdae3a4bb46"},
+    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416115 GB read + 24.940 MB written
+    "decode": {"bytes": 6416114944 + 24940032,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
-               "sha256": "e6b1985a87f4803a25388c0999f795684d1fb490cbdd04333d8a8d63e6e3014d"},
+               "sha256": "9347f56122f9323d39e6922f7f7d6aa296a79a7a84666d1cf4a4b4b90a1885ee"},
 }
 
 
@@ -771,7 +771,9 @@ def run_case(args):
                chunk of the causal prefill over the whole prefix / one decode step of one
                sequence over all 1,048,576 rows
       swa_decode_layer  one sliding-window decode call at the self-decoder's shape (batch 4,
-               window 1024: ring write + window attention + merge over 16.8 MB of ring)
+               window 1024: window attention + merge with the new token's ring write, 16.8 MB of ring)
+      proj_small  the decode step's K/V projection of 4 tokens, d=4096 -> 2048, with the blend (16.8 MB
+               of weights)
     Prints one JSON line with the mean launch time and the work rate."""
     import torch
     import shared_kv_decoder_b200 as yoco
@@ -803,6 +805,20 @@ def run_case(args):
         v = wl.normal((1, T, Hkv, D), 9, bf, dev); o = torch.empty_like(q)
         fn = lambda: yoco.swa_prefill(q, k, v, Wn, o=o)
         work, unit = prefill_flops_per_layer(T, Hq, D, 0, Wn), "TFLOP/s"
+    elif args.case == "proj_small":
+        # the self-decoder decode step's projection: 4 new tokens, d=4096 -> [K | V] 2048, with the blend;
+        # 16 weights (one per layer) used in turn, so each launch reads its weight from HBM
+        n, d = SWA["B"], SWA["d"]
+        ws_ = [wl.normal((2 * Hkv * D, d), 30 + l, bf, dev, std=d ** -0.5) for l in range(16)]
+        x = wl.normal((n, d), 10, bf, dev)
+        kb = wl.normal((n, Hkv, D), 12, bf, dev); vb = wl.normal((n, Hkv, D), 13, bf, dev)
+        ko = torch.empty_like(kb); vo = torch.empty_like(vb)
+        turn = [0]
+
+        def fn():
+            turn[0] += 1
+            yoco.kv_project_blend(x, ws_[turn[0] % 16], Hkv, D, kb, vb, 0.5, 0.5, k_out=ko, v_out=vo)
+        work, unit = 2.0 * Hkv * D * d * 2, "GB/s"
     elif args.case == "swa_decode_layer":
         B, T, Wn = SWA["B"], 4096, SWA["W"]
         k = wl.normal((B, T, Hkv, D), 8, bf, dev); v = wl.normal((B, T, Hkv, D), 9, bf, dev)

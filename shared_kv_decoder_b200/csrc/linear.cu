@@ -293,6 +293,143 @@ __global__ void __launch_bounds__(32 * kSmallWarps, 2) linear_small_kernel(const
     }
 }
 
+// The same projection on the tensor cores, for bf16, n <= 15 rows and d_in a
+// multiple of 128: a CTA's eight output columns are one m16n8 MMA tile (A = the
+// n x rows, padded with zeros and a row of ones at row 15, whose products are
+// the columns' weight sums for the folded LayerNorm; B = the eight weight
+// rows), the CTA's eight warps split K and add their partial tiles through
+// shared memory.  The weight and x rows are bulk-copied in four K-quarters on
+// four mbarriers, so a warp starts on its quarter as soon as it lands.  Rows
+// are padded by 16 bytes in shared memory, so the eight rows one fragment load
+// touches fall in distinct banks.
+constexpr int kFewMaxRows = 15;   // row 15 carries the ones
+
+YOCO_DEV void mma_bf16_16816(float *c, const uint32_t *a, const uint32_t *b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+static inline size_t few_tc_smem_bytes(int n, int d_in) {
+    return (size_t)(kSmallWarps + n) * (d_in + 8) * 2 + (size_t)kSmallWarps * 16 * 8 * 4 + 4 * 8;
+}
+
+__global__ void __launch_bounds__(32 * kSmallWarps, 2) linear_few_tc_kernel(const LinearArgs a) {
+    typedef __nv_bfloat16 T;
+    extern __shared__ __align__(16) unsigned char sm[];
+    __shared__ float mu[kFewMaxRows], rs[kFewMaxRows];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int n = (int)a.n, K = a.d_in, ldr = K + 8, Kq = K / 4, Kw = K / kSmallWarps;
+    const int c0 = blockIdx.x * kSmallWarps;
+    const int n_cols = min(kSmallWarps, a.d_out - c0);
+    T *ws = reinterpret_cast<T *>(sm);                 // [8][ldr]
+    T *xs = ws + (size_t)kSmallWarps * ldr;            // [n][ldr]
+    float *part = reinterpret_cast<float *>(xs + (size_t)n * ldr);   // [8 warps][16][8]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(part + kSmallWarps * 16 * 8);
+    const T *w = static_cast<const T *>(a.w);
+    const T *x = static_cast<const T *>(a.x);
+
+    pdl_trigger();
+    if (warp < n_cols) {   // warm L2 with this warp's weight row while the previous kernel finishes
+        const uint4 *wrow = reinterpret_cast<const uint4 *>(w + (int64_t)(c0 + warp) * K);
+        for (int ch = lane * 8; ch < K / 8; ch += 256) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + ch));
+    }
+    if (threadIdx.x == 0) {
+        for (int q = 0; q < 4; ++q) mbar_init(&bars[q], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    if (threadIdx.x == 0) {
+        const uint32_t qb = (uint32_t)Kq * 2;
+        for (int q = 0; q < 4; ++q) {
+            mbar_arrive_expect_tx(&bars[q], (uint32_t)(n_cols + n) * qb);
+            for (int j = 0; j < n_cols; ++j)
+                bulk_g2s(ws + (size_t)j * ldr + q * Kq, w + (int64_t)(c0 + j) * K + q * Kq, qb, &bars[q]);
+            for (int r = 0; r < n; ++r)
+                bulk_g2s(xs + (size_t)r * ldr + q * Kq, x + (int64_t)r * K + q * Kq, qb, &bars[q]);
+        }
+    }
+    // this warp's K range lies in quarter warp / 2
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[warp / 2], 0, &g_status_linear));
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    if (ok) {
+        const uint32_t kOnes = 0x3F803F80u;   // two bf16 1.0
+        const T *xa = xs + (size_t)g * ldr, *xb = xs + (size_t)(g + 8) * ldr;
+        const T *wb = ws + (size_t)g * ldr;
+        for (int kk = warp * Kw; kk < (warp + 1) * Kw; kk += 16) {
+            const int k0 = kk + 2 * t4;
+            uint32_t af[4], bfr[2];
+            af[0] = g < n ? *reinterpret_cast<const uint32_t *>(xa + k0) : 0u;
+            af[2] = g < n ? *reinterpret_cast<const uint32_t *>(xa + k0 + 8) : 0u;
+            af[1] = g + 8 < n ? *reinterpret_cast<const uint32_t *>(xb + k0) : (g == 7 ? kOnes : 0u);
+            af[3] = g + 8 < n ? *reinterpret_cast<const uint32_t *>(xb + k0 + 8) : (g == 7 ? kOnes : 0u);
+            bfr[0] = *reinterpret_cast<const uint32_t *>(wb + k0);
+            bfr[1] = *reinterpret_cast<const uint32_t *>(wb + k0 + 8);
+            mma_bf16_16816(c, af, bfr);
+        }
+    }
+    float *pw = part + warp * 16 * 8;
+    pw[g * 8 + 2 * t4] = c[0];
+    pw[g * 8 + 2 * t4 + 1] = c[1];
+    pw[(g + 8) * 8 + 2 * t4] = c[2];
+    pw[(g + 8) * 8 + 2 * t4 + 1] = c[3];
+    // every quarter has landed before the row statistics read whole rows
+    for (int q = 0; q < 4 && ok; ++q) ok = __all_sync(0xffffffffu, mbar_wait(&bars[q], 0, &g_status_linear));
+    if (ok && warp < n) {
+        const int r = warp;
+        float mean = 0.f, rstd = 1.f;
+        if (a.apply_ln) {
+            const T *xr = xs + (size_t)r * ldr;
+            const float x0 = to_f32(xr[0]);
+            const uint64_t sh = pack2(-x0, -x0);
+            uint64_t s1 = 0, s2 = 0;
+            for (int ch = lane; ch < K / 8; ch += 32) {
+                uint64_t p[4];
+                chunk_pairs<T>(*reinterpret_cast<const uint4 *>(xr + ch * 8), p);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint64_t d = add2(p[i], sh);
+                    s1 = add2(s1, d);
+                    s2 = fma2(d, d, s2);
+                }
+            }
+            const float m1 = warp_sum(hsum2(s1)) / (float)K;
+            const float var = fmaxf(warp_sum(hsum2(s2)) / (float)K - m1 * m1, 0.f);
+            mean = x0 + m1;
+            rstd = rsqrtf(var + a.eps);
+        }
+        if (lane == 0) {
+            mu[r] = mean;
+            rs[r] = rstd;
+        }
+    }
+    __syncthreads();
+    // one thread per (row, column): the warps' partial sums, the fold, the blend
+    const int i = threadIdx.x, r = i / kSmallWarps, cc = i % kSmallWarps;
+    if (!ok || r >= n || cc >= n_cols) return;
+    float tot = 0.f, wsum = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < kSmallWarps; ++ww) {
+        tot += part[(ww * 16 + r) * 8 + cc];
+        wsum += part[(ww * 16 + 15) * 8 + cc];
+    }
+    const int col = c0 + cc, w1 = a.d_out - a.split_col;
+    const int64_t dr = a.dst_rows ? a.dst_rows[r] : r;
+    float val = a.apply_ln ? rs[r] * (tot - mu[r] * wsum) : tot;
+    if (col < a.split_col) {
+        if (a.base0) val = fmaf(a.w0, to_f32(static_cast<const T *>(a.base0)[(int64_t)r * a.split_col + col]), val);
+        static_cast<T *>(a.out0)[dr * a.split_col + col] = from_f32<T>(val);
+    } else {
+        const int c1 = col - a.split_col;
+        if (a.base1) val = fmaf(a.w1, to_f32(static_cast<const T *>(a.base1)[(int64_t)r * w1 + c1]), val);
+        static_cast<T *>(a.out1)[dr * w1 + c1] = from_f32<T>(val);
+    }
+}
+
 template <typename T, int NR>
 static cudaError_t launch_small(const LinearArgs &a, size_t smem, cudaStream_t st) {
     auto kern = linear_small_kernel<T, NR>;
@@ -313,6 +450,17 @@ static cudaError_t launch_small_t(const LinearArgs &a, size_t smem, cudaStream_t
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t st) {
     if (a.n == 0 || a.d_out == 0) return cudaSuccess;
     const int vec = a.dtype == kBF16 ? 8 : 4;
+    if (a.dtype == kBF16 && a.n <= kFewMaxRows && a.d_in % 128 == 0) {
+        const size_t fsm = few_tc_smem_bytes((int)a.n, a.d_in);
+        if (fsm <= kSmallMaxSmem) {
+            const cudaError_t e = cudaFuncSetAttribute(linear_few_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)kSmallMaxSmem);
+            if (e != cudaSuccess) return e;
+            note_launches(1);
+            const int grid = (a.d_out + kSmallWarps - 1) / kSmallWarps;
+            return launch_pdl(linear_few_tc_kernel, dim3(grid), dim3(32 * kSmallWarps), fsm, st, a);
+        }
+    }
     const size_t smem = small_smem_bytes((int)std::min<int64_t>(a.n, kSmallRows), a.d_in, (int)dtype_bytes(a.dtype));
     if (a.n <= kSmallRows && a.d_in % vec == 0 && smem <= kSmallMaxSmem)
         return a.dtype == kBF16 ? launch_small_t<__nv_bfloat16>(a, smem, st) : launch_small_t<float>(a, smem, st);
