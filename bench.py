@@ -987,7 +987,7 @@ def run_chunk_parallel(args):
     os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
     os.environ.setdefault("MASTER_PORT", "29511")
     dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), world_size=world,
-                            rank=int(os.environ.get("RANK", "0")))
+                            rank=int(os.environ.get("RANK", "0")), device_id=dev)
     yoco.load()
     rep, _ = chunk_parallel_measure(cp.DistComm(), cp.KernelOps, dev, torch.bfloat16, args.steps,
                                     args.warmup, **CP)
@@ -1055,7 +1055,7 @@ def main():
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     import shared_kv_decoder_b200 as yoco
     yoco.load()
     try:
