@@ -100,10 +100,10 @@ def load_peaks():
 # and the report carries null instead.
 _CSRC = "shared_kv_decoder_b200/csrc/"
 TRAFFIC = {
-    # attn_prefill_pair_kernel<128>, T=32768: 568.586 MB read + 232.266 MB written
-    "prefill": {"bytes": 568585984 + 232265984,
+    # attn_prefill_pair_kernel<128>, T=32768: 569.859 MB read + 239.108 MB written
+    "prefill": {"bytes": 569859328 + 239108096,
                 "sources": ["prefill_pair.cu", "schedule.h", "tc.cuh", "common.cuh"],
-                "sha256": "992d6629df8f74de25fecff8eeeccf505c37e589717e1947e48a9fdae3a4bb46"},
+                "sha256": "836177e0fbe98c89f48dc571b8a23986d590602891340cf2b4ce942e7e583e83"},
     # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416115 GB read + 24.940 MB written
     "decode": {"bytes": 6416114944 + 24940032,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],

@@ -21,7 +21,8 @@
 //              exponentials on MUFU, a quarter on an FMA-pipe polynomial --
 //              and writes P as bf16 over the first 64 columns of its S buffer.
 //              The running max only moves (and O is rescaled in TMEM) when it
-//              grows by more than 2^8.  The same warps run the epilogue.
+//              grows by more than 2^8.  The same warps run the epilogue, which
+//              frees the O columns as soon as they are in registers.
 //   warp 8     TMA producer: lane 0 loads the two Q tiles, lane 1 the K tiles
 //              (three stages), lane 2 the V tiles (two stages).
 //   warp 9     MMA issuer (one thread), in the order
@@ -80,6 +81,7 @@ struct PairParams {
     void *o;
     float *lse;
     int32_t n_work;
+    int32_t o_32B;   // o is 32-byte aligned: rows go out in 32-byte stores
 };
 
 enum Bar {
@@ -96,6 +98,15 @@ enum Bar {
     kDrain = 22,
     kNumBars = 23
 };
+
+// 32-byte global store (the sm_100 256-bit vector store), not kept in L1; the
+// address must be 32-byte aligned.
+YOCO_DEV void st_global_32B(void *p, const uint32_t (&w)[8]) {
+    asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :: "l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                    "r"(w[7])
+                 : "memory");
+}
 
 YOCO_DEV bool wait1(uint64_t *bar, uint32_t parity) {
     return mbar_wait(bar, parity, &g_status_prefill_pair);
@@ -309,15 +320,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < BN; c += 32) tc::tmem_ld32(tS + c, s + c);
                 tc::wait_ld();
                 if (sched::prefill_tile_masked(p.s, x, t)) {
-                    // visible columns of this row form one range [c_lo, c_hi)
+                    // visible columns of this row form one range [c_lo, c_hi); the
+                    // diagonal tile has c_lo = 0 and a window's lower-edge tile
+                    // c_hi = BN, which need one comparison per column, not two
                     const int64_t j0 = (int64_t)(x.jt_lo + t) * BN;
                     const int64_t dg = pos - j0;
                     const int c_hi = (int)max((int64_t)0, min(min(dg + 1, p.s.Tkv - j0), (int64_t)BN));
                     const int c_lo =
                         p.s.window > 0 ? (int)max((int64_t)0, min(dg - p.s.window + 1, (int64_t)BN)) : 0;
-                    const unsigned width = (unsigned)max(0, c_hi - c_lo);
+                    if (c_lo == 0) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) s[c] = (unsigned)(c - c_lo) < width ? s[c] : -INFINITY;
+                        for (int c = 0; c < BN; ++c) s[c] = c < c_hi ? s[c] : -INFINITY;
+                    } else if (c_hi == BN) {
+#pragma unroll
+                        for (int c = 0; c < BN; ++c) s[c] = c >= c_lo ? s[c] : -INFINITY;
+                    } else {
+                        const unsigned width = (unsigned)max(0, c_hi - c_lo);
+#pragma unroll
+                        for (int c = 0; c < BN; ++c) s[c] = (unsigned)(c - c_lo) < width ? s[c] : -INFINITY;
+                    }
                 }
                 // row max: 3-input max tree, eight independent chains
                 float a8[8];
@@ -393,33 +414,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bars[kPFull + hh]);
             }
             if (!ok) break;
-            // epilogue: the last P.V of this work tile, then O / l -> global
+            // epilogue: the last P.V of this work tile.  O is read out of TMEM
+            // whole and its columns handed to the next work tile's first P.V
+            // before O / l goes to global memory.  Each thread writes its own
+            // row, so a warp's store covers 32 rows: 32-byte stores make that
+            // 32 whole sectors per instruction, not 32 half sectors.
             if (!waitw(&bars[kODone + hh], (g - 1) & 1)) { ok = false; break; }
             tc::fence_after_sync();
+            float o[D];
+#pragma unroll
+            for (int c = 0; c < D; c += 32) tc::tmem_ld32(tO + c, o + c);
+            tc::wait_ld();
+            tc::fence_before_sync();
+            mbar_arrive(&bars[kOFree + hh]);
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *dst =
                 static_cast<__nv_bfloat16 *>(p.o) + (((int64_t)x.b * p.s.Tq + i) * p.s.Hq + h) * D;
+            if (i < p.s.Tq) {
+                if (p.o_32B) {
 #pragma unroll
-            for (int c = 0; c < D; c += 32) {
-                float o[32];
-                tc::tmem_ld32(tO + c, o);
-                tc::wait_ld();
-                if (i < p.s.Tq) {
+                    for (int e = 0; e < D; e += 16) {
+                        uint32_t wv[8];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
+                        for (int u = 0; u < 8; ++u) wv[u] = tc::pack_bf16x2(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
+                        st_global_32B(dst + e, wv);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < D; e += 8) {
                         uint4 wv;
                         wv.x = tc::pack_bf16x2(o[e] * inv, o[e + 1] * inv);
                         wv.y = tc::pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
                         wv.z = tc::pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
                         wv.w = tc::pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
-                        *reinterpret_cast<uint4 *>(dst + c + e) = wv;
+                        *reinterpret_cast<uint4 *>(dst + e) = wv;
                     }
                 }
             }
             if (p.lse && i < p.s.Tq)
                 p.lse[((int64_t)x.b * p.s.Hq + h) * p.s.Tq + i] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
-            tc::fence_before_sync();
-            mbar_arrive(&bars[kOFree + hh]);
         }
         if (!ok) *abort_flag = 1;
         tc::wait_st();  // no TMEM store may be in flight when TMEM is freed
@@ -455,6 +488,7 @@ cudaError_t launch_pair_d(const PrefillArgs &a, cudaStream_t st) {
     p.s.Tq = a.Tq; p.s.Tkv = a.Tkv; p.s.q_pos0 = a.q_pos0; p.s.window = a.window;
     p.scale_log2 = a.scale * kLog2e;
     p.o = a.o; p.lse = a.lse;
+    p.o_32B = (reinterpret_cast<uintptr_t>(a.o) & 31u) == 0;
     const int64_t n_qtiles = (a.Tq + BM - 1) / BM;
     const int64_t n_work = n_qtiles * (a.Hq / 2) * a.B;
     if (n_work > INT32_MAX / 2) return cudaErrorNotSupported;

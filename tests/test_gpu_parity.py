@@ -75,6 +75,24 @@ def test_swa_prefill_and_ring_match_oracle(cuda_lib, dtype, B, T, Hq, Hkv, D, W)
         np.testing.assert_array_equal(to_np(rv[b]), ev)
 
 
+@pytest.mark.parametrize("D,W", [(128, 0), (64, 0), (128, 128), (64, 100)])
+def test_prefill_output_16B_aligned(cuda_lib, D, W):
+    # o 16 bytes past a 32-byte boundary: the paired kernel writes rows with
+    # 16-byte stores there (32-byte stores otherwise)
+    B, T, Hq, Hkv = 2, 300, 8, 2
+    q, k, v = _qkv(B, T, T, Hq, Hkv, D, BF, 300 + D + W)
+    flat = torch.zeros(q.numel() + 8, dtype=BF, device="cuda")
+    o = flat[8:].view(q.shape)
+    assert o.data_ptr() % 32 == 16
+    if W:
+        cuda_lib.swa_prefill(q.cuda(), k.cuda(), v.cuda(), W, o=o)
+    else:
+        cuda_lib.cross_prefill(q.cuda(), k.cuda(), v.cuda(), 0, o=o)
+    ro, _ = oracle.attention(q, k, v, 0, W)
+    assert_close(o, ro, BF, "o")
+    assert float(flat[:8].float().abs().max()) == 0.0   # nothing written before o
+
+
 # -------------------------------------------------------------- swa decode
 @pytest.mark.parametrize("dtype", [BF, F32])
 def test_swa_decode_steps_match_oracle(cuda_lib, dtype):
