@@ -240,7 +240,7 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     if (!make_decode_plan(B, window, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl))
         return YOCO_ERR_UNSUPPORTED;
     if (!workspace || !aligned16(workspace) || ws_bytes < pl.ws_bytes) return YOCO_ERR_WORKSPACE;
-    // the window read skips the new token's slot and the merge adds the new
+    // the window read skips the new token's slot; the merge adds the new
     // token and writes it into the ring (no separate ring-write kernel)
     DecodeArgs a;
     a.q = q; a.k = ring_k; a.v = ring_v; a.seq_start = nullptr; a.seq_len = nullptr;
@@ -249,6 +249,10 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     a.cache_rows = (int64_t)B * window; a.max_len = window;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = nullptr; a.ws = workspace;
+    // bf16: one clustered launch (window read, merge, new token, ring write);
+    // other shapes: the split kernel and the merge
+    const cudaError_t e = launch_ring_decode(a, stream);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
     return from_cuda(launch_decode(a, pl, stream));
 }
 
@@ -425,7 +429,8 @@ yoco_status yoco_get_device_status(cudaStream_t stream) {
     const cudaError_t e = cudaStreamSynchronize(stream);
     const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc() |
                            read_and_clear_status_prefill_pair() | read_and_clear_status_project_tc() |
-                           read_and_clear_status_gret_tc() | read_and_clear_status_linear();
+                           read_and_clear_status_gret_tc() | read_and_clear_status_linear() |
+                           read_and_clear_status_ring();
     if (s & 1u) return YOCO_ERR_TIMEOUT;
     if (s & 2u) return YOCO_ERR_INVALID;
     return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;

@@ -51,6 +51,9 @@ struct DecodeArgs {
     void *ws;      // workspace
 };
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s);
+// Sliding-window decode step in one clustered launch (bf16, D 64 / 128, group
+// size 1, 2, 4 or 8); cudaErrorNotSupported for any other shape.
+cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t s);
 
 // Ring fill after a prefill of T tokens.
 cudaError_t launch_ring_fill(const void *k, const void *v, int32_t B, int64_t T, int32_t window,
@@ -133,6 +136,7 @@ unsigned int read_and_clear_status_prefill_pair();
 unsigned int read_and_clear_status_gret_tc();
 unsigned int read_and_clear_status_project_tc();
 unsigned int read_and_clear_status_linear();
+unsigned int read_and_clear_status_ring();
 
 int device_sm_count();
 

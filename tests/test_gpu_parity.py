@@ -117,6 +117,38 @@ def test_swa_decode_steps_match_oracle(cuda_lib, dtype):
             np.testing.assert_array_equal(to_np(rk[b]), rings[b][0])
 
 
+@pytest.mark.parametrize("Hq,Hkv,D,W,T", [
+    (8, 8, 128, 300, 700),      # group 1; three slices of 112 slots, the last one short
+    (8, 4, 64, 1000, 1500),     # group 2; eight slices, the last one 104 slots
+    (16, 2, 128, 2048, 2500),   # group 8; two 128-slot chunks per slice (two stages)
+    (32, 8, 128, 5000, 5100),   # group 4; five chunks per slice
+    (8, 2, 128, 129, 100),      # ring not yet full (empty slots), two slices
+])
+def test_swa_decode_window_shapes(cuda_lib, Hq, Hkv, D, W, T):
+    # the bf16 window decode at group sizes, windows and slice shapes that the
+    # 16-slot window above does not reach; ring and slot_pos bit-exact
+    B, n_dec = 2, 3
+    N = T + n_dec
+    q, k, v = _qkv(B, N, N, Hq, Hkv, D, BF, 320 + W)
+    rk = torch.empty((B, W, Hkv, D), dtype=BF, device="cuda")
+    rv = torch.empty((B, W, Hkv, D), dtype=BF, device="cuda")
+    sp = torch.empty((B, W), dtype=torch.int32, device="cuda")
+    cuda_lib.swa_prefill(q[:, :T].contiguous().cuda(), k[:, :T].contiguous().cuda(),
+                         v[:, :T].contiguous().cuda(), W, ring=(rk, rv, sp))
+    rings = [oracle.ring_from_prefill(k[b, :T], v[b, :T], W) for b in range(B)]
+    for p in range(T, N):
+        pos = torch.full((B,), p, dtype=torch.int64, device="cuda")
+        o = cuda_lib.swa_decode(q[:, p].contiguous().cuda(), k[:, p].contiguous().cuda(),
+                                v[:, p].contiguous().cuda(), pos, rk, rv, sp, W)
+        ro, _ = oracle.attention(q, k, v, 0, W, rows=[(b, p) for b in range(B)])
+        assert_close(o, ro, BF, f"o@{p}")
+        for b in range(B):
+            oracle.ring_push(rings[b][0], rings[b][1], rings[b][2], p, k[b, p], v[b, p])
+            np.testing.assert_array_equal(sp[b].cpu().numpy(), rings[b][2])
+            np.testing.assert_array_equal(to_np(rk[b]), rings[b][0])
+            np.testing.assert_array_equal(to_np(rv[b]), rings[b][1])
+
+
 def test_swa_decode_ragged_positions(cuda_lib):
     # sequences at different positions, some with a partly empty ring
     B, Hq, Hkv, D, W = 4, 4, 2, 64, 8
