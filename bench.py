@@ -312,7 +312,7 @@ def self_decoder_decode(W):
 
 
 def capture_self_decoder_decode(W):
-    """One CUDA graph of the 256 x 16 decode layer-steps (4 kernels each), so
+    """One CUDA graph of the 256 x 16 decode layer-steps (2 kernels each), so
     the steps run back to back without host launch overhead.  The rings must
     hold a prefill's contents (the graph is recorded after one eager run).
     Returns the number of library kernels one replay launches."""
@@ -1177,7 +1177,7 @@ def measure(args, world, rank, local, dev):
                 "decode_bytes_per_layer_step": layer_step_bytes,
                 "note": "attention times include the ring fill; decode = 256 steps x 16 layers from one "
                         "CUDA graph, each layer-step = projection of the 4 new tokens with the blend, "
-                        "ring write, window attention, split merge"},
+                        "then one clustered launch: window attention, merge with the new token, ring write"},
         "gkv": {"ms": statistics.mean(gkv_ms), "tflops": gkv_fl / (statistics.mean(gkv_ms) * 1e-3) / 1e12},
         "roofline": {"kernel": "cross prefill (yoco_cross_prefill)", "bound": "tensor",
                      "achieved": pre_tflops_launch, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
