@@ -104,6 +104,17 @@ TRAFFIC = {
     "prefill": {"bytes": 569859328 + 239108096,
                 "sources": ["prefill_pair.cu", "schedule.h", "tc.cuh", "common.cuh"],
                 "sha256": "836177e0fbe98c89f48dc571b8a23986d590602891340cf2b4ce942e7e583e83"},
+    # attn_prefill_pair_kernel<128>, sliding window 1024, B=1 x T=65536 (806.840 MB read +
+    # 507.447 MB written), times 4 for the benchmark's B=4 launch: the batches are independent
+    # and each reads its own Q, K, V and writes its own O once
+    "swa_prefill": {"bytes": 4 * (806840320 + 507446528),
+                    "sources": ['prefill_pair.cu', 'schedule.h', 'tc.cuh', 'common.cuh'],
+                    "sha256": "836177e0fbe98c89f48dc571b8a23986d590602891340cf2b4ce942e7e583e83"},
+    # one decode layer-step at batch 4, window 1024: ring_decode_cluster_kernel<128, 4>
+    # 16.883 MB read + linear_few_tc_kernel (the 4-token projection) 16.848 MB read
+    "swa_decode": {"bytes": 16883200 + 16848128,
+                   "sources": ['ring_decode.cu', 'linear.cu', 'tc.cuh', 'common.cuh'],
+                   "sha256": "93fb8fab138133c2cafe13aba3b2b1074f632d7d90615f251a19f52034236422"},
     # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416115 GB read + 24.940 MB written
     "decode": {"bytes": 6416114944 + 24940032,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
@@ -1189,11 +1200,11 @@ def measure(args, world, rank, local, dev):
                             "peak_src": f"{peaks['src']} hbm"},
         "roofline_swa_prefill": {"kernel": "sliding-window prefill (yoco_swa_prefill)", "bound": "tensor",
                                  "achieved": swa_att_tf, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                                 "frac": swa_att_tf / peaks["bf16_sus"], "traffic": None,
+                                 "frac": swa_att_tf / peaks["bf16_sus"], "traffic": traffic("swa_prefill"),
                                  "peak_src": f"{peaks['src']} bf16 sustained"},
         "roofline_swa_decode": {"kernel": "sliding-window decode layer-step (projection + yoco_swa_decode)",
                                 "bound": "hbm", "achieved": swa_dec_gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                                "frac": swa_dec_gbs / peaks["hbm"], "traffic": None,
+                                "frac": swa_dec_gbs / peaks["hbm"], "traffic": traffic("swa_decode"),
                                 "peak_src": f"{peaks['src']} hbm"},
         "gpu_launches": launches,
         "clocks": clk,
