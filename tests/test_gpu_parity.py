@@ -149,6 +149,43 @@ def test_swa_decode_window_shapes(cuda_lib, Hq, Hkv, D, W, T):
             np.testing.assert_array_equal(to_np(rv[b]), rings[b][1])
 
 
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 1, 128), (4, 2, 64)])
+def test_swa_decode_window_one_is_the_new_value(cuda_lib, Hq, Hkv, D):
+    # window 1: the only slot is the new token's, so every ring slot is left
+    # out and o is the new token's value row, exactly (weight 2^0 / 2^0)
+    B, W = 3, 1
+    q = wl.normal((B, Hq, D), 330, BF).cuda()
+    kn = wl.normal((B, Hkv, D), 331, BF).cuda()
+    vn = wl.normal((B, Hkv, D), 332, BF).cuda()
+    rk = wl.normal((B, W, Hkv, D), 333, BF).cuda()
+    rv = (wl.normal((B, W, Hkv, D), 334, BF) * 1e4).to(BF).cuda()   # would dominate if read
+    sp = torch.full((B, W), 5, dtype=torch.int32, device="cuda")
+    pos = torch.tensor([6, 7, 100], dtype=torch.int64, device="cuda")
+    o = cuda_lib.swa_decode(q, kn, vn, pos, rk, rv, sp, W)
+    assert torch.equal(o, vn.repeat_interleave(Hq // Hkv, dim=1))
+    assert torch.equal(rk[:, 0], kn) and torch.equal(rv[:, 0], vn)
+    assert sp[:, 0].tolist() == [6, 7, 100]
+
+
+@pytest.mark.parametrize("W,T", [(2, 5), (2, 1)])
+def test_swa_decode_window_two(cuda_lib, W, T):
+    # the smallest window with a ring read: one old slot plus the new token
+    B, Hq, Hkv, D, n_dec = 2, 8, 1, 128, 3
+    N = T + n_dec
+    q, k, v = _qkv(B, N, N, Hq, Hkv, D, BF, 340 + T)
+    rk = torch.empty((B, W, Hkv, D), dtype=BF, device="cuda")
+    rv = torch.empty((B, W, Hkv, D), dtype=BF, device="cuda")
+    sp = torch.empty((B, W), dtype=torch.int32, device="cuda")
+    cuda_lib.swa_prefill(q[:, :T].contiguous().cuda(), k[:, :T].contiguous().cuda(),
+                         v[:, :T].contiguous().cuda(), W, ring=(rk, rv, sp))
+    ro, _ = oracle.attention(q, k, v, 0, W)
+    for p in range(T, N):
+        pos = torch.full((B,), p, dtype=torch.int64, device="cuda")
+        o = cuda_lib.swa_decode(q[:, p].contiguous().cuda(), k[:, p].contiguous().cuda(),
+                                v[:, p].contiguous().cuda(), pos, rk, rv, sp, W)
+        assert_close(o, ro[:, p], BF, f"o@{p}")
+
+
 def test_swa_decode_ragged_positions(cuda_lib):
     # sequences at different positions, some with a partly empty ring
     B, Hq, Hkv, D, W = 4, 4, 2, 64, 8
