@@ -643,9 +643,13 @@ def e2e_prefill(W, steps, warmup):
     step's Q (14 layers) and the shared K/V from pinned host memory and reads
     every layer's output back into its own pinned host buffer, all inside the
     timed region.  The copies run on their own streams and overlap the
-    kernels as a caller would arrange them: layer l+1's Q goes up while layer
-    l computes, and layer l-1's O comes down (two device buffers each, events
-    for the hand-offs)."""
+    kernels as a caller serving one prompt after another would arrange them:
+    layer l+1's Q goes up while layer l computes, layer l-1's O comes down,
+    and the next step's K/V and first Q go up while this step's last layers
+    run (two device buffers each, events for the hand-offs).  The steps are
+    timed as one region (the same kernels and copies as step by step; L2 is
+    flushed between steps on the compute stream).  Returns one time per step
+    (the region's time divided evenly) and the bytes each step copies."""
     import torch
     import shared_kv_decoder_b200 as yoco
     L = P["layers"]
@@ -655,47 +659,68 @@ def e2e_prefill(W, steps, warmup):
     ho = [torch.empty(W["o"].shape, dtype=W["o"].dtype).pin_memory() for _ in range(L)]
     dq = [torch.empty_like(W["qs"][0]) for _ in range(2)]
     do = [torch.empty_like(W["o"]) for _ in range(2)]
-    dk, dv = torch.empty_like(W["kg"]), torch.empty_like(W["vg"])
+    dk = [torch.empty_like(W["kg"]) for _ in range(2)]
+    dv = [torch.empty_like(W["vg"]) for _ in range(2)]
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
-    times = []
-    for it in range(warmup + steps):
-        W["flush"].zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(comp)
-        in_ready = [ev() for _ in range(L)]
-        comp_done = [ev() for _ in range(L)]
-        out_done = [ev() for _ in range(L)]
-        s_in.wait_stream(comp)
-        s_out.wait_stream(comp)
-        with torch.cuda.stream(s_in):
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            dq[0].copy_(hq[0], non_blocking=True)
-            in_ready[0].record(s_in)
-        for l in range(L):
-            if l + 1 < L:
-                with torch.cuda.stream(s_in):
-                    if l >= 1:
-                        s_in.wait_event(comp_done[l - 1])     # dq[(l+1)%2] is free again
-                    dq[(l + 1) % 2].copy_(hq[l + 1], non_blocking=True)
-                    in_ready[l + 1].record(s_in)
-            comp.wait_event(in_ready[l])
-            if l >= 2:
-                comp.wait_event(out_done[l - 2])              # do[l%2] has been read out
-            yoco.cross_prefill(dq[l % 2], dk, dv, o=do[l % 2])
-            comp_done[l].record(comp)
+
+    def run(n_steps):
+        # global layer index g = step * L + l: Q / O buffers alternate by g,
+        # K / V buffers by step
+        n = n_steps * L
+        if n == 0:
+            return
+        in_ready = [ev() for _ in range(n)]
+        comp_done = [ev() for _ in range(n)]
+        out_done = [ev() for _ in range(n)]
+        kv_ready = [ev() for _ in range(n_steps)]
+
+        def upload(g):
+            st, l = divmod(g, L)
+            with torch.cuda.stream(s_in):
+                if l == 0:
+                    if st >= 2:
+                        s_in.wait_event(comp_done[(st - 2) * L + L - 1])   # dk/dv[st % 2] free again
+                    dk[st % 2].copy_(hk, non_blocking=True)
+                    dv[st % 2].copy_(hv, non_blocking=True)
+                    kv_ready[st].record(s_in)
+                if g >= 2:
+                    s_in.wait_event(comp_done[g - 2])                      # dq[g % 2] free again
+                dq[g % 2].copy_(hq[l], non_blocking=True)
+                in_ready[g].record(s_in)
+
+        upload(0)
+        for g in range(n):
+            st, l = divmod(g, L)
+            if g + 1 < n:
+                upload(g + 1)
+            if l == 0 and st >= 1:
+                W["flush"].zero_()                  # L2 flushed between steps
+            comp.wait_event(kv_ready[st])
+            comp.wait_event(in_ready[g])
+            if g >= 2:
+                comp.wait_event(out_done[g - 2])    # do[g % 2] has been read out
+            yoco.cross_prefill(dq[g % 2], dk[st % 2], dv[st % 2], o=do[g % 2])
+            comp_done[g].record(comp)
             with torch.cuda.stream(s_out):
-                s_out.wait_event(comp_done[l])
-                ho[l].copy_(do[l % 2], non_blocking=True)
-                out_done[l].record(s_out)
-        comp.wait_event(out_done[L - 1])
+                s_out.wait_event(comp_done[g])
+                ho[l].copy_(do[g % 2], non_blocking=True)
+                out_done[g].record(s_out)
+        comp.wait_event(out_done[n - 1])
         comp.wait_stream(s_in)
-        e1.record(comp)
-        torch.cuda.synchronize()
-        if it >= warmup:
-            times.append(e0.elapsed_time(e1))
+
+    W["flush"].zero_()
+    run(warmup)
+    torch.cuda.synchronize()
+    W["flush"].zero_()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    run(steps)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    total = e0.elapsed_time(e1)
+    times = [total / steps] * steps
     h2d = sum(q.numel() * q.element_size() for q in hq) + 2 * hk.numel() * hk.element_size()
     d2h = sum(o.numel() * o.element_size() for o in ho)
     return times, h2d, d2h
