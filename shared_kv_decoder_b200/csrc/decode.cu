@@ -378,29 +378,17 @@ YOCO_DEV float ex2f(float x) {
 // padded by 16 bytes against bank conflicts) kept fewer bytes in flight and
 // streamed 9% slower.  For a head, the eight token rows one ldmatrix gathers
 // are consecutive swizzled rows, so they fall in eight different bank groups.
-// A stage that ends a sequence short of stage_tokens is not copied: no box
-// may read past the sequence (the cache's end is not known to the kernel), so
-// each consumer warp loads its own head's valid rows with plain loads and
-// zeroes the rest.
+// A stage that ends a sequence short of stage_tokens is not copied (its box
+// would read the next sequence's rows, or rows past the cache's end that the
+// map fills with zeros); each consumer warp loads its own head's valid rows
+// with plain loads and zeroes the rest.  This kernel reads the packed shared
+// cache only: the bf16 sliding-window decode has a kernel of its own
+// (ring_decode.cu).
 template <int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeKParams p) {
     pdl_trigger();
-    if (!p.seq_len && threadIdx.x == 32 * kConsumerWarps) {
-        // ring mode: every sequence has the same units and finding this CTA's
-        // first one reads no memory, so its K and V rows can be pulled into L2
-        // while the previous kernel (the ring write) finishes
-        const int64_t nu = sched::decode_units(p.window, p.split, p.n_split);
-        if ((int64_t)blockIdx.x < nu * p.B) {
-            const int64_t b = blockIdx.x / nu, t0 = (blockIdx.x % nu) * p.split;
-            const int64_t n_tok = min(p.split, (int64_t)p.window - t0);
-            const size_t off = ((size_t)b * p.window + t0) * p.Hkv * D * 2;
-            const uint32_t bytes = (uint32_t)(n_tok * p.Hkv * D * 2);
-            bulk_prefetch_l2(static_cast<const unsigned char *>(p.k) + off, bytes);
-            bulk_prefetch_l2(static_cast<const unsigned char *>(p.v) + off, bytes);
-        }
-    }
     pdl_wait();
     if (*(volatile unsigned int *)&g_status_decode & kStatusTimeout) return;  // an earlier CTA timed out
     static_assert(G >= 1 && G <= 8, "query heads per KV head");
@@ -434,10 +422,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         int b;
         int64_t s;
         if (!find_unit(p, u, &b, &s)) break;
-        const int64_t len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
+        const int64_t len = (int64_t)p.seq_len[b];
         const int64_t t0 = s * p.split;
         const int64_t n_tok = min(p.split, len - t0);
-        const int64_t row0 = (p.seq_start ? p.seq_start[b] : (int64_t)b * p.window) + t0;
+        const int64_t row0 = p.seq_start[b] + t0;
         const int n_st = (int)((n_tok + ST - 1) / ST);
 
         if (warp == kConsumerWarps) {
@@ -472,11 +460,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const int j = warp / p.Hkv;      // 16-token subset of every stage
             const int gq = lane >> 2;        // fragment row: query head of the group
             const int t = lane & 3;
-            const int64_t pos_b = p.pos ? p.pos[b] : 0;
-            const int32_t *sp = p.slot_pos ? p.slot_pos + (int64_t)b * p.window + t0 : nullptr;
-            // ring mode: the slot the new token goes to is left out here (whatever it
-            // holds is replaced); the merge adds the new token from k_new / v_new
-            const int64_t new_slot = p.window > 0 ? ((pos_b % p.window) + p.window) % p.window : -1;
 
             uint32_t qa[D / 16][2];
             if (gq < G) {
@@ -557,13 +540,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                     for (int e = 0; e < 2; ++e) {
                         const int lt = 8 * n + 2 * t + e;
                         const int64_t tok = base_tok + lt;
-                        bool vld = tok < n_tok;
-                        if (vld && sp) {
-                            const int32_t sp_t = sp[tok];
-                            vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window &&
-                                  t0 + tok != new_slot;
-                        }
-                        const float v = vld ? sc[n][e] * p.scale_log2 : -INFINITY;
+                        const float v = tok < n_tok ? sc[n][e] * p.scale_log2 : -INFINITY;
                         pv[n][e] = v;
                         mx = fmaxf(mx, v);
                     }
@@ -734,10 +711,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         int b;
         int64_t s;
         if (!find_unit(p, u, &b, &s)) break;
-        const int64_t len = p.seq_len ? (int64_t)p.seq_len[b] : (int64_t)p.window;
+        const int64_t len = (int64_t)p.seq_len[b];
         const int64_t t0 = s * p.split;
         const int64_t n_tok = min(p.split, len - t0);
-        const int64_t row0 = (p.seq_start ? p.seq_start[b] : (int64_t)b * p.window) + t0;
+        const int64_t row0 = p.seq_start[b] + t0;
         const int n_st = (int)((n_tok + ST - 1) / ST);
 
         if (warp == kConsumerWarps) {
@@ -771,8 +748,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const int j = warp / p.Hkv;      // 16-token subset of every stage
             const int gq = lane >> 2;        // S^T row (token) / P^T column (query head)
             const int t = lane & 3;
-            const int64_t pos_b = p.pos ? p.pos[b] : 0;
-            const int32_t *sp = p.slot_pos ? p.slot_pos + (int64_t)b * p.window + t0 : nullptr;
             const int tok0 = j * kTokPerWarp;
 
             // q of head gq as two int8 parts (B operand: dims 32kb + 4t.. and
@@ -905,11 +880,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
                 for (int h8 = 0; h8 < 2; ++h8) {
                     const int64_t tok = base_tok + gq + 8 * h8;
-                    bool vld = tok < n_tok;
-                    if (vld && sp) {
-                        const int32_t sp_t = sp[tok];
-                        vld = sp_t >= 0 && sp_t <= pos_b && (int64_t)sp_t > pos_b - p.window;
-                    }
+                    const bool vld = tok < n_tok;
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const float acc = (float)(128 * ah[2 * h8 + e] + al[2 * h8 + e]);
@@ -1266,6 +1237,8 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const DecodePlan &pl, cu
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, device_sm_count()));
     cudaError_t e;
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // the bf16 window decode runs in ring_decode.cu; this kernel reads the packed cache
+        if (!a.seq_len || !a.seq_start) return cudaErrorNotSupported;
         e = launch_decode_tma<D, G>(a, pl, p, grid, st);
     } else {
         auto kern = decode_split_kernel<T, D, G>;
