@@ -115,10 +115,10 @@ TRAFFIC = {
     "swa_decode": {"bytes": 16883200 + 16848128,
                    "sources": ['ring_decode.cu', 'linear.cu', 'tc.cuh', 'common.cuh'],
                    "sha256": "93fb8fab138133c2cafe13aba3b2b1074f632d7d90615f251a19f52034236422"},
-    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416354 GB read + 27.793 MB written
-    "decode": {"bytes": 6416353536 + 27793152,
+    # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416165 GB read + 25.238 MB written
+    "decode": {"bytes": 6416165120 + 25238272,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
-               "sha256": "16c19fdba885c8a62f0596904bdec8ad257995931c01de4b65c657df9a80dad2"},
+               "sha256": "e0b8311437112b861d4c0f91d6e071903fe71e380c3dfe04e2c884c4d197bd6f"},
 }
 
 

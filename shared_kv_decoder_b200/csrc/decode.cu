@@ -52,6 +52,7 @@ constexpr int kLanesPerTok = 8;
 constexpr int kTokPerPass = 32 / kLanesPerTok;
 constexpr int kPasses = kTokPerWarp / kTokPerPass;
 constexpr int64_t kMinUnits = 148, kMaxUnits = 148 * 12;   // decode units per call (see make_decode_plan)
+constexpr int64_t kMaxUnitsPerSeq = 148 * 2;                 // units of one sequence at most
 constexpr int64_t kUnitBytes = (int64_t)2 << 20;
 
 struct DecodeKParams {
@@ -1157,10 +1158,14 @@ bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dt
     pl.sub = kConsumerWarps / Hkv;
     // Units: about kUnitBytes of K and V each, between one per SM and twelve
     // per SM (many units balance ragged batches; few keep a short decode from
-    // paying per-unit overhead and a long merge), and at least two pipeline
-    // stages each.  A 16 x 64K-128K batch or a 1M-token sequence gets the
-    // maximum; a 4 x 1024 sliding-window ring ~128 units of two stages, each
-    // CTA with its whole unit in flight; one 32K-token sequence ~150 units.
+    // paying per-unit overhead and a long merge), at least two pipeline
+    // stages each, and at most two per SM for one sequence: the merge gives a
+    // sequence one CTA per query head, which folds the sequence's partials
+    // one after another.  A 16 x 64K-128K batch gets the maximum (~111 units
+    // a sequence); a 1M-token sequence 296 units, two per CTA (1776 made its
+    // merge ~0.1 ms of a 0.75 ms call); a 4 x 1024 sliding-window ring ~128
+    // units of two stages, each CTA with its whole unit in flight; one
+    // 32K-token sequence ~150 units.
     const int64_t total = (int64_t)std::max(B, 1) * max_len;
     const int64_t tok_bytes = 2 * (int64_t)Hkv * D * (int64_t)dtype_bytes(dtype);
     const int64_t target = std::min<int64_t>(kMaxUnits, std::max<int64_t>(kMinUnits, total * tok_bytes / kUnitBytes));
@@ -1168,6 +1173,8 @@ bool make_decode_plan(int32_t B, int64_t max_len, int Hq, int Hkv, int D, int dt
     int64_t per = (total + target - 1) / target;
     per = ((per + pl.stage_tokens - 1) / pl.stage_tokens) * pl.stage_tokens;
     pl.split = std::max(per, min_split);
+    const int64_t per_seq = (max_len + kMaxUnitsPerSeq - 1) / kMaxUnitsPerSeq;
+    pl.split = std::max(pl.split, ((per_seq + pl.stage_tokens - 1) / pl.stage_tokens) * pl.stage_tokens);
     pl.n_split = (max_len + pl.split - 1) / pl.split;
     // a stage holds 128 token-head rows of K and of V; the bf16 kernel adds
     // 1 KB so that its swizzled stages can start on a 1024-byte boundary
