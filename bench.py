@@ -76,7 +76,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["prefill", "decode", "swa", "proj", "prefill_layer", "decode_layer",
                                        "gret", "gret_decode", "decode_i8_layer", "gret1", "decode_i8",
-                                       "long_prefill", "long_decode", "swa_decode_layer", "proj_small"],
+                                       "long_prefill", "long_decode", "swa_decode_layer", "swa_step_layer", "proj_small"],
                     default=None,
                     help="time one kernel on a small case larger than L2 (for profiling)")
     return ap.parse_args()
@@ -110,11 +110,12 @@ TRAFFIC = {
     "swa_prefill": {"bytes": 4 * (806840320 + 507446528),
                     "sources": ['prefill_pair.cu', 'schedule.h', 'tc.cuh', 'common.cuh'],
                     "sha256": "836177e0fbe98c89f48dc571b8a23986d590602891340cf2b4ce942e7e583e83"},
-    # one decode layer-step at batch 4, window 1024: ring_decode_cluster_kernel<128, 4>
-    # 16.883 MB read + linear_few_tc_kernel (the 4-token projection) 16.848 MB read
-    "swa_decode": {"bytes": 16883200 + 16848128,
-                   "sources": ['ring_decode.cu', 'linear.cu', 'tc.cuh', 'common.cuh'],
-                   "sha256": "93fb8fab138133c2cafe13aba3b2b1074f632d7d90615f251a19f52034236422"},
+    # one decode layer-step at batch 4, window 1024 (yoco_swa_decode_step):
+    # linear_few_reg_kernel (the 4-token projection) 16.851 MB read +
+    # ring_decode_cluster_kernel<128, 4> (early copies, 4 CTAs a head) 16.891 MB read
+    "swa_decode": {"bytes": 16850688 + 16891392,
+                   "sources": ['ring_decode.cu', 'step_proj.cu', 'cluster.cuh', 'tc.cuh', 'common.cuh'],
+                   "sha256": "73e3c1455a92d30dd6cd3735e630680c7f7d3bb6904f751b2d3f2f8ac4f65aa8"},
     # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416165 GB read + 25.238 MB written
     "decode": {"bytes": 6416165120 + 25238272,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
@@ -265,10 +266,9 @@ def make_workload(dev):
     W["x4d"] = wl.normal((S4, L4, B4, d), 3400, bf, dev)
     W["q4d"] = wl.normal((S4, L4, B4, Hq, D), 3401, bf, dev)
     W["pos4"] = (T4 + torch.arange(S4, dtype=torch.int64, device=dev))[:, None].repeat(1, B4).contiguous()
-    W["k1t"], W["v1t"], W["k4t"], W["v4t"] = (torch.empty((B4, Hkv, D), dtype=bf, device=dev)
-                                              for _ in range(4))
+    W["k1t"], W["v1t"] = (torch.empty((B4, Hkv, D), dtype=bf, device=dev) for _ in range(2))
     W["o4t"] = torch.empty((B4, Hq, D), dtype=bf, device=dev)
-    W["ws4"] = torch.empty(yoco.swa_decode_workspace_size(B4, W4, Hq, Hkv, D, bf),
+    W["ws4"] = torch.empty(yoco.swa_decode_step_workspace_size(B4, W4, Hq, Hkv, D, bf),
                            dtype=torch.uint8, device=dev)
     W["flush"] = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     return W
@@ -302,24 +302,23 @@ def self_decoder_prefill(W, ev=None):
 
 def self_decoder_decode(W):
     """256 decode steps of the 16 sliding-window layers: per step and layer
-    the 4 new tokens' K/V projection (blended with the bottom layer's K/V of
-    the same tokens), their ring write and the window read.  Position T + s
-    of step s overwrites the ring slot of T + s - window, so replaying the
-    steps after a prefill is idempotent."""
+    one yoco_swa_decode_step call -- the 4 new tokens' K/V projection
+    (blended with the bottom layer's K/V of the same tokens), the window
+    read, the merge with the new token and its ring write.  Position T + s of
+    step s overwrites the ring slot of T + s - window, so replaying the steps
+    after a prefill is idempotent."""
     import shared_kv_decoder_b200 as yoco
-    Hkv, D, Wn = SWA["Hkv"], SWA["D"], SWA["W"]
+    Wn = SWA["W"]
     for s in range(SWA["steps"]):
         for l in range(SWA["layers"]):
-            if l == 0:
-                yoco.kv_project_blend(W["x4d"][s, 0], W["w4"][0], Hkv, D, k_out=W["k1t"], v_out=W["v1t"])
-                kn, vn = W["k1t"], W["v1t"]
-            else:
-                yoco.kv_project_blend(W["x4d"][s, l], W["w4"][l], Hkv, D, W["k1t"], W["v1t"],
-                                      W["w_l"][l], W["w_l"][l], k_out=W["k4t"], v_out=W["v4t"])
-                kn, vn = W["k4t"], W["v4t"]
             rk, rv, sp = W["rings"][l]
-            yoco.swa_decode(W["q4d"][s, l], kn, vn, W["pos4"][s], rk, rv, sp, Wn,
-                            workspace=W["ws4"], o=W["o4t"])
+            if l == 0:   # the bottom layer's new K/V: the base of the layers above
+                yoco.swa_decode_step(W["x4d"][s, 0], W["w4"][0], W["q4d"][s, 0], W["pos4"][s], rk, rv, sp, Wn,
+                                     k_out=W["k1t"], v_out=W["v1t"], workspace=W["ws4"], o=W["o4t"])
+            else:
+                yoco.swa_decode_step(W["x4d"][s, l], W["w4"][l], W["q4d"][s, l], W["pos4"][s], rk, rv, sp, Wn,
+                                     W["k1t"], W["v1t"], W["w_l"][l], W["w_l"][l], workspace=W["ws4"],
+                                     o=W["o4t"])
 
 
 def capture_self_decoder_decode(W):
@@ -808,6 +807,8 @@ def run_case(args):
                sequence over all 1,048,576 rows
       swa_decode_layer  one sliding-window decode call at the self-decoder's shape (batch 4,
                window 1024: window attention + merge with the new token's ring write, 16.8 MB of ring)
+      swa_step_layer  one self-decoder decode step call at that shape (the 4 tokens' projection, d=4096,
+               then the window decode): 16.8 MB of weights + 16.8 MB of ring
       proj_small  the decode step's K/V projection of 4 tokens, d=4096 -> 2048, with the blend (16.8 MB
                of weights)
     Prints one JSON line with the mean launch time and the work rate."""
@@ -867,6 +868,21 @@ def run_case(args):
         ws = torch.empty(yoco.swa_decode_workspace_size(B, Wn, Hq, Hkv, D, bf), dtype=torch.uint8, device=dev)
         fn = lambda: yoco.swa_decode(q, kn, vn, pos, ring[0], ring[1], ring[2], Wn, workspace=ws, o=o)
         work, unit = 2.0 * B * Wn * Hkv * D * 2, "GB/s"
+    elif args.case == "swa_step_layer":
+        B, T, Wn, d = SWA["B"], 4096, SWA["W"], SWA["d"]
+        k = wl.normal((B, T, Hkv, D), 8, bf, dev); v = wl.normal((B, T, Hkv, D), 9, bf, dev)
+        ring = (torch.empty((B, Wn, Hkv, D), dtype=bf, device=dev), torch.empty((B, Wn, Hkv, D), dtype=bf, device=dev),
+                torch.empty((B, Wn), dtype=torch.int32, device=dev))
+        yoco.swa_prefill(wl.normal((B, T, Hq, D), 7, bf, dev), k, v, Wn, ring=ring)
+        q = wl.normal((B, Hq, D), 10, bf, dev); o = torch.empty_like(q)
+        x = wl.normal((B, d), 11, bf, dev)
+        w = wl.normal((2 * Hkv * D, d), 12, bf, dev, std=d ** -0.5)
+        kb = wl.normal((B, Hkv, D), 13, bf, dev); vb = wl.normal((B, Hkv, D), 14, bf, dev)
+        pos = torch.full((B,), T, dtype=torch.int64, device=dev)
+        ws = torch.empty(yoco.swa_decode_step_workspace_size(B, Wn, Hq, Hkv, D, bf), dtype=torch.uint8, device=dev)
+        fn = lambda: yoco.swa_decode_step(x, w, q, pos, ring[0], ring[1], ring[2], Wn, kb, vb, 0.5, 0.5,
+                                          workspace=ws, o=o)
+        work, unit = 2.0 * B * Wn * Hkv * D * 2 + 2.0 * Hkv * D * d * 2, "GB/s"
     elif args.case in ("decode_i8_layer", "decode_i8"):
         lens = (wl.ragged_lengths(DEC["B"], DEC["lo"], DEC["hi"], DEC["seed"]) if args.case == "decode_i8_layer"
                 else wl.ragged_lengths(16, 16384, 32768, 9))
@@ -1212,8 +1228,10 @@ def measure(args, world, rank, local, dev):
                 "decode_ms_per_layer_step": layer_step_ms, "decode_hbm_gbs": swa_dec_gbs,
                 "decode_bytes_per_layer_step": layer_step_bytes,
                 "note": "attention times include the ring fill; decode = 256 steps x 16 layers from one "
-                        "CUDA graph, each layer-step = projection of the 4 new tokens with the blend, "
-                        "then one clustered launch: window attention, merge with the new token, ring write"},
+                        "CUDA graph, each layer-step = one yoco_swa_decode_step call: the 4 new tokens' "
+                        "projection with the blend, and the clustered window decode (window attention, "
+                        "merge with the new token, ring write) whose first window copies go out while "
+                        "the projection runs"},
         "gkv": {"ms": statistics.mean(gkv_ms), "tflops": gkv_fl / (statistics.mean(gkv_ms) * 1e-3) / 1e12},
         "roofline": {"kernel": "cross prefill (yoco_cross_prefill)", "bound": "tensor",
                      "achieved": pre_tflops_launch, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
@@ -1227,7 +1245,7 @@ def measure(args, world, rank, local, dev):
                                  "achieved": swa_att_tf, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
                                  "frac": swa_att_tf / peaks["bf16_sus"], "traffic": traffic("swa_prefill"),
                                  "peak_src": f"{peaks['src']} bf16 sustained"},
-        "roofline_swa_decode": {"kernel": "sliding-window decode layer-step (projection + yoco_swa_decode)",
+        "roofline_swa_decode": {"kernel": "sliding-window decode layer-step (yoco_swa_decode_step: projection + window decode)",
                                 "bound": "hbm", "achieved": swa_dec_gbs, "peak": peaks["hbm"], "unit": "GB/s",
                                 "frac": swa_dec_gbs / peaks["hbm"], "traffic": traffic("swa_decode"),
                                 "peak_src": f"{peaks['src']} hbm"},

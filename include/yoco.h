@@ -121,6 +121,27 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
                             void *ring_v, int32_t *slot_pos, void *o, void *workspace,
                             size_t ws_bytes, const yoco_attn_cfg *cfg, cudaStream_t stream);
 
+/* One self-decoder decode step: yoco_kv_project_blend of the B new tokens
+ * (n_tok = B, no dst_rows) followed by yoco_swa_decode with the projected
+ * K/V -- the YOCO++ blended K/V producer (YOCO++ Abstract) and the section 3
+ * "Sliding-Window Attention" decode -- with the same results.  Two launches;
+ * for bf16 with B <= 4 and d_model a multiple of 256 the window's first
+ * copies are already in flight while the projection runs.
+ * x [B, d_model]; w_kv [2 Hkv D, d_model]; k_base, v_base [B, Hkv, D] or
+ * NULL (then w_k / w_v are ignored); q [B, Hq, D]; pos device int64 [B];
+ * ring_k, ring_v [B, window, Hkv, D]; slot_pos int32 [B, window]; o [B, Hq, D].
+ * k_out, v_out [B, Hkv, D] or NULL: receive the new tokens' blended K / V
+ * (what yoco_kv_project_blend would write; a bottom layer's output is the
+ * base of the layers above it); with NULL the workspace holds them.  The new
+ * K/V is rounded to the cache dtype before it is attended to and stored.
+ * workspace: yoco_swa_decode_step_workspace_size() bytes. */
+yoco_status yoco_swa_decode_step(const void *x, int32_t d_model, const void *w_kv, int32_t apply_ln,
+                                 float ln_eps, const void *k_base, const void *v_base, float w_k, float w_v,
+                                 const void *q, const int64_t *pos, int32_t B, int32_t window, void *ring_k,
+                                 void *ring_v, int32_t *slot_pos, void *o, void *k_out, void *v_out,
+                                 void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg,
+                                 cudaStream_t stream);
+
 /* Cross-decoder causal prefill over the one shared KV.  Section 2 and
  * podcast cue 12: every cross layer has its own Q and attends causally to the
  * same K_g, V_g.
@@ -188,6 +209,8 @@ yoco_status yoco_attention_prefill(const void *q, const void *k, const void *v, 
 /* Workspace bytes for yoco_cross_decode / yoco_swa_decode (0 on bad args). */
 size_t yoco_cross_decode_workspace_size(int32_t B, int64_t max_len, const yoco_attn_cfg *cfg);
 size_t yoco_swa_decode_workspace_size(int32_t B, int32_t window, const yoco_attn_cfg *cfg);
+/* Workspace bytes for yoco_swa_decode_step (0 on bad args). */
+size_t yoco_swa_decode_step_workspace_size(int32_t B, int32_t window, const yoco_attn_cfg *cfg);
 
 /* Auxiliary dense projection used around the attention core (query and
  * output projections of the small end-to-end stack):

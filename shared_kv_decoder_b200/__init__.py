@@ -20,7 +20,8 @@ import os
 import torch
 
 __all__ = ["YocoError", "load", "lib_path", "kv_project_blend", "linear", "swa_prefill",
-           "swa_decode", "cross_prefill", "cross_decode", "cross_decode_workspace_size",
+           "swa_decode", "swa_decode_step", "swa_decode_step_workspace_size", "cross_prefill",
+           "cross_decode", "cross_decode_workspace_size",
            "swa_decode_workspace_size", "cache_bytes", "device_status", "launch_count", "AttnCfg",
            "debug_tile_schedule", "SCHEDULE_PREFILL", "SCHEDULE_DECODE", "gret_prefill", "gret_decode",
            "kv_i8_row_bytes", "kv_quantize_i8", "cross_decode_i8",
@@ -71,6 +72,9 @@ def load():
         "yoco_linear": (st, [vp, i64, i32, vp, i32, i32, f32, vp, f32, vp, i32, vp]),
         "yoco_swa_prefill": (st, [vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, cfgp, vp]),
         "yoco_swa_decode": (st, [vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_swa_decode_step": (st, [vp, i32, vp, i32, f32, vp, vp, f32, f32, vp, vp, i32, i32, vp, vp, vp,
+                                      vp, vp, vp, vp, sz, cfgp, vp]),
+        "yoco_swa_decode_step_workspace_size": (sz, [i32, i32, cfgp]),
         "yoco_cross_prefill": (st, [vp, vp, vp, i32, i64, i64, i64, vp, vp, cfgp, vp]),
         "yoco_attention_prefill": (st, [vp, vp, vp, i32, i64, i64, i64, i32, vp, vp, cfgp, vp]),
         "yoco_cross_decode": (st, [vp, vp, vp, i64, vp, vp, i32, i64, vp, vp, vp, sz, cfgp, vp]),
@@ -201,6 +205,37 @@ def swa_decode(q, k_new, v_new, pos, ring_k, ring_v, slot_pos, window, workspace
                              _ptr(ring_k), _ptr(ring_v), _ptr(slot_pos), _ptr(o), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), ctypes.byref(cfg),
                              _stream()), "yoco_swa_decode")
+    return o
+
+
+def swa_decode_step_workspace_size(B, window, Hq, Hkv, D, dtype):
+    cfg = _cfg(Hq, Hkv, D, dtype)
+    return int(load().yoco_swa_decode_step_workspace_size(B, window, ctypes.byref(cfg)))
+
+
+def swa_decode_step(x, w_kv, q, pos, ring_k, ring_v, slot_pos, window, k_base=None, v_base=None,
+                    w_k=0.0, w_v=0.0, apply_ln=True, eps=1e-5, o=None, k_out=None, v_out=None,
+                    workspace=None, scale=0.0):
+    """One self-decoder decode step: kv_project_blend of the B new tokens, then
+    swa_decode with that K/V.  x [B, d]; w_kv [2*Hkv*D, d]; q [B, Hq, D];
+    pos int64 [B]; ring_k, ring_v [B, window, Hkv, D]; slot_pos int32 [B, window];
+    k_out / v_out [B, Hkv, D] (optional) receive the blended new K / V."""
+    L = load()
+    B, Hq, D = q.shape
+    Hkv = ring_k.shape[2]
+    d = x.shape[1]
+    if workspace is None:
+        workspace = torch.empty(swa_decode_step_workspace_size(B, window, Hq, Hkv, D, q.dtype),
+                                dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    _dev(x, w_kv, q, pos, ring_k, ring_v, slot_pos, k_base, v_base, o, k_out, v_out, workspace)
+    cfg = _cfg(Hq, Hkv, D, q.dtype, scale)
+    _check(L.yoco_swa_decode_step(_ptr(x), d, _ptr(w_kv), int(bool(apply_ln)), eps, _ptr(k_base),
+                                  _ptr(v_base), float(w_k), float(w_v), _ptr(q), _ptr(pos), B, int(window),
+                                  _ptr(ring_k), _ptr(ring_v), _ptr(slot_pos), _ptr(o), _ptr(k_out),
+                                  _ptr(v_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  ctypes.byref(cfg), _stream()), "yoco_swa_decode_step")
     return o
 
 

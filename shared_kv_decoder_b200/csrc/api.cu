@@ -256,6 +256,70 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
     return from_cuda(launch_decode(a, pl, stream));
 }
 
+size_t yoco_swa_decode_step_workspace_size(int32_t B, int32_t window, const yoco_attn_cfg *cfg) {
+    if (check_cfg(cfg) != YOCO_OK || B < 0 || window < 1) return 0;
+    const size_t dws = yoco_swa_decode_workspace_size(B, window, cfg);
+    if (dws == 0) return 0;
+    const size_t kv = ((size_t)B * cfg->Hkv * cfg->D * dtype_bytes(cfg->dtype) + 15) / 16 * 16;
+    return 2 * kv + dws;
+}
+
+yoco_status yoco_swa_decode_step(const void *x, int32_t d_model, const void *w_kv, int32_t apply_ln,
+                                 float ln_eps, const void *k_base, const void *v_base, float w_k, float w_v,
+                                 const void *q, const int64_t *pos, int32_t B, int32_t window, void *ring_k,
+                                 void *ring_v, int32_t *slot_pos, void *o, void *k_out, void *v_out,
+                                 void *workspace, size_t ws_bytes, const yoco_attn_cfg *cfg,
+                                 cudaStream_t stream) {
+    yoco_status st = check_cfg(cfg);
+    if (st != YOCO_OK) return st;
+    if (B < 0 || window < 1 || d_model < 1 || !(ln_eps > 0.f) || !isfinite(w_k) || !isfinite(w_v))
+        return YOCO_ERR_INVALID;
+    if (B == 0) return YOCO_OK;
+    if (!ok_ptr(x) || !ok_ptr(w_kv) || !ok_ptr(q) || !ok_ptr(pos) || !ok_ptr(ring_k) || !ok_ptr(ring_v) ||
+        !ok_ptr(slot_pos) || !ok_ptr(o) || !ok_opt(k_base) || !ok_opt(v_base) || !ok_opt(k_out) ||
+        !ok_opt(v_out))
+        return YOCO_ERR_INVALID;
+    if ((int64_t)d_model * dtype_bytes(cfg->dtype) % 16 != 0) return YOCO_ERR_INVALID;
+    DecodePlan pl;
+    if (!make_decode_plan(B, window, cfg->Hq, cfg->Hkv, cfg->D, cfg->dtype, &pl)) return YOCO_ERR_UNSUPPORTED;
+    const size_t need = yoco_swa_decode_step_workspace_size(B, window, cfg);
+    if (!workspace || !aligned16(workspace) || need == 0 || ws_bytes < need) return YOCO_ERR_WORKSPACE;
+    // the projection into k_out / v_out (or the workspace), then the window
+    // decode.  bf16 few-token projections stream their weights through
+    // registers and release the decode only after their own wait, so the
+    // decode issues its first window copies while the projection still runs.
+    const size_t kvb = ((size_t)B * cfg->Hkv * cfg->D * dtype_bytes(cfg->dtype) + 15) / 16 * 16;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    void *kn = k_out ? k_out : ws;
+    void *vn = v_out ? v_out : ws + kvb;
+    LinearArgs la;
+    la.x = x; la.w = w_kv; la.n = B; la.d_in = d_model;
+    la.d_out = 2 * cfg->Hkv * cfg->D; la.split_col = cfg->Hkv * cfg->D;
+    la.apply_ln = apply_ln ? 1 : 0; la.eps = ln_eps;
+    la.out0 = kn; la.out1 = vn; la.base0 = k_base; la.base1 = v_base;
+    la.w0 = w_k; la.w1 = w_v; la.dst_rows = nullptr; la.dtype = cfg->dtype;
+    cudaError_t e = launch_linear_few_reg(la, stream);
+    const bool early = e == cudaSuccess;
+    if (e == cudaErrorNotSupported) {
+        cudaGetLastError();
+        st = run_linear(la, stream);
+        if (st != YOCO_OK) return st;
+    } else if (e != cudaSuccess) {
+        return from_cuda(e);
+    }
+    DecodeArgs a;
+    a.q = q; a.k = ring_k; a.v = ring_v; a.seq_start = nullptr; a.seq_len = nullptr;
+    a.slot_pos = slot_pos; a.pos = pos; a.window = window;
+    a.k_new = kn; a.v_new = vn;
+    a.cache_rows = (int64_t)B * window; a.max_len = window;
+    a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
+    a.scale = eff_scale(cfg); a.o = o; a.lse = nullptr; a.ws = ws + 2 * kvb;
+    const cudaError_t e2 = launch_ring_decode(a, stream, early);
+    if (e2 != cudaErrorNotSupported) return from_cuda(e2);
+    cudaGetLastError();
+    return from_cuda(launch_decode(a, pl, stream));
+}
+
 int64_t yoco_kv_i8_row_bytes(const yoco_attn_cfg *cfg) {
     if (!cfg || cfg->Hkv < 1 || (cfg->D != 64 && cfg->D != 128)) return 0;
     return i8_row_bytes(cfg->Hkv, cfg->D);
@@ -430,7 +494,7 @@ yoco_status yoco_get_device_status(cudaStream_t stream) {
     const unsigned int s = read_and_clear_status_decode() | read_and_clear_status_prefill_tc() |
                            read_and_clear_status_prefill_pair() | read_and_clear_status_project_tc() |
                            read_and_clear_status_gret_tc() | read_and_clear_status_linear() |
-                           read_and_clear_status_ring();
+                           read_and_clear_status_ring() | read_and_clear_status_step_proj();
     if (s & 1u) return YOCO_ERR_TIMEOUT;
     if (s & 2u) return YOCO_ERR_INVALID;
     return e == cudaSuccess ? YOCO_OK : YOCO_ERR_CUDA;

@@ -52,8 +52,13 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s);
 // Sliding-window decode step in one clustered launch (bf16, D 64 / 128, group
-// size 1, 2, 4 or 8); cudaErrorNotSupported for any other shape.
-cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t s);
+// size 1, 2, 4 or 8); cudaErrorNotSupported for any other shape.  early: the
+// window's first copies are issued before the programmatic wait, which is
+// correct only when no kernel that may still run when this one starts writes
+// the ring -- the kernel before it on the stream released its dependents
+// after its own wait (launch_linear_few_reg) and writes neither the ring nor
+// slot_pos.
+cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t s, bool early = false);
 
 // Ring fill after a prefill of T tokens.
 cudaError_t launch_ring_fill(const void *k, const void *v, int32_t B, int64_t T, int32_t window,
@@ -98,6 +103,11 @@ struct LinearArgs {
     int32_t dtype;
 };
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
+// Few-token projection with the weight rows streamed through registers (bf16,
+// 1 <= n <= 4, d_in a multiple of 256, d_out a multiple of 16); it releases
+// programmatic dependents only after its own wait.  cudaErrorNotSupported
+// otherwise.
+cudaError_t launch_linear_few_reg(const LinearArgs &a, cudaStream_t s);
 // Tensor-core path (bf16, >= 512 tokens, output width a multiple of 256):
 // LayerNorm folded into the epilogue.  cudaErrorNotSupported otherwise.
 cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
@@ -137,6 +147,7 @@ unsigned int read_and_clear_status_gret_tc();
 unsigned int read_and_clear_status_project_tc();
 unsigned int read_and_clear_status_linear();
 unsigned int read_and_clear_status_ring();
+unsigned int read_and_clear_status_step_proj();
 
 int device_sm_count();
 

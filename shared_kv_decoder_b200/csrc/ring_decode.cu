@@ -39,6 +39,7 @@
 #include <algorithm>
 #include <cstdint>
 
+#include "cluster.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -48,6 +49,8 @@ namespace yoco {
 static __device__ unsigned int g_status_ring;
 
 namespace {
+
+using namespace wmma16;
 
 constexpr int kWarps = 8;                   // consumer warps
 constexpr int kThreads = 32 * (kWarps + 1); // + one producer warp
@@ -67,6 +70,7 @@ struct RingParams {
     int32_t per;       // slots per CTA (a multiple of 16)
     int32_t chunks;    // chunks per CTA
     int32_t stages;    // 1 or 2
+    int32_t early;     // 1: the first stages' copies go out before the programmatic wait
     float scale_log2;
 };
 
@@ -82,51 +86,7 @@ struct RingSmem {
     static size_t bytes(int stages) { return (size_t)stages * STAGE + 64 + FLOATS * sizeof(float) + 1024; }
 };
 
-YOCO_DEV uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-YOCO_DEV uint32_t cluster_size() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-    return r;
-}
-YOCO_DEV void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-YOCO_DEV void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
-YOCO_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
-// The address of the same shared-memory offset in CTA `rank` of the cluster.
-YOCO_DEV uint32_t map_rank(uint32_t local, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-    return r;
-}
-YOCO_DEV void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
 YOCO_DEV void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kWarps) : "memory"); }
-
-YOCO_DEV void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-YOCO_DEV void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-// c += A * B for one m16n8k16 tile whose A rows 8-15 are zero (only the
-// c[0], c[1] halves -- rows 0-7 -- are kept by the callers).
-YOCO_DEV void mma_16816(float *c, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
-}
 
 YOCO_DEV bool wait_bar(uint64_t *bar, uint32_t parity) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, &g_status_ring));
@@ -156,14 +116,15 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
     volatile int *skip = reinterpret_cast<volatile int *>(v_new + D);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const uint32_t rank = cluster_rank(), C = cluster_size();
+    const uint32_t rank = clu::rank(), C = clu::size();
     const int bg = (int)(blockIdx.x / C);
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int s0 = (int)rank * p.per;
     const int s1 = min(p.window, s0 + p.per);
 
+    const int first = min(p.chunks, p.stages);   // chunks whose stages are free at the start
     pdl_trigger();
-    if (threadIdx.x == 32 * kWarps) {
+    if (threadIdx.x == 32 * kWarps && !p.early) {
         // the CTA's K and V boxes into L2 while the previous kernel finishes
         // (a prefetch changes no data, so it may run before the wait)
         for (int c = 0; c < p.chunks; ++c)
@@ -180,12 +141,30 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
         }
         fence_mbar_init();
     }
+    if (p.early) {
+        // early mode: the window's first copies go out while the previous
+        // kernel (the step's projection) still runs.  The launcher allows it
+        // only when no kernel that may still be running writes the ring: the
+        // projection writes only the new K/V, and it released this kernel
+        // after its own wait, so every kernel before it has finished.
+        __syncthreads();   // the barriers are initialised
+        if (threadIdx.x == 32 * kWarps)
+            for (int c = 0; c < first; ++c) {
+                const uint32_t dst = sbase + (uint32_t)c * L::STAGE;
+                mbar_arrive_expect_tx(&full[c], L::STAGE);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    tc::tma_load_4d(dst + kb * kBoxBytes, &tm_k, kb * 64, g, s0 + c * kChunk, b, &full[c]);
+                    tc::tma_load_4d(dst + (KB + kb) * kBoxBytes, &tm_v, kb * 64, g, s0 + c * kChunk, b, &full[c]);
+                }
+            }
+    }
     pdl_wait();
     if (threadIdx.x == 0) *skip = (*(volatile unsigned int *)&g_status_ring) != 0;
     __syncthreads();
     // first cluster phase: every CTA of the cluster is running before any
     // writes into another's shared memory (waited for just before that)
-    cluster_arrive_relaxed();
+    clu::arrive_relaxed();
 
     const int64_t pos_b = p.pos[b];
     const int W = p.window;
@@ -193,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
 
     if (warp == kWarps) {
         // ------------------------------------------------------------ producer
-        uint32_t issued = 0;
+        uint32_t issued = p.early ? (uint32_t)first : 0u;
         auto issue = [&](int c) -> bool {
             const int st = c % p.stages;
             const uint32_t ph = (uint32_t)(c / p.stages) & 1u;
@@ -208,8 +187,7 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
             ++issued;
             return true;
         };
-        const int first = min(p.chunks, p.stages);   // their stages are free: no wait
-        if (lane == 0 && !*skip)
+        if (lane == 0 && !*skip && !p.early)
             for (int c = 0; c < first; ++c) issue(c);
         __syncwarp();
         if (rank == 0) {
@@ -231,8 +209,8 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
             }
             for (int i = lane; i < D; i += 32) v_new[i] = __bfloat162float(p.v_new[((int64_t)b * p.Hkv + g) * D + i]);
         }
-        if (lane == 0 && !*skip) {
-            bool ok = issued == (uint32_t)first;
+        if (lane == 0) {
+            bool ok = !*skip && issued == (uint32_t)first;
             for (int c = first; c < p.chunks && ok; ++c) ok = issue(c);
             // the copies issued must have landed before this CTA's shared
             // memory is reused or released (at once on the normal path)
@@ -240,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
                 if (!mbar_wait(&full[c % p.stages], (c / p.stages) & 1u, &g_status_ring)) break;
         }
         __syncwarp();
-        cluster_wait();
+        clu::wait();
     } else {
         // ----------------------------------------------------------- consumers
         const int gq = lane >> 2;   // fragment row: query head of the group
@@ -294,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(kst + (uint32_t)(kk >> 2) * kBoxBytes + rowS + (((uint32_t)((kk & 3) << 1) ^ xs) << 4),
                         b0, b1, b2, b3);
-                mma_16816(sc[0], qa[kk][0], qa[kk][1], b0, b1);
-                mma_16816(sc[1], qa[kk][0], qa[kk][1], b2, b3);
+                mma_rows8(sc[0], qa[kk][0], qa[kk][1], b0, b1);
+                mma_rows8(sc[1], qa[kk][0], qa[kk][1], b2, b3);
             }
             float pv[2][2];
             float mx = -INFINITY;
@@ -334,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_t(vst + (uint32_t)(n >> 3) * kBoxBytes + rowP + ((((uint32_t)n & 7u) ^ xp) << 4), b0, b1,
                           b2, b3);
-                mma_16816(o[n], a0, a2, b0, b1);
-                mma_16816(o[n + 1], a0, a2, b2, b3);
+                mma_rows8(o[n], a0, a2, b0, b1);
+                mma_rows8(o[n + 1], a0, a2, b2, b3);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
@@ -361,10 +339,10 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
             }
         }
         consumers_sync();
-        cluster_wait();
+        clu::wait();
         // the CTA's partial: the warps' partials under one reference max,
         // stored into slot `rank` of rank 0's gather area
-        const uint32_t dst0 = map_rank(smem_u32(gather), 0) + 4u * (rank * G * PART);
+        const uint32_t dst0 = clu::map_rank(smem_u32(gather), 0) + 4u * (rank * G * PART);
         for (int idx = threadIdx.x; idx < G * D; idx += 32 * kWarps) {
             const int hq = idx / D, d = idx % D;
             float M = -INFINITY;
@@ -378,10 +356,10 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
                 acc = fmaf(src[d], f, acc);
                 Ls = fmaf(src[D + 1], f, Ls);
             }
-            st_cluster_f32(dst0 + 4u * (hq * PART + d), acc);
+            clu::st_f32(dst0 + 4u * (hq * PART + d), acc);
             if (d == 0) {
-                st_cluster_f32(dst0 + 4u * (hq * PART + D), M);
-                st_cluster_f32(dst0 + 4u * (hq * PART + D + 1), Ls);
+                clu::st_f32(dst0 + 4u * (hq * PART + D), M);
+                clu::st_f32(dst0 + 4u * (hq * PART + D + 1), Ls);
             }
         }
     }
@@ -389,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
     // ---------------------------------------------------- cluster merge (rank 0)
     // the barrier's release / acquire makes every rank's stores into the
     // gather area visible here; after it no CTA touches another's memory
-    cluster_sync_all();
+    clu::sync_all();
     if (rank == 0 && warp < kWarps && !*skip) {
         for (int idx = threadIdx.x; idx < G * D; idx += 32 * kWarps) {
             const int hq = idx / D, d = idx % D;
@@ -432,7 +410,7 @@ bool make_ring_map(CUtensorMap *m, const void *ring, int64_t B, int64_t W, int64
 }
 
 template <int D, int G>
-cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st) {
+cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st, bool early) {
     CUtensorMap mk, mv;
     if (!make_ring_map(&mk, a.k, a.B, a.window, a.Hkv, D) || !make_ring_map(&mv, a.v, a.B, a.window, a.Hkv, D))
         return cudaErrorNotSupported;
@@ -448,12 +426,16 @@ cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st) {
     p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.window = a.window;
     p.scale_log2 = a.scale * kLog2e;
     // C CTAs per (sequence, KV head): one 128-slot chunk each up to W = 1024,
-    // then eight CTAs of several chunks
-    const int C = (int)std::min<int64_t>(kMaxCluster, ((int64_t)a.window + kChunk - 1) / kChunk);
+    // then eight CTAs of several chunks.  Early mode takes half as many CTAs,
+    // each with two chunks in flight, so that one of its CTAs fits on an SM
+    // beside one CTA of the projection that runs at the same time.
+    const int cmax = early ? kMaxCluster / 2 : kMaxCluster;
+    const int C = (int)std::min<int64_t>(cmax, ((int64_t)a.window + kChunk - 1) / kChunk);
     const int64_t per = (((int64_t)a.window + C - 1) / C + kWarpTok - 1) / kWarpTok * kWarpTok;
     p.per = (int32_t)per;
     p.chunks = (int32_t)((per + kChunk - 1) / kChunk);
     p.stages = p.chunks > 1 ? 2 : 1;
+    p.early = early ? 1 : 0;
     const int64_t grid = (int64_t)a.B * a.Hkv * C;
     if (grid > INT32_MAX) return cudaErrorNotSupported;
     const size_t smem = RingSmem<D, G>::bytes(p.stages);
@@ -479,22 +461,22 @@ cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st) {
 }
 
 template <int D>
-cudaError_t launch_ring_d(const DecodeArgs &a, cudaStream_t st) {
+cudaError_t launch_ring_d(const DecodeArgs &a, cudaStream_t st, bool early) {
     switch (a.Hq / a.Hkv) {
-        case 1: return launch_ring_dg<D, 1>(a, st);
-        case 2: return launch_ring_dg<D, 2>(a, st);
-        case 4: return launch_ring_dg<D, 4>(a, st);
-        case 8: return launch_ring_dg<D, 8>(a, st);
+        case 1: return launch_ring_dg<D, 1>(a, st, early);
+        case 2: return launch_ring_dg<D, 2>(a, st, early);
+        case 4: return launch_ring_dg<D, 4>(a, st, early);
+        case 8: return launch_ring_dg<D, 8>(a, st, early);
         default: return cudaErrorNotSupported;
     }
 }
 
 }  // namespace
 
-cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t st) {
+cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t st, bool early) {
     if (a.dtype != kBF16 || !a.k_new || !a.pos || !a.slot_pos || a.window < 1) return cudaErrorNotSupported;
-    if (a.D == 128) return launch_ring_d<128>(a, st);
-    if (a.D == 64) return launch_ring_d<64>(a, st);
+    if (a.D == 128) return launch_ring_d<128>(a, st, early);
+    if (a.D == 64) return launch_ring_d<64>(a, st, early);
     return cudaErrorNotSupported;
 }
 
