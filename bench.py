@@ -481,7 +481,10 @@ def early_exit(W, reps):
 def gret_layer(W, reps):
     """The gated-retention self-decoder layer, measured beside the step (it is
     not part of it): the chunkwise prefill over B=4 x T=65536 tokens with 32
-    heads, then one decode step for a batch of 16.  Device ms, mean over reps."""
+    heads (one launch, L2 flushed before it), and the decode step for a batch
+    of 16 as a decode loop runs it: 16 layers of their own states (536 MB, far
+    beyond L2) back to back in a CUDA graph, the time per layer.  Device ms,
+    mean over reps."""
     import torch
     import shared_kv_decoder_b200 as yoco
     import workloads as wl
@@ -491,10 +494,11 @@ def gret_layer(W, reps):
     g = wl.normal((B, T, H), 5004, torch.float32, dev) + 3.0
     o = torch.empty_like(q)
     st = torch.zeros((B, H, D, D), dtype=torch.float32, device=dev)
-    qd, kd, vd = (wl.normal((Bd, H, D), 5011 + i, bf, dev) for i in range(3))
-    gd = wl.normal((Bd, H), 5014, torch.float32, dev) + 3.0
-    sd = torch.zeros((Bd, H, D, D), dtype=torch.float32, device=dev)
-    od = torch.empty_like(qd)
+    Ld = 16
+    qd, kd, vd = ([wl.normal((Bd, H, D), 5011 + 10 * l + i, bf, dev) for l in range(Ld)] for i in range(3))
+    gd = [wl.normal((Bd, H), 5014 + l, torch.float32, dev) + 3.0 for l in range(Ld)]
+    sd = [torch.zeros((Bd, H, D, D), dtype=torch.float32, device=dev) for _ in range(Ld)]
+    od = torch.empty_like(qd[0])
 
     def timed(fn):
         ts = []
@@ -508,7 +512,21 @@ def gret_layer(W, reps):
         return statistics.mean(ts)
 
     t_pre = timed(lambda: yoco.gret_prefill(q, k, v, g, tau, state=st, o=o))
-    t_dec = timed(lambda: yoco.gret_decode(qd, kd, vd, gd, tau, sd, o=od))
+    dec_layers = lambda: [yoco.gret_decode(qd[l], kd[l], vd[l], gd[l], tau, sd[l], o=od) for l in range(Ld)]
+    dec_layers()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dec_layers()
+    tl = []
+    for i in range(reps + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(); graph.replay(); e1.record()
+        torch.cuda.synchronize()
+        if i > 0:
+            tl.append(e0.elapsed_time(e1) / Ld)
+    t_dec = statistics.mean(tl)
+    del graph
     # batch 1: 32 sequences for 148 SMs, so each runs as superchunks on
     # separate CTAs (the workspace the library asks for)
     q1, k1, v1, g1, o1 = q[:1], k[:1], v[:1], g[:1], o[:1]
