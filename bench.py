@@ -112,7 +112,7 @@ TRAFFIC = {
                     "sha256": "836177e0fbe98c89f48dc571b8a23986d590602891340cf2b4ce942e7e583e83"},
     # one decode layer-step at batch 4, window 1024 (yoco_swa_decode_step):
     # linear_few_reg_kernel (the 4-token projection) 16.851 MB read +
-    # ring_decode_cluster_kernel<128, 4> (early copies, 4 CTAs a head) 16.891 MB read
+    # ring_decode_cluster_kernel<128, 4> (4 CTAs a head) 16.891 MB read
     "swa_decode": {"bytes": 16850688 + 16891392,
                    "sources": ['ring_decode.cu', 'step_proj.cu', 'cluster.cuh', 'tc.cuh', 'common.cuh'],
                    "sha256": "73e3c1455a92d30dd6cd3735e630680c7f7d3bb6904f751b2d3f2f8ac4f65aa8"},
@@ -1247,9 +1247,8 @@ def measure(args, world, rank, local, dev):
                 "decode_bytes_per_layer_step": layer_step_bytes,
                 "note": "attention times include the ring fill; decode = 256 steps x 16 layers from one "
                         "CUDA graph, each layer-step = one yoco_swa_decode_step call: the 4 new tokens' "
-                        "projection with the blend, and the clustered window decode (window attention, "
-                        "merge with the new token, ring write) whose first window copies go out while "
-                        "the projection runs"},
+                        "projection with the blend, then the clustered window decode (window attention, "
+                        "merge with the new token, ring write)"},
         "gkv": {"ms": statistics.mean(gkv_ms), "tflops": gkv_fl / (statistics.mean(gkv_ms) * 1e-3) / 1e12},
         "roofline": {"kernel": "cross prefill (yoco_cross_prefill)", "bound": "tensor",
                      "achieved": pre_tflops_launch, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",

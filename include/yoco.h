@@ -125,8 +125,9 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
  * (n_tok = B, no dst_rows) followed by yoco_swa_decode with the projected
  * K/V -- the YOCO++ blended K/V producer (YOCO++ Abstract) and the section 3
  * "Sliding-Window Attention" decode -- with the same results.  Two launches;
- * for bf16 with B <= 4 and d_model a multiple of 256 the window's first
- * copies are already in flight while the projection runs.
+ * for bf16 with B <= 4 and d_model a multiple of 256 the projection streams
+ * its weights through registers and the window decode takes its compact
+ * layout.
  * x [B, d_model]; w_kv [2 Hkv D, d_model]; k_base, v_base [B, Hkv, D] or
  * NULL (then w_k / w_v are ignored); q [B, Hq, D]; pos device int64 [B];
  * ring_k, ring_v [B, window, Hkv, D]; slot_pos int32 [B, window]; o [B, Hq, D].

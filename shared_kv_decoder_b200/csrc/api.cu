@@ -286,8 +286,8 @@ yoco_status yoco_swa_decode_step(const void *x, int32_t d_model, const void *w_k
     if (!workspace || !aligned16(workspace) || need == 0 || ws_bytes < need) return YOCO_ERR_WORKSPACE;
     // the projection into k_out / v_out (or the workspace), then the window
     // decode.  bf16 few-token projections stream their weights through
-    // registers and release the decode only after their own wait, so the
-    // decode issues its first window copies while the projection still runs.
+    // registers; after that kernel the window decode runs in its compact
+    // layout (four CTAs a head), the faster one there.
     const size_t kvb = ((size_t)B * cfg->Hkv * cfg->D * dtype_bytes(cfg->dtype) + 15) / 16 * 16;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     void *kn = k_out ? k_out : ws;
@@ -299,7 +299,7 @@ yoco_status yoco_swa_decode_step(const void *x, int32_t d_model, const void *w_k
     la.out0 = kn; la.out1 = vn; la.base0 = k_base; la.base1 = v_base;
     la.w0 = w_k; la.w1 = w_v; la.dst_rows = nullptr; la.dtype = cfg->dtype;
     cudaError_t e = launch_linear_few_reg(la, stream);
-    const bool early = e == cudaSuccess;
+    const bool compact = e == cudaSuccess;
     if (e == cudaErrorNotSupported) {
         cudaGetLastError();
         st = run_linear(la, stream);
@@ -314,7 +314,7 @@ yoco_status yoco_swa_decode_step(const void *x, int32_t d_model, const void *w_k
     a.cache_rows = (int64_t)B * window; a.max_len = window;
     a.B = B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.dtype = cfg->dtype;
     a.scale = eff_scale(cfg); a.o = o; a.lse = nullptr; a.ws = ws + 2 * kvb;
-    const cudaError_t e2 = launch_ring_decode(a, stream, early);
+    const cudaError_t e2 = launch_ring_decode(a, stream, compact);
     if (e2 != cudaErrorNotSupported) return from_cuda(e2);
     cudaGetLastError();
     return from_cuda(launch_decode(a, pl, stream));

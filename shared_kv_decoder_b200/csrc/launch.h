@@ -52,13 +52,10 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s);
 // Sliding-window decode step in one clustered launch (bf16, D 64 / 128, group
-// size 1, 2, 4 or 8); cudaErrorNotSupported for any other shape.  early: the
-// window's first copies are issued before the programmatic wait, which is
-// correct only when no kernel that may still run when this one starts writes
-// the ring -- the kernel before it on the stream released its dependents
-// after its own wait (launch_linear_few_reg) and writes neither the ring nor
-// slot_pos.
-cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t s, bool early = false);
+// size 1, 2, 4 or 8); cudaErrorNotSupported for any other shape.  compact: at
+// most four CTAs per (sequence, KV head) instead of eight, each with two
+// window chunks in flight (faster after launch_linear_few_reg).
+cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t s, bool compact = false);
 
 // Ring fill after a prefill of T tokens.
 cudaError_t launch_ring_fill(const void *k, const void *v, int32_t B, int64_t T, int32_t window,
@@ -104,9 +101,8 @@ struct LinearArgs {
 };
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
 // Few-token projection with the weight rows streamed through registers (bf16,
-// 1 <= n <= 4, d_in a multiple of 256, d_out a multiple of 16); it releases
-// programmatic dependents only after its own wait.  cudaErrorNotSupported
-// otherwise.
+// 1 <= n <= 4, d_in a multiple of 256, d_out a multiple of 16).
+// cudaErrorNotSupported otherwise.
 cudaError_t launch_linear_few_reg(const LinearArgs &a, cudaStream_t s);
 // Tensor-core path (bf16, >= 512 tokens, output width a multiple of 256):
 // LayerNorm folded into the epilogue.  cudaErrorNotSupported otherwise.

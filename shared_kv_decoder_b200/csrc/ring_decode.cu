@@ -70,7 +70,6 @@ struct RingParams {
     int32_t per;       // slots per CTA (a multiple of 16)
     int32_t chunks;    // chunks per CTA
     int32_t stages;    // 1 or 2
-    int32_t early;     // 1: the first stages' copies go out before the programmatic wait
     float scale_log2;
 };
 
@@ -122,9 +121,8 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
     const int s0 = (int)rank * p.per;
     const int s1 = min(p.window, s0 + p.per);
 
-    const int first = min(p.chunks, p.stages);   // chunks whose stages are free at the start
     pdl_trigger();
-    if (threadIdx.x == 32 * kWarps && !p.early) {
+    if (threadIdx.x == 32 * kWarps) {
         // the CTA's K and V boxes into L2 while the previous kernel finishes
         // (a prefetch changes no data, so it may run before the wait)
         for (int c = 0; c < p.chunks; ++c)
@@ -141,24 +139,6 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
         }
         fence_mbar_init();
     }
-    if (p.early) {
-        // early mode: the window's first copies go out while the previous
-        // kernel (the step's projection) still runs.  The launcher allows it
-        // only when no kernel that may still be running writes the ring: the
-        // projection writes only the new K/V, and it released this kernel
-        // after its own wait, so every kernel before it has finished.
-        __syncthreads();   // the barriers are initialised
-        if (threadIdx.x == 32 * kWarps)
-            for (int c = 0; c < first; ++c) {
-                const uint32_t dst = sbase + (uint32_t)c * L::STAGE;
-                mbar_arrive_expect_tx(&full[c], L::STAGE);
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    tc::tma_load_4d(dst + kb * kBoxBytes, &tm_k, kb * 64, g, s0 + c * kChunk, b, &full[c]);
-                    tc::tma_load_4d(dst + (KB + kb) * kBoxBytes, &tm_v, kb * 64, g, s0 + c * kChunk, b, &full[c]);
-                }
-            }
-    }
     pdl_wait();
     if (threadIdx.x == 0) *skip = (*(volatile unsigned int *)&g_status_ring) != 0;
     __syncthreads();
@@ -172,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
 
     if (warp == kWarps) {
         // ------------------------------------------------------------ producer
-        uint32_t issued = p.early ? (uint32_t)first : 0u;
+        uint32_t issued = 0;
         auto issue = [&](int c) -> bool {
             const int st = c % p.stages;
             const uint32_t ph = (uint32_t)(c / p.stages) & 1u;
@@ -187,7 +167,8 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
             ++issued;
             return true;
         };
-        if (lane == 0 && !*skip && !p.early)
+        const int first = min(p.chunks, p.stages);   // their stages are free: no wait
+        if (lane == 0 && !*skip)
             for (int c = 0; c < first; ++c) issue(c);
         __syncwarp();
         if (rank == 0) {
@@ -209,8 +190,8 @@ __global__ void __launch_bounds__(kThreads, 2) ring_decode_cluster_kernel(const 
             }
             for (int i = lane; i < D; i += 32) v_new[i] = __bfloat162float(p.v_new[((int64_t)b * p.Hkv + g) * D + i]);
         }
-        if (lane == 0) {
-            bool ok = !*skip && issued == (uint32_t)first;
+        if (lane == 0 && !*skip) {
+            bool ok = issued == (uint32_t)first;
             for (int c = first; c < p.chunks && ok; ++c) ok = issue(c);
             // the copies issued must have landed before this CTA's shared
             // memory is reused or released (at once on the normal path)
@@ -410,7 +391,7 @@ bool make_ring_map(CUtensorMap *m, const void *ring, int64_t B, int64_t W, int64
 }
 
 template <int D, int G>
-cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st, bool early) {
+cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st, bool compact) {
     CUtensorMap mk, mv;
     if (!make_ring_map(&mk, a.k, a.B, a.window, a.Hkv, D) || !make_ring_map(&mv, a.v, a.B, a.window, a.Hkv, D))
         return cudaErrorNotSupported;
@@ -426,16 +407,14 @@ cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st, bool early) {
     p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.window = a.window;
     p.scale_log2 = a.scale * kLog2e;
     // C CTAs per (sequence, KV head): one 128-slot chunk each up to W = 1024,
-    // then eight CTAs of several chunks.  Early mode takes half as many CTAs,
-    // each with two chunks in flight, so that one of its CTAs fits on an SM
-    // beside one CTA of the projection that runs at the same time.
-    const int cmax = early ? kMaxCluster / 2 : kMaxCluster;
+    // then eight CTAs of several chunks.  The compact layout takes at most
+    // four CTAs, each with two chunks in flight (one CTA an SM at W = 1024).
+    const int cmax = compact ? kMaxCluster / 2 : kMaxCluster;
     const int C = (int)std::min<int64_t>(cmax, ((int64_t)a.window + kChunk - 1) / kChunk);
     const int64_t per = (((int64_t)a.window + C - 1) / C + kWarpTok - 1) / kWarpTok * kWarpTok;
     p.per = (int32_t)per;
     p.chunks = (int32_t)((per + kChunk - 1) / kChunk);
     p.stages = p.chunks > 1 ? 2 : 1;
-    p.early = early ? 1 : 0;
     const int64_t grid = (int64_t)a.B * a.Hkv * C;
     if (grid > INT32_MAX) return cudaErrorNotSupported;
     const size_t smem = RingSmem<D, G>::bytes(p.stages);
@@ -461,22 +440,22 @@ cudaError_t launch_ring_dg(const DecodeArgs &a, cudaStream_t st, bool early) {
 }
 
 template <int D>
-cudaError_t launch_ring_d(const DecodeArgs &a, cudaStream_t st, bool early) {
+cudaError_t launch_ring_d(const DecodeArgs &a, cudaStream_t st, bool compact) {
     switch (a.Hq / a.Hkv) {
-        case 1: return launch_ring_dg<D, 1>(a, st, early);
-        case 2: return launch_ring_dg<D, 2>(a, st, early);
-        case 4: return launch_ring_dg<D, 4>(a, st, early);
-        case 8: return launch_ring_dg<D, 8>(a, st, early);
+        case 1: return launch_ring_dg<D, 1>(a, st, compact);
+        case 2: return launch_ring_dg<D, 2>(a, st, compact);
+        case 4: return launch_ring_dg<D, 4>(a, st, compact);
+        case 8: return launch_ring_dg<D, 8>(a, st, compact);
         default: return cudaErrorNotSupported;
     }
 }
 
 }  // namespace
 
-cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t st, bool early) {
+cudaError_t launch_ring_decode(const DecodeArgs &a, cudaStream_t st, bool compact) {
     if (a.dtype != kBF16 || !a.k_new || !a.pos || !a.slot_pos || a.window < 1) return cudaErrorNotSupported;
-    if (a.D == 128) return launch_ring_d<128>(a, st, early);
-    if (a.D == 64) return launch_ring_d<64>(a, st, early);
+    if (a.D == 128) return launch_ring_d<128>(a, st, compact);
+    if (a.D == 64) return launch_ring_d<64>(a, st, compact);
     return cudaErrorNotSupported;
 }
 

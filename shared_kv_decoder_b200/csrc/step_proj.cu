@@ -7,26 +7,23 @@
 // (podcast transcript "YOCO: Caching Once ...", cue 12; YOCO++ Abstract), the
 // same result as the other projection kernels of linear.cu.
 //
-// Built to run beside the sliding-window decode that follows it: a CTA takes
-// 16 output columns (one m16 tile of weight rows, 128 KB at d_in = 4096) and
-// holds no weights in shared memory -- its eight warps each load their
-// d_in / 8 columns of the 16 rows as 16-byte register loads, twelve 32-column
-// blocks in flight at a time, and multiply them with the n token rows on the
-// tensor cores (the MMA's N columns: tokens 0..n-1, and a column of ones at 7
-// whose products are the rows' weight sums, for the folded LayerNorm).  The
-// token rows are bulk-copied into shared memory; the warps also add up their
-// columns' share of each row's LayerNorm sums.  A CTA takes ~40 KB of shared
-// memory and 140 registers a thread (256 threads): two of them do not fit on
-// an SM, one of them and one CTA of the window decode (96 x 288 registers)
-// do, so the decode's CTAs start -- and issue their first copies -- while
-// this kernel runs.  Measured in CUDA graphs of 4096 layer-steps (4 x 4096 ->
-// 2048, window 1024): 15.3 us a layer-step, against 16.6 with two of these
-// CTAs an SM and 16.5 for linear.cu's projection followed by the decode.
+// A CTA takes 16 output columns (one m16 tile of weight rows, 128 KB at
+// d_in = 4096) and holds no weights in shared memory: its eight warps each
+// load their d_in / 8 columns of the 16 rows as 16-byte register loads,
+// twelve 32-column blocks in flight at a time, and multiply them with the n
+// token rows on the tensor cores (the MMA's N columns: tokens 0..n-1, and a
+// column of ones at 7 whose products are the rows' weight sums, for the folded
+// LayerNorm).  The token rows are bulk-copied into shared memory; the warps
+// also add up their columns' share of each row's LayerNorm sums.  A CTA takes
+// ~37 KB of shared memory and 140 registers a thread (256 threads, one CTA an
+// SM).  Measured in CUDA graphs of 4096 layer-steps (4 x 4096 -> 2048, then
+// the window decode over a 4 x 1024 ring): 15.2 us a layer-step, against 16.2
+// with 126 registers (two CTAs an SM) and 16.6 for linear.cu's few-row
+// projection followed by the decode.
 //
 // Programmatic launch: the weight rows and the token rows are prefetched into
-// L2 before the wait (a prefetch changes no data), and dependents are released
-// only after the wait, so a kernel that starts early after this one may read,
-// before its own wait, anything that every kernel before this one wrote.
+// L2 before the wait (a prefetch changes no data).
+
 #include <algorithm>
 
 #include "common.cuh"
