@@ -112,10 +112,10 @@ TRAFFIC = {
                     "sha256": "836177e0fbe98c89f48dc571b8a23986d590602891340cf2b4ce942e7e583e83"},
     # one decode layer-step at batch 4, window 1024 (yoco_swa_decode_step):
     # linear_few_reg_kernel (the 4-token projection) 16.851 MB read +
-    # ring_decode_cluster_kernel<128, 4> (4 CTAs a head) 16.891 MB read
-    "swa_decode": {"bytes": 16850688 + 16891392,
+    # ring_decode_cluster_kernel<128, 4> (4 CTAs a head) 16.888 MB read
+    "swa_decode": {"bytes": 16850944 + 16887552,
                    "sources": ['ring_decode.cu', 'step_proj.cu', 'cluster.cuh', 'tc.cuh', 'common.cuh'],
-                   "sha256": "73e3c1455a92d30dd6cd3735e630680c7f7d3bb6904f751b2d3f2f8ac4f65aa8"},
+                   "sha256": "61e72110b05ff916ecc8e7d733bf5a6f34f768927e4ea845cd76263f8ff1f9dc"},
     # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416165 GB read + 25.238 MB written
     "decode": {"bytes": 6416165120 + 25238272,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],
