@@ -143,6 +143,41 @@ def test_i8_cache_arguments_rejected_before_launch():
     assert L.yoco_kv_quantize_i8(FAKE, FAKE, 0, None, FAKE, FAKE, b, None) == yoco.OK
 
 
+def test_swa_decode_step_arguments_rejected_before_launch():
+    L = yoco.load()
+    c = _cfg()
+    b = ctypes.byref(c)
+    B, W, d = 4, 1024, 4096
+    need = L.yoco_swa_decode_step_workspace_size(B, W, b)
+    # the decode workspace plus the new K/V scratch of the fallback path
+    assert need == L.yoco_swa_decode_workspace_size(B, W, b) + 2 * B * 8 * 128 * 2
+    assert L.yoco_swa_decode_step_workspace_size(B, 0, b) == 0
+    assert L.yoco_swa_decode_step_workspace_size(-1, W, b) == 0
+
+    def call(x=FAKE, dm=d, w=FAKE, eps=1e-5, wk=0.5, q=FAKE, pos=FAKE, nb=B, win=W, o=FAKE, ko=None, ws=FAKE,
+             wsb=None):
+        return L.yoco_swa_decode_step(x, dm, w, 1, eps, FAKE, FAKE, wk, 0.5, q, pos, nb, win, FAKE, FAKE, FAKE,
+                                      o, ko, None, ws, need if wsb is None else wsb, b, None)
+    assert call(nb=-1) == yoco.ERR_INVALID
+    assert call(win=0) == yoco.ERR_INVALID
+    assert call(dm=0) == yoco.ERR_INVALID
+    assert call(dm=100) == yoco.ERR_INVALID              # x rows not a multiple of 16 bytes
+    assert call(eps=0.0) == yoco.ERR_INVALID
+    assert call(wk=float("nan")) == yoco.ERR_INVALID
+    assert call(x=None) == yoco.ERR_INVALID
+    assert call(pos=None) == yoco.ERR_INVALID
+    assert call(o=MISALIGNED) == yoco.ERR_INVALID
+    assert call(ko=MISALIGNED) == yoco.ERR_INVALID        # optional outputs must still be aligned
+    assert call(ws=None) == yoco.ERR_WORKSPACE
+    assert call(wsb=need - 16) == yoco.ERR_WORKSPACE
+    assert call(ws=MISALIGNED) == yoco.ERR_WORKSPACE
+    assert L.yoco_swa_decode_step(FAKE, d, FAKE, 1, 1e-5, None, None, 0.0, 0.0, FAKE, FAKE, B, W, FAKE, FAKE,
+                                  FAKE, FAKE, None, None, FAKE, need, ctypes.byref(_cfg(D=96)),
+                                  None) == yoco.ERR_UNSUPPORTED
+    # an empty batch is a successful no-op (nothing launched)
+    assert call(nb=0) == yoco.OK
+
+
 def test_workspace_size_monotone_and_positive():
     sizes = [yoco.cross_decode_workspace_size(B, L, 32, 8, 128, torch.bfloat16)
              for B, L in [(1, 1), (1, 4096), (16, 131072), (16, 262144)]]
