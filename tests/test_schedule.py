@@ -130,6 +130,30 @@ def test_decode_plan_partitions_sequences(lens, max_len, Hq, Hkv, D, n_cta):
         assert max(per_cta_units.values()) - min(per_cta_units.values()) <= 1
 
 
+@pytest.mark.parametrize("lens,max_len,max_units", [
+    ([1 << 20], 1 << 20, 296),                       # one 1M-token sequence: two units an SM at most
+    ([32768], 32768, 296),                           # one 32K sequence: ~2 MB units
+    ([65536 + 4096 * i for i in range(16)], 131072, 1776),   # 16 long sequences: the call's maximum
+])
+def test_decode_plan_unit_counts(lens, max_len, max_units):
+    # a sequence gets at most 296 units (its merge folds them in one CTA per
+    # query head) and a call at most 12 per SM; the 1M-token sequence's split
+    # is set by that cap (14 MB units), the others' by the call's unit count
+    starts = np.cumsum([0] + lens[:-1])
+    rec = yoco.debug_tile_schedule(yoco.SCHEDULE_DECODE, 32, 8, 128, B=len(lens), seq_start=starts,
+                                   seq_len=lens, max_len=max_len, n_cta=148)
+    per_seq = np.bincount(rec[:, 1], minlength=len(lens))
+    assert per_seq.max() <= 296
+    assert len(rec) <= max_units
+    tok_bytes = 2 * 8 * 128 * 2
+    split = int(rec[0, 4])
+    if len(lens) == 1 and lens[0] == (1 << 20):
+        assert per_seq[0] == 296 or per_seq[0] == -(-lens[0] // split)
+        assert split * tok_bytes > (2 << 20)          # the cap, not the 2 MB target, sets the split
+    else:
+        assert split * tok_bytes < 5 * (1 << 20)
+
+
 def test_schedule_rejects_bad_arguments():
     with pytest.raises(yoco.YocoError):
         _prefill(1, 4, 2, 100, 50, 0, 0, 4)      # q_pos0 + Tq > Tkv
