@@ -115,7 +115,7 @@ TRAFFIC = {
     # ring_decode_cluster_kernel<128, 4> (4 CTAs a head) 16.888 MB read
     "swa_decode": {"bytes": 16850944 + 16887552,
                    "sources": ['ring_decode.cu', 'step_proj.cu', 'cluster.cuh', 'tc.cuh', 'common.cuh'],
-                   "sha256": "61e72110b05ff916ecc8e7d733bf5a6f34f768927e4ea845cd76263f8ff1f9dc"},
+                   "sha256": "1ba3719db7da2734bf0f878d3b4de9b199d3706259aeb3eea7ef611026e8bfea"},
     # decode_tma_kernel<128, 4>, batch 16 at 64K-128K: 6.416165 GB read + 25.238 MB written
     "decode": {"bytes": 6416165120 + 25238272,
                "sources": ["decode.cu", "schedule.h", "tc.cuh", "common.cuh"],

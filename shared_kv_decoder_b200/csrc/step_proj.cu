@@ -17,9 +17,9 @@
 // also add up their columns' share of each row's LayerNorm sums.  A CTA takes
 // ~37 KB of shared memory and 140 registers a thread (256 threads, one CTA an
 // SM).  Measured in CUDA graphs of 4096 layer-steps (4 x 4096 -> 2048, then
-// the window decode over a 4 x 1024 ring): 15.2 us a layer-step, against 16.2
-// with 126 registers (two CTAs an SM) and 16.6 for linear.cu's few-row
-// projection followed by the decode.
+// the window decode over a 4 x 1024 ring): 15.2 us a layer-step, against
+// 16.2-16.6 with 126 registers (two CTAs an SM) and 16.6 for linear.cu's
+// few-row projection followed by the decode.
 //
 // Programmatic launch: the weight rows and the token rows are prefetched into
 // L2 before the wait (a prefetch changes no data).
