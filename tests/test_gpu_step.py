@@ -26,6 +26,7 @@ def _bf16_round(a):
     (3, 16, 2, 128, 129, 100, 2048, 2, True, True),     # ring not yet full; group 8
     (4, 8, 8, 128, 64, 200, 512, 2, False, True),       # group 1, no LayerNorm
     (2, 4, 2, 128, 16, 40, 1024, 3, True, True),        # window 16
+    (2, 8, 2, 128, 2100, 2200, 1024, 2, True, True),    # five 128-slot chunks a CTA on two stages, the last one short
     (2, 8, 4, 64, 100, 150, 1024, 2, True, True),       # head_dim 64
     (5, 8, 2, 128, 100, 150, 1024, 2, True, True),      # five tokens: the other projection kernels, plain window copies
     (2, 8, 2, 128, 100, 150, 320, 2, True, True),       # d_model 320: the other projection kernels
