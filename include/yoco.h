@@ -135,7 +135,13 @@ yoco_status yoco_swa_decode(const void *q, const void *k_new, const void *v_new,
  * (what yoco_kv_project_blend would write; a bottom layer's output is the
  * base of the layers above it); with NULL the workspace holds them.  The new
  * K/V is rounded to the cache dtype before it is attended to and stored.
- * workspace: yoco_swa_decode_step_workspace_size() bytes. */
+ * workspace: yoco_swa_decode_step_workspace_size() bytes.
+ * Errors (before any launch): YOCO_ERR_INVALID for B < 0, window < 1,
+ * d_model < 1 or rows of d_model elements not a multiple of 16 bytes,
+ * ln_eps <= 0, non-finite w_k / w_v, a null required pointer or any
+ * pointer not 16-byte aligned; YOCO_ERR_UNSUPPORTED for a head shape no
+ * decode is built for; YOCO_ERR_WORKSPACE for a null, misaligned or short
+ * workspace.  B = 0 launches nothing and returns YOCO_OK. */
 yoco_status yoco_swa_decode_step(const void *x, int32_t d_model, const void *w_kv, int32_t apply_ln,
                                  float ln_eps, const void *k_base, const void *v_base, float w_k, float w_v,
                                  const void *q, const int64_t *pos, int32_t B, int32_t window, void *ring_k,
